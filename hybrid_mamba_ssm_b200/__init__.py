@@ -1,0 +1,25 @@
+"""B200-native Mamba-2 selective state-space scan.
+
+Two entry points, both hand-written CUDA for sm_100a behind the C ABI declared
+in ``include/ssm.h`` (library ``libssm.so``):
+
+* ``ssd_chunk_scan``   -- chunked SSD prefill over packed sequences, returning
+  y and the final fp32 state;
+* ``ssm_state_update`` -- single-token decode update, in place on an fp32
+  ``[batch, heads, head_dim, d_state]`` state.
+
+The Python binding (``hybrid_mamba_ssm_b200.ssm``) only marshals torch tensors
+into that ABI; importing it loads the CUDA library and raises if it is missing.
+``hybrid_mamba_ssm_b200.inputs`` (seeded synthetic inputs) needs neither torch
+nor the library.
+"""
+
+__all__ = ["ssd_chunk_scan", "ssm_state_update", "ssd_chunk_scan_workspace_size",
+           "SSMError"]
+
+
+def __getattr__(name):
+    if name in __all__:
+        from . import ssm
+        return getattr(ssm, name)
+    raise AttributeError(name)

@@ -1,0 +1,160 @@
+"""fp64 CPU oracle of the Mamba-2 selective state-space recurrence.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg use it; the product path never does.  It shares
+no code with the CUDA library and does not import the ``hybrid_mamba_ssm_b200``
+package.
+
+The arithmetic lives in ``ssm_oracle.c`` (plain sequential C, double
+precision, OpenMP over (sequence, head)).  This module compiles it with gcc,
+loads it with ctypes and only marshals numpy arrays to and from it.
+
+Source of the definition: the selective-SSM recurrence of the note
+"Mamba 与 Nemotron 系列模型深度调研" (section "1. Selective SSM 的直觉"),
+restated for decode in the modeling_nemotron_h.py walk-through (section
+"Decode 阶段").  Per token t, head h, group g = h // (H // G):
+``h <- exp(dt*A_h) * h + dt * x (outer) B`` and ``y = h . C + D_h * x``, the
+output reading the updated state.
+
+Every function here is pinned by tests/test_oracle.py against results that do
+not come from this code: a brute-force evaluation of the structured
+semiseparable (SSD) matrix form, closed forms for dt = 0, A = 0, d_state = 1
+and time-invariant inputs, split-and-carry, and linearity.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssm_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libssm_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False) -> str:
+    """Compile ssm_oracle.c into oracle/libssm_oracle.so (gcc -O2 -fopenmp)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+           "-o", tmp, _SRC, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            lib.oracle_scan.restype = ctypes.c_int
+            lib.oracle_scan.argtypes = [
+                ctypes.c_int, _i64p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
+            lib.oracle_state_update.restype = ctypes.c_int
+            lib.oracle_state_update.argtypes = [
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
+            lib.oracle_num_threads.restype = ctypes.c_int
+            lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses."""
+    return _load().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    _load().oracle_set_num_threads(int(n))
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_dp)
+
+
+def scan(x, dt, A, B, C, D=None, h0=None, cu_seqlens=None):
+    """Sequential recurrence over (possibly packed) sequences, in fp64.
+
+    x  : [T, H, P] or [nseq, L, H, P]
+    dt : [T, H]    or [nseq, L, H]
+    A  : [H]
+    B, C : [T, G, N] or [nseq, L, G, N]
+    D  : [H] or None (zero skip term)
+    h0 : [nseq, H, P, N] or None (zero initial state)
+    cu_seqlens : [nseq+1] offsets for packed input, or None (then x is either
+        [nseq, L, H, P], or [T, H, P] holding one sequence).
+
+    Returns (y, h_final): y shaped like x, h_final [nseq, H, P, N], both fp64.
+    """
+    x = _f64(x)
+    batched = x.ndim == 4
+    if batched:
+        nseq, L, H, P = x.shape
+        T = nseq * L
+        cu = np.arange(nseq + 1, dtype=np.int64) * L
+    else:
+        T, H, P = x.shape
+        if cu_seqlens is None:
+            cu = np.array([0, T], dtype=np.int64)
+        else:
+            cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+        nseq = cu.shape[0] - 1
+    B64, C64 = _f64(B), _f64(C)
+    G, N = B64.shape[-2], B64.shape[-1]
+    Bf = B64.reshape(T, G, N)
+    Cf = C64.reshape(T, G, N)
+    dtf = _f64(dt).reshape(T, H)
+    Af = _f64(A).reshape(H)
+    Df = None if D is None else _f64(D).reshape(H)
+    xf = x.reshape(T, H, P)
+    if h0 is None:
+        state = np.zeros((nseq, H, P, N), dtype=np.float64)
+    else:
+        state = _f64(h0).reshape(nseq, H, P, N).copy()
+    y = np.zeros((T, H, P), dtype=np.float64)
+    rc = _load().oracle_scan(int(nseq), cu.ctypes.data_as(_i64p), H, P, N, G,
+                             _ptr(xf), _ptr(dtf), _ptr(Af), _ptr(Bf), _ptr(Cf),
+                             _ptr(Df), _ptr(state), _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle_scan rejected its arguments (status {rc})")
+    return y.reshape(x.shape), state
+
+
+def state_update(state, x, dt, A, B, C, D=None):
+    """One decode step of the recurrence for a batch, in fp64.
+
+    state : [batch, H, P, N]  (not modified; the updated copy is returned)
+    x : [batch, H, P]   dt : [batch, H]   A : [H]   B, C : [batch, G, N]
+    Returns (y [batch, H, P], new_state [batch, H, P, N]).
+    """
+    st = _f64(state).copy()
+    batch, H, P, N = st.shape
+    xf, dtf, Af = _f64(x), _f64(dt), _f64(A)
+    Bf, Cf = _f64(B), _f64(C)
+    G = Bf.shape[1]
+    Df = None if D is None else _f64(D)
+    y = np.zeros((batch, H, P), dtype=np.float64)
+    rc = _load().oracle_state_update(batch, H, P, N, G, _ptr(st), _ptr(xf),
+                                     _ptr(dtf), _ptr(Af), _ptr(Bf), _ptr(Cf),
+                                     _ptr(Df), _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle_state_update rejected its arguments ({rc})")
+    return y, st

@@ -1,0 +1,164 @@
+/*
+ * ssm_oracle.c -- plain, slow fp64 CPU reference of the Mamba-2 selective
+ * state-space recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA path.
+ *
+ * What it computes (the selective-SSM recurrence as stated in the note
+ * "Mamba 与 Nemotron 系列模型深度调研", section "1. Selective SSM 的直觉",
+ * and restated for the decode path in "逐行精读 ... modeling_nemotron_h.py",
+ * section "Decode 阶段"):
+ *
+ *     h[p,n] <- exp(dt_t * A_h) * h[p,n] + dt_t * x_t[h,p] * B_t[g,n]
+ *     y_t[h,p] = sum over n of h[p,n] * C_t[g,n]  +  D_h * x_t[h,p]
+ *
+ * per token t, per head h, for every (p, n) element of the [head_dim, d_state]
+ * state, where A, D are per-head scalars, dt is per (token, head), x is per
+ * (token, head, p) and B, C are per (token, group, n), the group of head h
+ * being g(h) = h / (nheads / ngroups).  The output reads the UPDATED state.
+ *
+ * The prefill ("chunked SSD scan") reaches exactly this result in exact
+ * arithmetic, so the oracle is the plain sequential definition: one token at a
+ * time, in order, for every (sequence, head).  There is no chunking, blocking
+ * or reordering here.  Everything is double precision; inputs arrive already
+ * widened to double (bf16 and fp32 values convert exactly).
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Status codes of this library (independent of the CUDA library's). */
+enum { ORACLE_OK = 0, ORACLE_BAD_ARG = 1 };
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/*
+ * One token of the recurrence for one head.
+ *   h    [P*N]  state of this (sequence, head), updated in place
+ *   xv   [P]    x of this token and head
+ *   bv   [N]    B of this token, in the head's group
+ *   cv   [N]    C of this token, in the head's group
+ *   yv   [P]    output of this token and head
+ */
+static void recurrence_step(int P, int N, double dt, double A, double D,
+                            const double *xv, const double *bv,
+                            const double *cv, double *h, double *yv)
+{
+    const double decay = exp(A * dt);
+    for (int p = 0; p < P; ++p) {
+        double *row = h + (size_t)p * N;
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n) {
+            row[n] = row[n] * decay + bv[n] * dt * xv[p];
+            acc += row[n] * cv[n];
+        }
+        yv[p] = acc + D * xv[p];
+    }
+}
+
+/*
+ * Sequential scan over packed sequences.
+ *
+ *   nseq          number of sequences
+ *   cu_seqlens    [nseq+1] token offsets (cu[0] = 0, non-decreasing)
+ *   H, P, N, G    heads, head_dim, d_state, groups (H % G == 0)
+ *   x   [T,H,P]   dt [T,H]   A [H]   B [T,G,N]   C [T,G,N]   D [H] or NULL
+ *   state [nseq,H,P,N]  in: initial state, out: final state
+ *   y   [T,H,P]   output
+ *
+ * Returns ORACLE_OK or ORACLE_BAD_ARG.
+ */
+int oracle_scan(int nseq, const int64_t *cu_seqlens, int H, int P, int N, int G,
+                const double *x, const double *dt, const double *A,
+                const double *B, const double *C, const double *D,
+                double *state, double *y)
+{
+    if (nseq < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0)
+        return ORACLE_BAD_ARG;
+    if (nseq == 0) return ORACLE_OK;
+    if (!cu_seqlens || !A || !state) return ORACLE_BAD_ARG;
+    if (cu_seqlens[0] != 0) return ORACLE_BAD_ARG;
+    for (int s = 0; s < nseq; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return ORACLE_BAD_ARG;
+    if (cu_seqlens[nseq] > 0 && (!x || !dt || !B || !C || !y))
+        return ORACLE_BAD_ARG;
+
+    const int heads_per_group = H / G;
+    const long work = (long)nseq * H;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long w = 0; w < work; ++w) {
+        const int s = (int)(w / H);
+        const int h = (int)(w % H);
+        const int g = h / heads_per_group;
+        double *hs = state + ((size_t)s * H + h) * (size_t)P * N;
+        const double Dh = D ? D[h] : 0.0;
+        for (int64_t t = cu_seqlens[s]; t < cu_seqlens[s + 1]; ++t) {
+            recurrence_step(P, N, dt[(size_t)t * H + h], A[h], Dh,
+                            x + ((size_t)t * H + h) * P,
+                            B + ((size_t)t * G + g) * N,
+                            C + ((size_t)t * G + g) * N,
+                            hs,
+                            y + ((size_t)t * H + h) * P);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/*
+ * Single-token decode update, in place on the state (the decode path of the
+ * same recurrence: one token per batch element).
+ *
+ *   state [batch,H,P,N]  updated in place
+ *   x [batch,H,P]  dt [batch,H]  A [H]  B, C [batch,G,N]  D [H] or NULL
+ *   y [batch,H,P]
+ */
+int oracle_state_update(int batch, int H, int P, int N, int G,
+                        double *state, const double *x, const double *dt,
+                        const double *A, const double *B, const double *C,
+                        const double *D, double *y)
+{
+    if (batch < 0 || H <= 0 || P <= 0 || N <= 0 || G <= 0 || H % G != 0)
+        return ORACLE_BAD_ARG;
+    if (batch == 0) return ORACLE_OK;
+    if (!state || !x || !dt || !A || !B || !C || !y) return ORACLE_BAD_ARG;
+
+    const int heads_per_group = H / G;
+    const long work = (long)batch * H;
+
+#pragma omp parallel for schedule(static)
+    for (long w = 0; w < work; ++w) {
+        const int b = (int)(w / H);
+        const int h = (int)(w % H);
+        const int g = h / heads_per_group;
+        recurrence_step(P, N, dt[(size_t)b * H + h], A[h], D ? D[h] : 0.0,
+                        x + ((size_t)b * H + h) * P,
+                        B + ((size_t)b * G + g) * N,
+                        C + ((size_t)b * G + g) * N,
+                        state + ((size_t)b * H + h) * (size_t)P * N,
+                        y + ((size_t)b * H + h) * P);
+    }
+    return ORACLE_OK;
+}
