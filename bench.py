@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Throughput of the Mamba-2 selective-scan hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  * prefill: ssd_chunk_scan over 4 sequences x 4096 tokens, 128 heads,
+    head_dim 64, d_state 128, 8 groups, 128-token chunks, bf16 x/B/C, fp32 dt,
+    bf16 y, fp32 final state (zero initial state);
+  * decode: one ssm_state_update token for a batch of 64 at the Nemotron-3
+    Ultra layer shape (256 heads, head_dim 64, d_state 128, 8 groups), in place
+    on a 512 MiB fp32 state, bf16 x/B/C, bf16 y; per-step inputs cycle through
+    a ring of 8 seeded input sets.
+``value`` is tokens/s over both (16384 prefill + 64 decode tokens per step and
+per GPU); the per-kernel numbers the metric names (prefill tokens/s and % of
+tensor peak, decode GB/s and % of HBM peak) are under ``parts``.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank runs its own batch (weak scaling, no data-path
+collective); timing is max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("Mamba-2 prefill SSD tokens/s (% tensor peak); "
+          "decode update HBM GB/s (% peak)")
+PREFILL = dict(nseq=4, seqlen=4096, H=128, P=64, N=128, G=8, Q=128)
+DECODE = dict(batch=64, H=256, P=64, N=128, G=8)
+RING = 8
+
+# Fallback roofline denominators (used only if MEASURED_PEAKS.json is absent).
+FALLBACK_PEAKS = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_work(p=PREFILL, y_bytes=2):
+    """Algorithmic flops and bytes of one prefill launch.
+
+    flops per token = H(2QP + 4NP) + G*2QN (full Q x Q masked tile, the four
+    per-head contractions C.B^T-masked.X, X^T.B, C.H^T and the group's C.B^T);
+    bytes = x + B + C + dt + y per token, plus the fp32 final state.
+    """
+    T = p["nseq"] * p["seqlen"]
+    H, P, N, G, Q = p["H"], p["P"], p["N"], p["G"], p["Q"]
+    flops = T * (H * (2 * Q * P + 4 * N * P) + G * 2 * Q * N)
+    per_tok = H * P * 2 + 2 * G * N * 2 + H * 4 + H * P * y_bytes
+    bytes_ = T * per_tok + p["nseq"] * H * P * N * 4 + 2 * H * 4
+    return flops, bytes_, T
+
+
+def decode_work(d=DECODE, y_bytes=2):
+    """Algorithmic bytes of one decode launch: state read + write, x, B, C, dt,
+    A, D, y.  ~5 flops per state element (plain ALU work)."""
+    b, H, P, N, G = d["batch"], d["H"], d["P"], d["N"], d["G"]
+    state = b * H * P * N * 4
+    bytes_ = 2 * state + b * H * P * 2 + 2 * b * G * N * 2 + b * H * 4 + 2 * H * 4 + b * H * P * y_bytes
+    flops = 5 * b * H * P * N
+    return flops, bytes_, b
+
+
+def kernel_source_hash(fname):
+    path = os.path.join(ROOT, "hybrid_mamba_ssm_b200", "csrc", fname)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(kernel, source_file):
+    """DRAM bytes per launch from a committed ncu summary, or None if the
+    kernel's source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash(source_file)
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel:
+                if parts[1] == want:
+                    return float(parts[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.gpu_id:
+            cmd.insert(1, f"--id={self.gpu_id}")
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) >= 9:
+                    rows.append(c)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def gpu_uuid(dev):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if args.impl == "reference":
+        return world, rank, local, None   # rank 0 alone times the oracle
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local, pg
+
+
+def max_over_ranks(pg, value, device):
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, device=None):
+    if pg is not None:
+        if device is not None:
+            pg.barrier(device_ids=[device.index])
+        else:
+            pg.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_step_sample(rank_seed, prefill_tokens, prefill_heads, decode_rows):
+    """Time the oracle on a bounded sample of one step; returns (seconds for a
+    full step, description, threads)."""
+    import oracle
+    from hybrid_mamba_ssm_b200 import inputs as synth
+    oracle.set_num_threads(os.cpu_count() or 1)
+    p, d = PREFILL, DECODE
+    inp = synth.make_scan_inputs(rank_seed, [prefill_tokens], prefill_heads, p["P"], p["N"],
+                                 1, dtype="bf16")
+    t = time.perf_counter()
+    oracle.scan(inp.x.values, inp.dt, inp.A, inp.B.values, inp.C.values, inp.D, None)
+    t_pre = time.perf_counter() - t
+    A, D = synth.make_head_params(rank_seed + 1, d["H"])
+    st = synth.make_state(rank_seed + 2, (decode_rows, d["H"], d["P"], d["N"]))
+    dec = synth.make_decode_step(rank_seed + 3, decode_rows, d["H"], d["P"], d["N"], d["G"])
+    t = time.perf_counter()
+    oracle.state_update(st, dec.x.values, dec.dt, A, dec.B.values, dec.C.values, D)
+    t_dec = time.perf_counter() - t
+    full_pre = p["nseq"] * p["seqlen"] * p["H"]
+    scale_pre = full_pre / (prefill_tokens * prefill_heads)
+    scale_dec = d["batch"] / decode_rows
+    step_s = t_pre * scale_pre + t_dec * scale_dec
+    desc = (f"prefill {prefill_tokens} tokens x {prefill_heads} heads (of 16384 x 128) and "
+            f"decode {decode_rows} of 64 batch rows x 256 heads, scaled to one full step")
+    return step_s, desc, oracle.num_threads()
+
+
+def run_reference(args, world, rank, pg):
+    if rank != 0:
+        return 0
+    tokens_per_step = PREFILL["nseq"] * PREFILL["seqlen"] + DECODE["batch"]
+    for _ in range(args.warmup):
+        oracle_step_sample(2000, 256, 4, 1)
+    total = 0.0
+    desc = cores = None
+    for k in range(args.steps):
+        s, desc, cores = oracle_step_sample(2000 + k, 256, 4, 1)
+        total += s
+    value = tokens_per_step * args.steps / total
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": "prefill 4x4096 H128 P64 N128 G8 Q128 + decode 64x256x64x128 G8",
+                       "reference": "fp64 CPU oracle (sequential recurrence), bounded sample per step"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU path
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank, local, pg):
+    import torch
+    from hybrid_mamba_ssm_b200 import inputs as synth
+    from hybrid_mamba_ssm_b200 import ssm
+
+    dev = torch.device("cuda", local)
+    p, d = PREFILL, DECODE
+    seed = 1000 + 2 + 7919 * rank
+
+    def bf16(t, pin=False):
+        a = torch.from_numpy(np.ascontiguousarray(t.bits).view(np.int16)).view(torch.bfloat16)
+        return a.pin_memory() if pin else a.to(dev)
+
+    def f32(a, pin=False):
+        t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+        return t.pin_memory() if pin else t.to(dev)
+
+    # prefill inputs (resident) and host copies (for the end-to-end leg)
+    pin = synth.make_scan_inputs(seed, [p["seqlen"]] * p["nseq"], p["H"], p["P"], p["N"],
+                                 p["G"], dtype="bf16")
+    L = p["seqlen"]
+    shp = lambda t, *s: t.view(p["nseq"], L, *s)
+    px, pdt = bf16(pin.x), f32(pin.dt)
+    pB, pC = bf16(pin.B), bf16(pin.C)
+    pA, pD = f32(pin.A), f32(pin.D)
+    py = torch.empty((p["nseq"], L, p["H"], p["P"]), dtype=torch.bfloat16, device=dev)
+    phT = torch.empty((p["nseq"], p["H"], p["P"], p["N"]), dtype=torch.float32, device=dev)
+    host_pre = dict(x=bf16(pin.x, True), dt=f32(pin.dt, True), B=bf16(pin.B, True),
+                    C=bf16(pin.C, True))
+
+    # decode: state, per-head params, a ring of per-step inputs
+    dA, dD = synth.make_head_params(1001 + 7919 * rank, d["H"])
+    dA, dD = f32(dA), f32(dD)
+    state = f32(synth.make_state(1001 + 7919 * rank + 1, (d["batch"], d["H"], d["P"], d["N"])))
+    ring, host_ring = [], []
+    for k in range(RING):
+        s = synth.make_decode_step(1001 + 7919 * rank + 100 + k, d["batch"], d["H"], d["P"],
+                                   d["N"], d["G"])
+        ring.append((bf16(s.x), f32(s.dt), bf16(s.B), bf16(s.C)))
+        host_ring.append((bf16(s.x, True), f32(s.dt, True), bf16(s.B, True), bf16(s.C, True)))
+    dy = torch.empty((d["batch"], d["H"], d["P"]), dtype=torch.bfloat16, device=dev)
+
+    stream = torch.cuda.current_stream(dev)
+
+    def prefill(x=px, dt=pdt, B=pB, C=pC):
+        ssm.ssd_chunk_scan(shp(x, p["H"], p["P"]), shp(dt, p["H"]), pA,
+                           shp(B, p["G"], p["N"]), shp(C, p["G"], p["N"]), pD, None,
+                           chunk_size=p["Q"], y=py, final_state=phT, stream=stream)
+
+    def decode(k, inp=None):
+        x, dt, B, C = inp if inp is not None else ring[k % RING]
+        ssm.ssm_state_update(state, x, dt, dA, B, C, dD, y=dy, stream=stream)
+
+    for k in range(args.warmup):
+        prefill()
+        decode(k)
+    torch.cuda.synchronize(dev)
+    barrier(pg, dev)
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(gpu_uuid(dev))
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        prefill()
+        ev[k][1].record(stream)
+        ev[k][2].record(stream)
+        decode(k)
+        ev[k][3].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clock_info = clocks.stop()
+    barrier(pg, dev)
+    ms = max_over_ranks(pg, start.elapsed_time(end), dev)
+    pre_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / K
+    pre_ms = max_over_ranks(pg, pre_ms, dev)
+    dec_ms = max_over_ranks(pg, dec_ms, dev)
+
+    # ---- end to end: pinned host inputs -> device, call, results -> host ----
+    out_host = dict(y=torch.empty(py.shape, dtype=py.dtype, pin_memory=True),
+                    hT=torch.empty(phT.shape, dtype=phT.dtype, pin_memory=True),
+                    dy=torch.empty(dy.shape, dtype=dy.dtype, pin_memory=True))
+    h2d = sum(t.numel() * t.element_size() for t in host_pre.values()) + \
+        sum(t.numel() * t.element_size() for t in host_ring[0])
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    e2e_steps = max(1, min(K, 50))
+    ex, edt, eB, eC = (torch.empty_like(px), torch.empty_like(pdt), torch.empty_like(pB),
+                       torch.empty_like(pC))
+    dbuf = [torch.empty_like(t) for t in ring[0]]
+
+    def e2e_step(k):
+        ex.copy_(host_pre["x"], non_blocking=True)
+        edt.copy_(host_pre["dt"], non_blocking=True)
+        eB.copy_(host_pre["B"], non_blocking=True)
+        eC.copy_(host_pre["C"], non_blocking=True)
+        for dst, src in zip(dbuf, host_ring[k % RING]):
+            dst.copy_(src, non_blocking=True)
+        prefill(ex, edt, eB, eC)
+        decode(k, dbuf)
+        out_host["y"].copy_(py, non_blocking=True)
+        out_host["hT"].copy_(phT, non_blocking=True)
+        out_host["dy"].copy_(dy, non_blocking=True)
+
+    for k in range(2):
+        e2e_step(k)
+    torch.cuda.synchronize(dev)
+    barrier(pg, dev)
+    torch.cuda.synchronize(dev)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for k in range(e2e_steps):
+        e2e_step(k)
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(pg, dev)
+    e2e_ms = max_over_ranks(pg, s2.elapsed_time(e2), dev)
+
+    # ---- numbers ----
+    peaks, peak_kind = load_peaks()
+    tok_step = p["nseq"] * p["seqlen"] + d["batch"]
+    value = world * tok_step * K / (ms * 1e-3)
+    e2e_value = world * tok_step * e2e_steps / (e2e_ms * 1e-3)
+    pf, pb, ptok = prefill_work()
+    df, db, _ = decode_work()
+    hbm = peaks["hbm_gbs"]
+    t_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    pre = {"tokens_per_s": ptok / (pre_ms * 1e-3), "ms": pre_ms,
+           "tflops": pf / (pre_ms * 1e-3) / 1e12,
+           "tensor_frac_sustained": pf / (pre_ms * 1e-3) / 1e12 / t_sus,
+           "tensor_frac_burst": pf / (pre_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+           "gbs": pb / (pre_ms * 1e-3) / 1e9, "hbm_frac": pb / (pre_ms * 1e-3) / 1e9 / hbm,
+           "flops_per_launch": pf, "bytes_per_launch": pb}
+    dec = {"gbs": db / (dec_ms * 1e-3) / 1e9, "ms": dec_ms,
+           "hbm_frac": db / (dec_ms * 1e-3) / 1e9 / hbm,
+           "hbm_frac_of_8TBs": db / (dec_ms * 1e-3) / 8e12,
+           "tokens_per_s": d["batch"] / (dec_ms * 1e-3), "bytes_per_launch": db}
+    # prefill is HBM-bound by arithmetic intensity (flops/byte below the ridge)
+    if pre_ms >= dec_ms:
+        ridge = t_sus * 1e12 / (hbm * 1e9)
+        if pf / pb < ridge:
+            roof = {"kernel": "ssd_chunk_scan", "bound": "hbm", "achieved": pre["gbs"],
+                    "peak": hbm, "unit": "GB/s", "frac": pre["hbm_frac"],
+                    "traffic": measured_traffic("ssd_chunk_scan", "scan_tc.cu")}
+        else:
+            roof = {"kernel": "ssd_chunk_scan", "bound": "tensor", "achieved": pre["tflops"],
+                    "peak": t_sus, "unit": "TFLOP/s", "frac": pre["tensor_frac_sustained"],
+                    "traffic": measured_traffic("ssd_chunk_scan", "scan_tc.cu")}
+    else:
+        roof = {"kernel": "ssm_state_update", "bound": "hbm", "achieved": dec["gbs"],
+                "peak": hbm, "unit": "GB/s", "frac": dec["hbm_frac"],
+                "traffic": measured_traffic("ssm_state_update", "state_update.cu")}
+    roof["peak_source"] = peak_kind
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "prefill 4x4096 H128 P64 N128 G8 Q128 + decode 64x256x64x128 G8",
+                       "prefill": dict(PREFILL, in_dtype="bf16", y_dtype="bf16",
+                                       initial_state="zero"),
+                       "decode": dict(DECODE, in_dtype="bf16", y_dtype="bf16", ring=RING),
+                       "l2": "inputs larger than L2 (about 1.7 GB touched per step)",
+                       "parallelism": f"replicas x{world} (independent batches per GPU)"},
+            "parts": {"prefill": pre, "decode": dec},
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": 2 * K,
+            "clocks": clock_info}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        step_s, desc, cores = oracle_step_sample(3000, 1024, 8, 4)
+        line["cpu_baseline"] = {"value": tok_step / step_s, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)   # timing rule: at least 3 warm-up steps
+    world, rank, local, pg = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            rc = run_reference(args, world, rank, pg)
+        else:
+            rc = run_ours(args, world, rank, local, pg)
+    finally:
+        if pg is not None:
+            pg.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

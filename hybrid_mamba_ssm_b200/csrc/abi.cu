@@ -1,0 +1,169 @@
+// abi.cu -- the extern "C" entry points of libssm: host-side validation of
+// every argument, then one kernel launch on the caller's stream.  Nothing
+// here allocates, synchronises or keeps state between calls.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ssm.h"
+#include "ssm_internal.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;   // [lo, hi)
+};
+
+Range range_of(const void *p, size_t bytes)
+{
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Range{a, a + bytes};
+}
+
+bool overlap(Range a, Range b)
+{
+    if (a.lo == a.hi || b.lo == b.hi || a.lo == 0 || b.lo == 0) return false;
+    return a.lo < b.hi && b.lo < a.hi;
+}
+
+size_t dtype_size(int dt) { return dt == SSM_BF16 ? 2 : 4; }
+
+bool valid_dtype(int dt) { return dt == SSM_F32 || dt == SSM_BF16; }
+
+bool pow2_in(int v, int lo, int hi)
+{
+    return v >= lo && v <= hi && (v & (v - 1)) == 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ssm_status_string(int status)
+{
+    switch (status) {
+    case SSM_OK: return "SSM_OK";
+    case SSM_ERR_INVALID_ARG: return "SSM_ERR_INVALID_ARG: invalid argument";
+    case SSM_ERR_UNSUPPORTED: return "SSM_ERR_UNSUPPORTED: shape or dtype not supported";
+    case SSM_ERR_MISALIGNED: return "SSM_ERR_MISALIGNED: pointer not 16-byte aligned";
+    case SSM_ERR_CUDA: return "SSM_ERR_CUDA: CUDA launch error";
+    case SSM_ERR_TIMEOUT: return "SSM_ERR_TIMEOUT: bounded device wait expired";
+    case SSM_ERR_DEVICE_INPUT: return "SSM_ERR_DEVICE_INPUT: inconsistent cu_seqlens";
+    default: return "unknown ssm status";
+    }
+}
+
+int ssm_version(void) { return 100; }
+
+size_t ssd_chunk_scan_workspace_size(int, int, int, int, int, int, int) { return 0; }
+
+int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
+                   int nheads, int head_dim, int d_state, int ngroups,
+                   int chunk_size, int in_dtype,
+                   const void *x, const float *dt, const float *A,
+                   const void *B, const void *C, const float *D,
+                   const float *initial_state,
+                   int y_dtype, void *y, float *final_state,
+                   void *workspace, size_t workspace_bytes,
+                   int *status_dev, cudaStream_t stream)
+{
+    (void)workspace; (void)workspace_bytes;
+    if (nseq < 0 || seqlen < 0 || nheads <= 0 || ngroups <= 0 || nheads % ngroups)
+        return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
+    if (!pow2_in(head_dim, 16, 128) || !pow2_in(d_state, 16, 128)) return SSM_ERR_UNSUPPORTED;
+    if (chunk_size != 64 && chunk_size != 128) return SSM_ERR_UNSUPPORTED;
+    if (nseq == 0) return SSM_OK;
+    const long long T = cu_seqlens ? (long long)seqlen : (long long)nseq * seqlen;
+    if (T > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    if (T == 0 && !cu_seqlens) {
+        // every sequence is empty: final = initial
+        if (final_state && final_state != initial_state) {
+            const size_t bytes = (size_t)nseq * nheads * head_dim * d_state * sizeof(float);
+            cudaError_t e = initial_state
+                ? cudaMemcpyAsync(final_state, initial_state, bytes, cudaMemcpyDeviceToDevice, stream)
+                : cudaMemsetAsync(final_state, 0, bytes, stream);
+            return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+        }
+        return SSM_OK;
+    }
+    if (!A) return SSM_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !dt || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {cu_seqlens, x, dt, A, B, C, D, initial_state, y, final_state, status_dev};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+
+    const size_t es = dtype_size(in_dtype);
+    const size_t state_bytes = (size_t)nseq * nheads * head_dim * d_state * sizeof(float);
+    const Range rx = range_of(x, (size_t)T * nheads * head_dim * es);
+    const Range rdt = range_of(dt, (size_t)T * nheads * sizeof(float));
+    const Range rA = range_of(A, (size_t)nheads * sizeof(float));
+    const Range rB = range_of(B, (size_t)T * ngroups * d_state * es);
+    const Range rC = range_of(C, (size_t)T * ngroups * d_state * es);
+    const Range rD = range_of(D, D ? (size_t)nheads * sizeof(float) : 0);
+    const Range rh0 = range_of(initial_state, initial_state ? state_bytes : 0);
+    const Range ry = range_of(y, (size_t)T * nheads * head_dim * dtype_size(y_dtype));
+    const Range rhT = range_of(final_state, final_state ? state_bytes : 0);
+    const Range rcu = range_of(cu_seqlens, cu_seqlens ? (size_t)(nseq + 1) * sizeof(int32_t) : 0);
+    const Range ins[] = {rx, rdt, rA, rB, rC, rD, rh0, rcu};
+    for (const Range &r : ins) {
+        if (overlap(ry, r)) return SSM_ERR_INVALID_ARG;
+        if (&r != &ins[6] && overlap(rhT, r)) return SSM_ERR_INVALID_ARG;
+    }
+    if (overlap(ry, rhT)) return SSM_ERR_INVALID_ARG;
+    if (initial_state && final_state && initial_state != final_state && overlap(rh0, rhT))
+        return SSM_ERR_INVALID_ARG;
+
+    ssm::ScanArgs a;
+    a.nseq = nseq; a.seqlen = seqlen; a.cu_seqlens = cu_seqlens;
+    a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
+    a.ngroups = ngroups; a.chunk_size = chunk_size;
+    a.in_dtype = in_dtype; a.y_dtype = y_dtype;
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.initial_state = initial_state; a.y = y; a.final_state = final_state;
+    a.status_dev = status_dev;
+    const cudaError_t e = ssm::scan_tc_supports(a) ? ssm::launch_scan_tc(a, stream)
+                                                   : ssm::launch_scan_simt(a, stream);
+    return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_state_update(int batch, int nheads, int head_dim, int d_state,
+                     int ngroups, int in_dtype, float *state,
+                     const void *x, const float *dt, const float *A,
+                     const void *B, const void *C, const float *D,
+                     int y_dtype, void *y, cudaStream_t stream)
+{
+    if (batch < 0 || nheads <= 0 || ngroups <= 0 || nheads % ngroups || head_dim <= 0)
+        return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
+    if (head_dim > 256 || !pow2_in(d_state, 16, 256)) return SSM_ERR_UNSUPPORTED;
+    if ((long long)batch * nheads > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    if (batch == 0) return SSM_OK;
+    if (!state || !x || !dt || !A || !B || !C || !y) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {state, x, dt, A, B, C, D, y};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+
+    const size_t es = dtype_size(in_dtype);
+    const Range rs = range_of(state, (size_t)batch * nheads * head_dim * d_state * sizeof(float));
+    const Range rx = range_of(x, (size_t)batch * nheads * head_dim * es);
+    const Range rdt = range_of(dt, (size_t)batch * nheads * sizeof(float));
+    const Range rA = range_of(A, (size_t)nheads * sizeof(float));
+    const Range rB = range_of(B, (size_t)batch * ngroups * d_state * es);
+    const Range rC = range_of(C, (size_t)batch * ngroups * d_state * es);
+    const Range rD = range_of(D, D ? (size_t)nheads * sizeof(float) : 0);
+    const Range ry = range_of(y, (size_t)batch * nheads * head_dim * dtype_size(y_dtype));
+    const Range ins[] = {rx, rdt, rA, rB, rC, rD};
+    for (const Range &r : ins)
+        if (overlap(ry, r) || overlap(rs, r)) return SSM_ERR_INVALID_ARG;
+    if (overlap(ry, rs)) return SSM_ERR_INVALID_ARG;
+
+    ssm::StateUpdateArgs a;
+    a.batch = batch; a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
+    a.ngroups = ngroups; a.in_dtype = in_dtype; a.y_dtype = y_dtype;
+    a.state = state; a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.y = y;
+    return ssm::launch_state_update(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+}  // extern "C"

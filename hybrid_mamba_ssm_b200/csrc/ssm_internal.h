@@ -1,0 +1,47 @@
+// ssm_internal.h -- argument bundles passed from the C ABI layer (abi.cu),
+// which has already validated them, to the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssm {
+
+struct StateUpdateArgs {
+    int batch, nheads, head_dim, d_state, ngroups;
+    int in_dtype, y_dtype;        // 0 = fp32, 1 = bf16
+    float *state;
+    const void *x;
+    const float *dt, *A;
+    const void *B, *C;
+    const float *D;
+    void *y;
+};
+
+struct ScanArgs {
+    int nseq, seqlen;             // seqlen = T when cu_seqlens is given
+    const int32_t *cu_seqlens;    // device [nseq+1] or nullptr
+    int nheads, head_dim, d_state, ngroups, chunk_size;
+    int in_dtype, y_dtype;
+    const void *x;
+    const float *dt, *A;
+    const void *B, *C;
+    const float *D;
+    const float *initial_state;   // nullptr = zero
+    void *y;
+    float *final_state;           // nullptr = not written
+    int *status_dev;              // nullptr = not reported
+};
+
+cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);
+
+// General chunked scan on the CUDA cores: any supported shape and dtype.
+cudaError_t launch_scan_simt(const ScanArgs &a, cudaStream_t stream);
+
+// Tensor-core (tcgen05 / TMEM / TMA) chunked scan.  Returns
+// cudaErrorNotSupported, launching nothing, for shapes it does not cover.
+bool scan_tc_supports(const ScanArgs &a);
+cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t stream);
+
+}  // namespace ssm

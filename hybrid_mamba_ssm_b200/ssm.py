@@ -1,0 +1,171 @@
+"""Python binding of libssm (include/ssm.h): argument marshalling only.
+
+Torch tensors supply device memory and the current CUDA stream; every step of
+the scan runs in the library's kernels.  Importing this module loads
+``libssm.so`` and raises ImportError if it is missing or cannot be loaded --
+there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm.so")
+
+SSM_F32, SSM_BF16 = 0, 1
+STATUS_NAMES = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED",
+                3: "SSM_ERR_MISALIGNED", 4: "SSM_ERR_CUDA", 5: "SSM_ERR_TIMEOUT",
+                6: "SSM_ERR_DEVICE_INPUT"}
+EXPORTS = ("ssd_chunk_scan", "ssd_chunk_scan_workspace_size", "ssm_state_update",
+           "ssm_status_string", "ssm_version")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libssm.so is not built ({LIB_PATH}); run "
+                          "`python -m hybrid_mamba_ssm_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.ssd_chunk_scan.restype = i
+    lib.ssd_chunk_scan.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp,
+                                   vp, vp, i, vp, vp, vp, sz, vp, vp]
+    lib.ssd_chunk_scan_workspace_size.restype = sz
+    lib.ssd_chunk_scan_workspace_size.argtypes = [i] * 7
+    lib.ssm_state_update.restype = i
+    lib.ssm_state_update.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, i,
+                                     vp, vp]
+    lib.ssm_status_string.restype = ctypes.c_char_p
+    lib.ssm_status_string.argtypes = [i]
+    lib.ssm_version.restype = i
+    return lib
+
+
+lib = _load()
+
+
+class SSMError(RuntimeError):
+    """A libssm entry point returned a nonzero status."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.ssm_status_string(status).decode()}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise SSMError(status, where)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return SSM_BF16
+    if t == torch.float32:
+        return SSM_F32
+    raise TypeError(f"unsupported dtype {t}; use torch.bfloat16 or torch.float32")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, name, dtype=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def ssd_chunk_scan(x, dt, A, B, C, D=None, initial_state=None, cu_seqlens=None,
+                   chunk_size: int = 128, y=None, final_state=None, y_dtype=None,
+                   return_final_state: bool = True, status=None, stream=None):
+    """Chunked SSD prefill scan.
+
+    x  : [nseq, L, H, P] (fixed length) or [T, H, P] with ``cu_seqlens``
+    dt : [nseq, L, H] or [T, H], fp32
+    A  : [H] fp32;  D : [H] fp32 or None
+    B, C : [nseq, L, G, N] or [T, G, N], same dtype as x
+    initial_state : [nseq, H, P, N] fp32 or None (zeros); may be ``final_state``
+    cu_seqlens : int32 [nseq+1] CUDA tensor of packed offsets, or None
+    y / final_state : optional preallocated outputs
+    Returns (y, final_state) -- final_state is None if not requested.
+    """
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens", torch.int32)
+        T, H, P = x.shape
+        nseq = cu_seqlens.shape[0] - 1
+        seqlen = T
+    else:
+        nseq, L, H, P = x.shape
+        T, seqlen = nseq * L, L
+    G, N = B.shape[-2], B.shape[-1]
+    _dev(dt, "dt", torch.float32)
+    _dev(A, "A", torch.float32)
+    _dev(B, "B", x.dtype)
+    _dev(C, "C", x.dtype)
+    _dev(D, "D", torch.float32)
+    _dev(initial_state, "initial_state", torch.float32)
+    if y_dtype is None:
+        y_dtype = x.dtype if y is None else y.dtype
+    if y is None:
+        y = torch.empty(x.shape, dtype=y_dtype, device=x.device)
+    _dev(y, "y", y_dtype)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((nseq, H, P, N), dtype=torch.float32, device=x.device)
+    _dev(final_state, "final_state", torch.float32)
+    _dev(status, "status", torch.int32)
+    st = lib.ssd_chunk_scan(nseq, seqlen, _ptr(cu_seqlens), H, P, N, G, int(chunk_size),
+                            in_code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                            _ptr(D), _ptr(initial_state), _dtype_code(y.dtype), _ptr(y),
+                            _ptr(final_state), None, 0, _ptr(status), _stream(stream))
+    _check(st, "ssd_chunk_scan")
+    return y, final_state
+
+
+def ssd_chunk_scan_workspace_size(nseq, seqlen, nheads, head_dim, d_state, ngroups,
+                                  chunk_size=128) -> int:
+    return int(lib.ssd_chunk_scan_workspace_size(nseq, seqlen, nheads, head_dim, d_state,
+                                                 ngroups, chunk_size))
+
+
+def ssm_state_update(state, x, dt, A, B, C, D=None, y=None, y_dtype=None, stream=None):
+    """One-token decode update, in place on ``state`` [batch, H, P, N] fp32.
+
+    x : [batch, H, P];  dt : [batch, H] fp32;  A, D : [H] fp32;
+    B, C : [batch, G, N] (same dtype as x).  Returns y [batch, H, P].
+    """
+    _dev(state, "state", torch.float32)
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    batch, H, P, N = state.shape
+    G = B.shape[-2]
+    _dev(dt, "dt", torch.float32)
+    _dev(A, "A", torch.float32)
+    _dev(B, "B", x.dtype)
+    _dev(C, "C", x.dtype)
+    _dev(D, "D", torch.float32)
+    if y_dtype is None:
+        y_dtype = x.dtype if y is None else y.dtype
+    if y is None:
+        y = torch.empty((batch, H, P), dtype=y_dtype, device=state.device)
+    _dev(y, "y", y_dtype)
+    st = lib.ssm_state_update(batch, H, P, N, G, in_code, _ptr(state), _ptr(x), _ptr(dt),
+                              _ptr(A), _ptr(B), _ptr(C), _ptr(D), _dtype_code(y.dtype),
+                              _ptr(y), _stream(stream))
+    _check(st, "ssm_state_update")
+    return y

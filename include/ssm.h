@@ -1,0 +1,160 @@
+/*
+ * ssm.h -- C ABI of libssm, the B200 (sm_100a) Mamba-2 selective state-space
+ * scan.
+ *
+ * The operation (the selective-SSM recurrence of the note "Mamba 与 Nemotron
+ * 系列模型深度调研", section "1. Selective SSM 的直觉"; its decode form in the
+ * modeling_nemotron_h.py walk-through, section "Decode 阶段"): for every
+ * sequence, head h (group g = h / (nheads / ngroups)) and token t in order,
+ *
+ *     state[p][n] <- exp(dt[t][h] * A[h]) * state[p][n] + dt[t][h] * x[t][h][p] * B[t][g][n]
+ *     y[t][h][p]   = sum_n state[p][n] * C[t][g][n] + D[h] * x[t][h][p]
+ *
+ * y reads the state AFTER the token's update.  A and D are per-head fp32
+ * scalars, dt is the final per-(token, head) step size in fp32 (already passed
+ * through any bias / softplus / clamp), and B, C are shared by the heads of a
+ * group.  The recurrent state is always fp32 (the walk-through's section on
+ * why the SSM cache defaults to float32).
+ *
+ * Layouts (row-major, contiguous, no padding between rows):
+ *   x, y          [T][nheads][head_dim]
+ *   dt            [T][nheads]               fp32
+ *   A, D          [nheads]                  fp32
+ *   B, C          [T][ngroups][d_state]
+ *   state         [nseq or batch][nheads][head_dim][d_state]   fp32
+ * where T is the number of tokens (for decode, T = batch).
+ *
+ * Ownership: the caller allocates every buffer and owns it.  No entry point
+ * allocates device memory, synchronises the device or the stream, or keeps
+ * state between calls; all work is enqueued on the given stream.  Pointers
+ * marked "device" must be device-accessible (cudaMalloc'd or managed).
+ *
+ * Errors: shapes, dtypes, null pointers and alignment are checked on the host
+ * BEFORE anything is launched; on any error nothing is launched and the call
+ * returns the status.  A launch failure returns SSM_ERR_CUDA (from
+ * cudaGetLastError, no synchronisation).  Problems only the device can see
+ * (inconsistent cu_seqlens) are reported through the optional status word.
+ */
+#ifndef LIBSSM_SSM_H
+#define LIBSSM_SSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define SSM_API __attribute__((visibility("default")))
+#else
+#define SSM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1,   /* bad shape, null pointer, aliasing, range */
+    SSM_ERR_UNSUPPORTED = 2,   /* valid request this build does not handle */
+    SSM_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+    SSM_ERR_CUDA = 4,          /* the CUDA runtime reported a launch error */
+    SSM_ERR_TIMEOUT = 5,       /* reserved: a bounded device wait expired */
+    SSM_ERR_DEVICE_INPUT = 6   /* written to status_dev: bad cu_seqlens */
+} ssm_status;
+
+typedef enum {
+    SSM_F32 = 0,
+    SSM_BF16 = 1
+} ssm_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+SSM_API const char *ssm_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+SSM_API int ssm_version(void);
+
+/*
+ * ssd_chunk_scan -- prefill: the recurrence over whole sequences, computed as
+ * a chunked SSD (structured state-space duality) scan.  Chunks of chunk_size
+ * tokens restart at every sequence start; inside a chunk the token-to-token
+ * interactions form a decay-masked C.B^T product on the tensor cores, and the
+ * state is carried from chunk to chunk on chip.  This is the
+ * mamba_chunk_scan_combined(..., return_final_states=True) step of the
+ * walk-through's section "Prefill 阶段" (128-token chunks), and the in-place
+ * initial/final state of the MAX mamba2_ssd_chunk_scan_varlen_fwd_inplace
+ * kernel (MAX nemotron_h article, section 5.4 item 3).
+ *
+ * Sequences:
+ *   cu_seqlens == NULL: nseq sequences of seqlen tokens each, T = nseq*seqlen.
+ *   cu_seqlens != NULL: device int32 [nseq+1], packed varlen; cu[0] = 0,
+ *     non-decreasing, cu[nseq] = seqlen = T (seqlen is then the total).  A
+ *     device-side inconsistency (cu[0] != 0, a decreasing offset, cu[nseq] !=
+ *     seqlen) skips the affected sequences and writes SSM_ERR_DEVICE_INPUT to
+ *     *status_dev when status_dev is given.
+ *
+ * Shapes: nheads % ngroups == 0; head_dim in {16, 32, 64, 128};
+ *   d_state in {16, 32, 64, 128}; chunk_size in {64, 128}; seqlen >= 0.
+ * in_dtype: storage type of x, B and C (SSM_BF16 or SSM_F32).  dt, A, D are
+ *   always fp32.  Accumulation is fp32; bf16 operands of the tensor-core
+ *   products are carried as fp16 (exact for |v| < 65504) so that derived
+ *   operands (decay-masked C.B^T, decay-weighted x, the carried state) keep
+ *   11 significant bits.
+ * D: device [nheads] or NULL (no skip term).
+ * initial_state: device fp32 [nseq][nheads][head_dim][d_state] or NULL (zero).
+ *   It may be the same pointer as final_state (in-place update of a state
+ *   slot); any other overlap with an output is rejected.
+ * y: device [T][nheads][head_dim], y_dtype (SSM_F32 or SSM_BF16, round to
+ *   nearest even).  Must not overlap any input.
+ * final_state: device fp32 [nseq][nheads][head_dim][d_state] or NULL.
+ * workspace / workspace_bytes: reserved; pass NULL / 0 (the required size,
+ *   ssd_chunk_scan_workspace_size, is 0 in this version).
+ * status_dev: device int32 or NULL; the kernels only ever write a nonzero
+ *   status into it (the caller zeroes it).
+ * stream: the CUDA stream to enqueue on (0 = legacy default stream).
+ * All device pointers must be 16-byte aligned (SSM_ERR_MISALIGNED).
+ */
+SSM_API int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
+                   int nheads, int head_dim, int d_state, int ngroups,
+                   int chunk_size, int in_dtype,
+                   const void *x, const float *dt, const float *A,
+                   const void *B, const void *C, const float *D,
+                   const float *initial_state,
+                   int y_dtype, void *y, float *final_state,
+                   void *workspace, size_t workspace_bytes,
+                   int *status_dev, cudaStream_t stream);
+
+/* Workspace bytes ssd_chunk_scan needs for these shapes (0 in this version). */
+SSM_API size_t ssd_chunk_scan_workspace_size(int nseq, int seqlen, int nheads,
+                                     int head_dim, int d_state, int ngroups,
+                                     int chunk_size);
+
+/*
+ * ssm_state_update -- decode: one token per batch element, applied in place
+ * to the fp32 state (the selective_state_update step of the walk-through's
+ * section "Decode 阶段"; the TensorRT MambaPlugin update_ssm_state of the
+ * deep-research note, section "TensorRT Plugin 做 selective state update",
+ * without its copy-to-output since the update here is in place).
+ *
+ *   state  device fp32 [batch][nheads][head_dim][d_state], read and written
+ *   x      device [batch][nheads][head_dim], in_dtype
+ *   dt     device fp32 [batch][nheads]
+ *   A      device fp32 [nheads]
+ *   B, C   device [batch][ngroups][d_state], in_dtype
+ *   D      device fp32 [nheads] or NULL
+ *   y      device [batch][nheads][head_dim], y_dtype; must not overlap state
+ *          or any input
+ * Shapes: nheads % ngroups == 0; head_dim >= 1 and <= 256;
+ *   d_state in {16, 32, 64, 128, 256}; batch >= 0 (0 is a no-op).
+ * The kernel reads and writes each state element exactly once.
+ */
+SSM_API int ssm_state_update(int batch, int nheads, int head_dim, int d_state,
+                     int ngroups, int in_dtype, float *state,
+                     const void *x, const float *dt, const float *A,
+                     const void *B, const void *C, const float *D,
+                     int y_dtype, void *y, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBSSM_SSM_H */

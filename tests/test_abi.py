@@ -1,0 +1,133 @@
+"""The C ABI: the library loads, exports every symbol include/ssm.h declares,
+and rejects bad arguments on the host before launching anything.
+
+No test here launches a kernel: every call either fails validation (which
+happens before any CUDA call) or is a documented no-op (batch 0, nseq 0).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hybrid_mamba_ssm_b200 import build as ssm_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED = 0, 1, 2, 3
+F32, BF16 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = ssm_build.build()
+    lib = ctypes.CDLL(path)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.ssd_chunk_scan.restype = i
+    lib.ssd_chunk_scan.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp,
+                                   vp, vp, i, vp, vp, vp, sz, vp, vp]
+    lib.ssm_state_update.restype = i
+    lib.ssm_state_update.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, i,
+                                     vp, vp]
+    lib.ssm_status_string.restype = ctypes.c_char_p
+    lib.ssm_status_string.argtypes = [i]
+    lib.ssd_chunk_scan_workspace_size.restype = sz
+    lib.ssd_chunk_scan_workspace_size.argtypes = [i] * 7
+    return lib
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"SSM_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("ssd_chunk_scan", "ssm_state_update", "ssd_chunk_scan_workspace_size",
+                     "ssm_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libssm.so does not export {name}"
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.ssm_status_string(code)
+    assert b"unknown" in lib.ssm_status_string(99)
+
+
+def test_workspace_size_is_zero(lib):
+    assert lib.ssd_chunk_scan_workspace_size(4, 4096, 128, 64, 128, 8, 128) == 0
+
+
+# Fake, never-dereferenced device addresses: validation rejects the call first.
+A16 = 0x10000
+A16b = 0x20000
+A16c = 0x30000
+ODD = 0x10008   # 8-byte aligned only
+
+
+def scan(lib, nseq=1, seqlen=128, cu=None, H=4, P=64, N=128, G=1, Q=128, ind=BF16,
+         x=A16, dt=A16b, A=A16c, B=0x40000, C=0x50000, D=None, h0=None, yd=BF16,
+         y=0x60000, hT=0x70000, status=None):
+    return lib.ssd_chunk_scan(nseq, seqlen, cu, H, P, N, G, Q, ind, x, dt, A, B, C, D,
+                              h0, yd, y, hT, None, 0, status, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(H=6, G=4), INVALID),             # heads not a multiple of groups
+    (dict(G=0), INVALID),
+    (dict(nseq=-1), INVALID),
+    (dict(seqlen=-5), INVALID),
+    (dict(ind=7), INVALID),
+    (dict(yd=3), INVALID),
+    (dict(P=48), UNSUPPORTED),
+    (dict(N=256), UNSUPPORTED),
+    (dict(Q=96), UNSUPPORTED),
+    (dict(A=None), INVALID),
+    (dict(x=None), INVALID),
+    (dict(y=None), INVALID),
+    (dict(x=ODD), MISALIGNED),
+    (dict(hT=ODD), MISALIGNED),
+    (dict(y=0x10000 + 1024), INVALID),     # y overlaps x
+    (dict(hT=0x40000 + 64), INVALID),      # final state overlaps B
+    (dict(h0=0x70000 + 4096), INVALID),    # partial overlap of initial / final
+])
+def test_scan_rejects(lib, kw, code):
+    assert scan(lib, **kw) == code
+
+
+def test_scan_nseq_zero_is_noop(lib):
+    assert scan(lib, nseq=0, x=None, dt=None, y=None, hT=None) == OK
+
+
+def update(lib, batch=2, H=4, P=64, N=128, G=2, ind=BF16, state=0x100000, x=A16,
+           dt=A16b, A=A16c, B=0x40000, C=0x50000, D=None, yd=F32, y=0x60000):
+    return lib.ssm_state_update(batch, H, P, N, G, ind, state, x, dt, A, B, C, D, yd, y,
+                                None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(H=5, G=2), INVALID),
+    (dict(batch=-1), INVALID),
+    (dict(P=0), INVALID),
+    (dict(P=300), UNSUPPORTED),
+    (dict(N=24), UNSUPPORTED),
+    (dict(N=512), UNSUPPORTED),
+    (dict(ind=2), INVALID),
+    (dict(state=None), INVALID),
+    (dict(B=None), INVALID),
+    (dict(state=ODD), MISALIGNED),
+    (dict(y=0x100000 + 256), INVALID),     # y inside the state
+    (dict(x=0x100000), INVALID),           # x inside the state
+])
+def test_update_rejects(lib, kw, code):
+    assert update(lib, **kw) == code
+
+
+def test_update_batch_zero_is_noop(lib):
+    assert update(lib, batch=0, state=None, x=None) == OK

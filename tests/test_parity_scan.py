@@ -1,0 +1,91 @@
+"""Prefill (ssd_chunk_scan) against the fp64 oracle, element by element.
+
+Small cases compare every element and span several chunks plus a ragged tail;
+the full-size workloads run in the benchmark's launch configuration and
+compare sampled heads, which the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from hybrid_mamba_ssm_b200 import inputs as synth
+from tests.gpu_helpers import TOL, oracle_scan, rel_err, scan_on_gpu, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def check(inp, chunk=128, y_dtype=torch.bfloat16, heads=None, initial_state=True,
+          use_D=True, inplace=False, varlen=None):
+    y, hT = scan_on_gpu(inp, chunk=chunk, y_dtype=y_dtype, initial_state=initial_state,
+                        use_D=use_D, inplace=inplace, varlen=varlen)
+    y_ref, h_ref = oracle_scan(inp, heads=heads, use_D=use_D, initial_state=initial_state)
+    yg, hg = to_np(y), to_np(hT)
+    if heads is not None:
+        yg, hg = yg[:, heads], hg[:, heads]
+    ey = rel_err(yg, y_ref, bf16=y_dtype == torch.bfloat16)
+    eh = rel_err(hg, h_ref)
+    # per (sequence, head) slice of the final state
+    ehs = max(rel_err(hg[s, k], h_ref[s, k]) for s in range(hg.shape[0]) for k in range(hg.shape[1])
+              if np.abs(h_ref[s, k]).max() > 0)
+    return ey, eh, ehs
+
+
+def test_tiny_f32_workload():
+    w = synth.WORKLOADS["tiny_f32"]
+    inp = synth.make_scan_inputs(synth.workload_seed("tiny_f32"), w["seqlens"], w["nheads"],
+                                 w["head_dim"], w["d_state"], w["ngroups"], dtype="f32")
+    ey, eh, ehs = check(inp, chunk=w["chunk"], y_dtype=torch.float32)
+    assert ey < 1e-4 and eh < 1e-4, (ey, eh)
+
+
+@pytest.mark.parametrize("seqlens,H,P,N,G,chunk", [
+    ([300], 4, 16, 16, 1, 64),
+    ([257, 128], 4, 32, 64, 2, 128),
+    ([1, 129], 2, 64, 128, 1, 128),
+    ([640], 8, 64, 128, 2, 128),
+    ([400, 3, 0, 200], 8, 64, 128, 4, 128),
+    ([333], 4, 128, 128, 2, 64),
+    ([200], 2, 64, 32, 1, 128),
+])
+@pytest.mark.parametrize("dtype,y_dtype", [("bf16", torch.bfloat16), ("bf16", torch.float32),
+                                           ("f32", torch.float32)])
+def test_scan_small_shapes(seqlens, H, P, N, G, chunk, dtype, y_dtype):
+    inp = synth.make_scan_inputs(sum(seqlens) + H * 3 + P, seqlens, H, P, N, G, dtype=dtype,
+                                 init_state=True)
+    ey, eh, ehs = check(inp, chunk=chunk, y_dtype=y_dtype)
+    assert ey < TOL and eh < TOL and ehs < 10 * TOL, (ey, eh, ehs)
+
+
+def test_scan_zero_initial_state_and_no_D():
+    inp = synth.make_scan_inputs(11, [384], 8, 64, 128, 2, dtype="bf16", init_state=True)
+    ey, eh, _ = check(inp, initial_state=False, use_D=False, y_dtype=torch.float32)
+    assert ey < TOL and eh < TOL, (ey, eh)
+
+
+def test_scan_in_place_state():
+    inp = synth.make_scan_inputs(12, [256, 300], 8, 64, 128, 2, dtype="bf16", init_state=True)
+    ey, eh, _ = check(inp, inplace=True, y_dtype=torch.float32)
+    assert ey < TOL and eh < TOL, (ey, eh)
+
+
+def test_scan_empty_sequences_keep_initial_state():
+    inp = synth.make_scan_inputs(13, [0, 0], 4, 64, 128, 1, dtype="bf16", init_state=True)
+    y, hT = scan_on_gpu(inp, varlen=True)
+    np.testing.assert_array_equal(to_np(hT), inp.h0.astype(np.float64))
+
+
+def test_bad_cu_seqlens_reported_on_device():
+    from hybrid_mamba_ssm_b200 import ssm
+    inp = synth.make_scan_inputs(14, [100, 60], 4, 64, 128, 1, dtype="bf16")
+    from tests.gpu_helpers import dev_f32, dev_tensor
+    cu = torch.tensor([0, 120, 160], dtype=torch.int32, device="cuda")   # sums to 160, T=160
+    bad = torch.tensor([0, 170, 160], dtype=torch.int32, device="cuda")  # decreasing
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    args = (dev_tensor(inp.x), dev_f32(inp.dt), dev_f32(inp.A), dev_tensor(inp.B),
+            dev_tensor(inp.C), dev_f32(inp.D))
+    ssm.ssd_chunk_scan(*args, cu_seqlens=cu, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ssm.ssd_chunk_scan(*args, cu_seqlens=bad, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 6
