@@ -1,0 +1,89 @@
+"""Small, self-contained launches of each kernel for profiling (ncu).
+
+    python -m hybrid_mamba_ssm_b200.profile_cases prefill --nseq 1 --seqlen 4096 --heads 128
+    python -m hybrid_mamba_ssm_b200.profile_cases decode --batch 16 --heads 256
+
+Each case draws seeded inputs, runs ``--warmup`` untimed launches and then
+``--launches`` more, and prints the device time of the last ones.  Inputs are
+sized by the flags; the defaults keep the working set above the 126 MB L2 while
+holding only a few hundred MB on the device.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import numpy as np
+import torch
+
+from . import inputs as synth
+from . import ssm
+
+
+def _bf16(t, dev):
+    return torch.from_numpy(np.ascontiguousarray(t.bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def _f32(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+
+
+def prefill(args, dev):
+    inp = synth.make_scan_inputs(77, [args.seqlen] * args.nseq, args.heads, args.head_dim,
+                                 args.d_state, args.groups, dtype="bf16")
+    n, L = args.nseq, args.seqlen
+    x = _bf16(inp.x, dev).view(n, L, args.heads, args.head_dim)
+    dt = _f32(inp.dt, dev).view(n, L, args.heads)
+    B = _bf16(inp.B, dev).view(n, L, args.groups, args.d_state)
+    C = _bf16(inp.C, dev).view(n, L, args.groups, args.d_state)
+    A, D = _f32(inp.A, dev), _f32(inp.D, dev)
+    y = torch.empty_like(x)
+    hT = torch.empty((n, args.heads, args.head_dim, args.d_state), dtype=torch.float32, device=dev)
+    return lambda: ssm.ssd_chunk_scan(x, dt, A, B, C, D, None, chunk_size=args.chunk, y=y,
+                                      final_state=hT)
+
+
+def decode(args, dev):
+    b, H, P, N, G = args.batch, args.heads, args.head_dim, args.d_state, args.groups
+    A, D = synth.make_head_params(78, H)
+    A, D = _f32(A, dev), _f32(D, dev)
+    state = _f32(synth.make_state(79, (b, H, P, N)), dev)
+    s = synth.make_decode_step(80, b, H, P, N, G)
+    x, dt, Bt, Ct = _bf16(s.x, dev), _f32(s.dt, dev), _bf16(s.B, dev), _bf16(s.C, dev)
+    y = torch.empty((b, H, P), dtype=torch.bfloat16, device=dev)
+    return lambda: ssm.ssm_state_update(state, x, dt, A, Bt, Ct, D, y=y)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["prefill", "decode"])
+    ap.add_argument("--nseq", type=int, default=1)
+    ap.add_argument("--seqlen", type=int, default=4096)
+    ap.add_argument("--batch", type=int, default=16)
+    ap.add_argument("--heads", type=int, default=None)
+    ap.add_argument("--head-dim", type=int, default=64)
+    ap.add_argument("--d-state", type=int, default=128)
+    ap.add_argument("--groups", type=int, default=8)
+    ap.add_argument("--chunk", type=int, default=128)
+    ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--launches", type=int, default=1)
+    args = ap.parse_args()
+    if args.heads is None:
+        args.heads = 128 if args.case == "prefill" else 256
+    dev = torch.device("cuda", 0)
+    run = prefill(args, dev) if args.case == "prefill" else decode(args, dev)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.launches):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"case": args.case, "ms_per_launch": s.elapsed_time(e) / args.launches,
+                      "args": vars(args)}))
+
+
+if __name__ == "__main__":
+    main()
