@@ -1,29 +1,49 @@
 // scan_tc.cu -- chunked SSD scan on the 5th-generation tensor cores
 // (tcgen05 MMAs with TMEM accumulators, operands staged by TMA).
 //
-// Covers bf16 x/B/C with head_dim 64, d_state 128 and 128-token chunks (the
-// Nemotron-H / Nemotron-3 Mamba-layer shape); other shapes run on the CUDA-core
-// kernel in scan_simt.cu.
+// Covers bf16 x/B/C with head_dim 64, d_state 128, 128-token chunks and an
+// even number of heads per group (the Nemotron-H / Nemotron-3 Mamba-layer
+// shapes); other shapes run on the CUDA-core kernel in scan_simt.cu.
 //
-// Per chunk of L <= 128 tokens of one (sequence, head), with group g, the
-// inclusive cumulative decay cs[i] = sum_{k<=i} dt_k A and the carried state H
-// ([head_dim, d_state], fp32), the chunked (state-space-duality) form of the
-// recurrence is four contractions and an elementwise state pass:
-//   G    = C B^T                          (128 x 128, K = d_state)     MMA
-//   M    = G o exp(cs_i - cs_j) dt_j [j<=i] (decay mask, fp16)          CUDA cores
-//   Y    = M X                            (128 x 64,  K = chunk)       MMA
-//   S^T  = B^T (w o X), w_j = exp(cs_L - cs_j) dt_j  (128 x 64, K = chunk)  MMA
-//   Yoff = C H^T                          (128 x 64,  K = d_state)     MMA
-//   y    = Y + exp(cs_i) Yoff + D x                                    epilogue
-//   H   <- exp(cs_L) H + S                                             epilogue
-// The diagonal j = i is part of M because the output reads the updated state.
+// Chunked (state-space-duality) form of the recurrence.  For one chunk of
+// L <= 128 tokens of one (sequence, head) with group g, cumulative decay
+// cs[i] = sum_{k<=i} dt_k A (inclusive, from the chunk start) and carried
+// state H ([head_dim, d_state], fp32):
+//   G    = C B^T                                   (shared by the group's heads)
+//   M    = G o exp(cs_i - cs_j) dt_j [j <= i]  + D I (decay mask; skip term on
+//                                                     the diagonal)
+//   Y    = M X
+//   S^T  = B^T (w o X),  w_j = exp(cs_{L-1} - cs_j) dt_j
+//   Yoff = C H^T
+//   y    = Y + exp(cs_i) Yoff,   H <- exp(cs_{L-1}) H + S
+// The diagonal j = i belongs to M because the output reads the updated state.
 //
-// One CTA of 128 threads per (sequence, head); thread i owns TMEM lane i, i.e.
-// row i of G / Y / Yoff and d_state index i of S^T and of the carried state,
-// which stays in registers (fp32) for the whole sequence.  B, C and x arrive
-// by TMA in 128-byte-swizzled tiles; bf16 operands are converted in place to
-// fp16 so that the derived operands (M, w o X, H) keep 11 significant bits and
-// every MMA is fp16 x fp16 -> fp32.
+// Work decomposition: one CTA per (sequence, pair of heads of one group),
+// sweeping the sequence's chunks in order.  256 threads = two warpgroups; the
+// warpgroup wg owns head 2k+wg: thread i of it owns TMEM lane i (row i of G,
+// M, Y, Yoff; d_state index i of S^T and of the carried state, which lives in
+// 64 fp32 registers for the whole sequence).  Thread 0 issues TMA and MMAs.
+//
+// Pipeline per chunk (single-buffered tiles, with prefetch where a buffer
+// frees early):
+//   cumsum / decay tables -> wait TMA(x), TMA(B, C) -> convert bf16 -> fp16
+//   (C rows by warpgroup 0, B rows by warpgroup 1, x and w o x per head)
+//   -> issue TMA(x of next chunk) into the raw x buffers
+//   -> MMA S^T (2 heads), G  [commit] , Yoff (2 heads) [commit]
+//   -> decay mask M per head (overlaps the Yoff MMAs)
+//   -> issue TMA(B, C of next chunk); MMA Y (2 heads) [commit]
+//   -> state update from S^T (overlaps the Y MMAs) -> epilogue y.
+//
+// Precision: bf16 inputs are converted to fp16 (exact for |v| < 65504) so the
+// derived operands M, w o x and H (rounded to fp16, 11 significant bits) keep
+// the result within ~3e-4 of the fp64 recurrence; accumulation is fp32.
+//
+// Decay factors are never ratios of exponentials.  With block ends r_K =
+// 32K+31, exp(cs_i - cs_j) = exp(cs_i - cs_{r_I}) exp(cs_{r_I} - cs_{r_J})
+// exp(cs_{r_J} - cs_j) for i in block I >= J >= j's block: the last two
+// factors are <= 1, the first is >= 1 but bounded by the decay over one
+// 32-token block; if that exceeds e^80 the block uses exp(cs_i - cs_j) per
+// element instead.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -36,37 +56,38 @@ namespace {
 constexpr int kQ = 128;       // chunk length
 constexpr int kP = 64;        // head_dim
 constexpr int kN = 128;       // d_state
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 
-// Shared memory (bytes from a 1024-aligned base).  16-bit tiles are stored in
-// the 128B-swizzled layout TMA writes and the MMA descriptors expect: rows of
-// 64 elements (128 bytes), 8-row groups of 1024 bytes, the 16-byte chunk c of
-// row r at position c ^ (r % 8).  Tiles 128 elements wide are two such
-// 64-column halves, 16 KB apart.
-constexpr uint32_t OFF_C = 0;          // C   [128 token i][128 n]
-constexpr uint32_t OFF_B = 32768;      // B   [128 token j][128 n]
-constexpr uint32_t OFF_X = 65536;      // X   [128 token j][64 p]
-constexpr uint32_t OFF_W = 81920;      // w o X [128 token j][64 p]
-constexpr uint32_t OFF_M = 98304;      // M   [128 i][128 j]
-constexpr uint32_t OFF_H = 131072;     // H^T [128 n][64 p]
-constexpr uint32_t OFF_CS = 147456;    // float[128] cumulative dt*A
-constexpr uint32_t OFF_DT = OFF_CS + 512;
-constexpr uint32_t OFF_WS = OFF_DT + 512;   // float[4] warp partial sums
-constexpr uint32_t OFF_BAR = OFF_WS + 64;   // two mbarriers
-constexpr uint32_t OFF_TM = OFF_BAR + 16;   // TMEM base address
-constexpr uint32_t SMEM_USED = OFF_TM + 16;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // + alignment slack
+// Shared memory (bytes from the 1024-aligned dynamic base).  16-bit tiles use
+// the 128B-swizzled layout TMA writes and the MMA descriptors read: rows of 64
+// elements (128 B), 8-row groups of 1024 B, 16-byte chunk c of row r stored at
+// c ^ (r % 8).  128-wide tiles are two 64-column halves 16 KB apart.
 constexpr uint32_t HALF = 16384;
-constexpr uint32_t TMA_BYTES = 2 * 2 * HALF + HALF;  // C, B (two halves each), X
+constexpr uint32_t OFF_C = 0;            // C [128 i][128 n]  (bf16 -> fp16 in place)
+constexpr uint32_t OFF_B = 32768;        // B [128 j][128 n]  (bf16 -> fp16 in place)
+constexpr uint32_t OFF_XR = 65536;       // raw x, 2 heads x [128 j][64 p] bf16 (TMA target)
+constexpr uint32_t OFF_XH = 98304;       // x as fp16, 2 heads
+constexpr uint32_t OFF_WM = 131072;      // w o x (2 heads), later M of head 0 [128][128]
+constexpr uint32_t OFF_MB = 163840;      // M of head 1
+constexpr uint32_t OFF_H = 196608;       // H^T fp16, 2 heads x [128 n][64 p]
+constexpr uint32_t OFF_MISC = 229376;
+constexpr uint32_t OFF_VD = OFF_MISC;              // float[2][128]
+constexpr uint32_t OFF_CSB = OFF_VD + 1024;        // float[2][8]: block-end cs, cs_last
+constexpr uint32_t OFF_PART = OFF_CSB + 64;        // float[2][4] warp partial sums
+constexpr uint32_t OFF_BAR = OFF_PART + 32;        // 5 mbarriers
+constexpr uint32_t OFF_TM = OFF_BAR + 40;
+constexpr uint32_t SMEM_BYTES = OFF_TM + 16;
 
 // TMEM columns (fp32 accumulators, lane = row).
-constexpr uint32_t TM_G = 0, TM_S = 128, TM_YO = 192, TM_Y = 256;
+constexpr uint32_t TM_G = 0, TM_S = 128, TM_YO = 256, TM_Y = 384;
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_G = tc::idesc_f16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
 constexpr uint32_t IDESC_S = tc::idesc_f16_f32(128, 64, 1, 1);    // B^T (MN-major) x wX (MN-major)
 constexpr uint32_t IDESC_YO = tc::idesc_f16_f32(128, 64, 0, 1);   // C (K-major) x H^T (MN-major)
 constexpr uint32_t IDESC_Y = tc::idesc_f16_f32(128, 64, 0, 1);    // M (K-major) x X (MN-major)
+
+constexpr float kSafeBlockDecay = 80.f;   // max exp argument taken by the factorised path
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
@@ -84,10 +105,6 @@ __device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-__device__ __forceinline__ float2 h2_to_f2(uint32_t v) {
-    return __half22float2(*reinterpret_cast<__half2 *>(&v));
-}
-
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -95,9 +112,25 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ float4 lds128f(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};"
                  ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// Shared address of float element idx of warpgroup wg's 128-entry table at off.
+__device__ __forceinline__ uint32_t smem_offset_f(uint32_t sbase, uint32_t off, int wg, int idx) {
+    return sbase + off + (uint32_t)(wg * 128 + idx) * 4u;
+}
+
+__device__ __forceinline__ void wg_sync(int wg) {
+    asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory");
 }
 
 __device__ __forceinline__ void store_row(float *dst, const float (&v)[32]) {
@@ -122,8 +155,8 @@ __device__ __forceinline__ void store_row(__nv_bfloat16 *dst, const float (&v)[3
     }
 }
 
-// Write the carried state (this thread's d_state row, 64 values) as fp16 into
-// the H^T tile.
+// This thread's d_state row of the carried state (64 values) as fp16 into the
+// H^T tile (MN-major operand: row n, p contiguous).
 __device__ __forceinline__ void write_state_tile(uint32_t sH, uint32_t n, const float (&Hs)[kP]) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -141,20 +174,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                const __grid_constant__ CUtensorMap map_c, const ScanArgs a)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = tc::smem_u32(smem);
-    float *sCS = reinterpret_cast<float *>(smem + OFF_CS);
-    float *sDT = reinterpret_cast<float *>(smem + OFF_DT);
-    float *sWS = reinterpret_cast<float *>(smem + OFF_WS);
-    const uint32_t bar_tma = sbase + OFF_BAR, bar_mma = sbase + OFF_BAR + 8;
+    const int tid = threadIdx.x;
+    const int wg = tid >> 7;             // warpgroup = head slot of the pair
+    const int i = tid & 127;             // row / TMEM lane / d_state index
+    const int wq = i >> 5;               // warp within the warpgroup = 32-row block
+    const int lane = tid & 31;
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.nheads, G = a.ngroups;
-    const int s = blockIdx.x / H;
-    const int h = blockIdx.x - s * H;
-    const int g = h / (H / G);
+    const int hpg = H / G;
+    const int pairs = H >> 1;
+    const int s = blockIdx.x / pairs;
+    const int h0 = (blockIdx.x - s * pairs) * 2;
+    const int g = h0 / hpg;
+    const int hh = h0 + wg;              // this warpgroup's head
+
+    if (sbase & 1023u) {                 // the swizzled layouts need 1024-B alignment
+        if (tid == 0) report_status(a.status_dev, 5);
+        return;
+    }
 
     long t0, t1;
     if (a.cu_seqlens) {
@@ -169,215 +208,271 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         t0 = (long)s * a.seqlen; t1 = t0 + a.seqlen;
     }
 
-    if (warp == 0) {
+    float *sVD = reinterpret_cast<float *>(smem + OFF_VD) + wg * 128;
+    float *sCSB = reinterpret_cast<float *>(smem + OFF_CSB) + wg * 8;
+    float *sPART = reinterpret_cast<float *>(smem + OFF_PART) + wg * 4;
+    const uint32_t bar_x = sbase + OFF_BAR, bar_cb = bar_x + 8, bar_sg = bar_x + 16;
+    const uint32_t bar_yo = bar_x + 24, bar_y = bar_x + 32;
+
+    if (tid < 32) {
         tc::tmem_alloc(sbase + OFF_TM, TM_COLS);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(bar_tma, 1);
-        tc::mbar_init(bar_mma, 1);
+        tc::mbar_init(bar_x, 1);
+        tc::mbar_init(bar_cb, 1);
+        tc::mbar_init(bar_sg, 1);
+        tc::mbar_init(bar_yo, 1);
+        tc::mbar_init(bar_y, 1);
         tc::fence_mbar_init();
     }
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_TM);
-    const uint32_t tlane = (uint32_t)(warp * 32) << 16;
+    const uint32_t tlane = (uint32_t)(wq * 32) << 16;
 
-    const size_t state_off = ((size_t)s * H + h) * (size_t)(kP * kN);
+    // first chunk's loads
+    if (tid == 0 && t1 > t0) {
+        tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
+        tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, h0, (int)t0);
+        tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, h0 + 1, (int)t0);
+        tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
+        tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)t0);
+        tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, g, (int)t0);
+        tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)t0);
+        tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)t0);
+    }
+
+    const size_t state_off = ((size_t)s * H + hh) * (size_t)(kP * kN);
     float Hs[kP];
 #pragma unroll
     for (int p = 0; p < kP; ++p)
-        Hs[p] = a.initial_state ? a.initial_state[state_off + (size_t)p * kN + tid] : 0.f;
-    write_state_tile(sbase + OFF_H, tid, Hs);
+        Hs[p] = a.initial_state ? a.initial_state[state_off + (size_t)p * kN + i] : 0.f;
+    write_state_tile(sbase + OFF_H + wg * HALF, i, Hs);
+
+    const float Ah = a.A[hh];
+    const float Dh = a.D ? a.D[hh] : 0.f;
+    TOut *y = static_cast<TOut *>(a.y);
+    float dt_next = (t0 + i < t1) ? a.dt[(size_t)(t0 + i) * H + hh] : 0.f;
+    bool ok = true;
+    uint32_t phase = 0;
     tc::fence_proxy_async_smem();
     __syncthreads();
 
-    const float Ah = a.A[h];
-    const float Dh = a.D ? a.D[h] : 0.f;
-    TOut *y = static_cast<TOut *>(a.y);
-    bool ok = true;
-    uint32_t ph_tma = 0, ph_mma = 0;
-
-    for (long c0 = t0; c0 < t1; c0 += kQ) {
+    for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u) {
         const int Lc = (int)min((long)kQ, t1 - c0);
-        if (tid == 0) {
-            tc::mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
-            tc::tma_load_3d(sbase + OFF_C, &map_c, bar_tma, 0, g, (int)c0);
-            tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_tma, 64, g, (int)c0);
-            tc::tma_load_3d(sbase + OFF_B, &map_b, bar_tma, 0, g, (int)c0);
-            tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_tma, 64, g, (int)c0);
-            tc::tma_load_3d(sbase + OFF_X, &map_x, bar_tma, 0, h, (int)c0);
-        }
+        const long c1 = c0 + kQ;
+        const bool has_next = c1 < t1;
+        const bool live = i < Lc;
 
-        // ---- decay: inclusive cumulative sum of dt*A over the chunk ----
-        const bool live = tid < Lc;
-        const float dtv = live ? a.dt[(size_t)(c0 + tid) * H + h] : 0.f;
+        // ---- cumulative decay of this warpgroup's head ----
+        const float dtv = dt_next;
+        dt_next = (has_next && c1 + i < t1) ? a.dt[(size_t)(c1 + i) * H + hh] : 0.f;
         float v = dtv * Ah;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const float u = __shfl_up_sync(0xffffffffu, v, o);
             if (lane >= o) v += u;
         }
-        if (lane == 31) sWS[warp] = v;
-        __syncthreads();
+        if (lane == 31) sPART[wq] = v;
+        wg_sync(wg);
         float pre = 0.f;
-        for (int w = 0; w < warp; ++w) pre += sWS[w];
-        const float cs_i = v + pre;
-        sCS[tid] = cs_i;
-        sDT[tid] = dtv;
-        __syncthreads();
-        const float cs_last = sCS[Lc - 1];
-        const float w_i = live ? expf(cs_last - cs_i) * dtv : 0.f;
+        for (int w = 0; w < wq; ++w) pre += sPART[w];
+        const float cs = v + pre;
+        if (lane == 31) sCSB[wq] = cs;
+        if (i == Lc - 1) sCSB[4] = cs;
+        wg_sync(wg);
+        const float cs_last = sCSB[4];
+        float cs_end[4];
+#pragma unroll
+        for (int K = 0; K < 4; ++K) cs_end[K] = sCSB[K];
+        const float cs_own_end = sCSB[wq];
+        const bool block_safe = (__shfl_sync(0xffffffffu, cs, 0) - cs_own_end) <= kSafeBlockDecay;
+        // ua[K] = exp(cs_i - cs_{r_K}): <= 1 for K < wq; for K = wq it is >= 1 and
+        // only used when the block's own decay is bounded (block_safe).
+        float ua[4];
+#pragma unroll
+        for (int K = 0; K < 4; ++K) ua[K] = (K <= wq) ? expf(cs - cs_end[K]) : 0.f;
+        sVD[i] = expf(cs_own_end - cs) * dtv;                  // <= dt
+        const float w_i = live ? expf(cs_last - cs) * dtv : 0.f;
+        const float e_i = expf(cs);
+        const float a_last = expf(cs_last);
 
-        // ---- operands: bf16 -> fp16 in place, w o X, rows past the end zeroed ----
-        tc::mbar_wait_bounded(bar_tma, ph_tma, ok);
-        ph_tma ^= 1;
+        // ---- operands to fp16 (rows past the chunk end zeroed) ----
+        tc::mbar_wait_bounded(bar_x, phase, ok);
+        tc::mbar_wait_bounded(bar_cb, phase, ok);
         {
             const float keep = live ? 1.f : 0.f;
+            const uint32_t tile = sbase + (wg == 0 ? OFF_C : OFF_B);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint32_t off = half * HALF + sw128(tid, k);
-                    uint4 c = lds128(sbase + OFF_C + off);
-                    uint4 b = lds128(sbase + OFF_B + off);
-                    c = make_uint4(bf2_to_h2(c.x, keep), bf2_to_h2(c.y, keep),
-                                   bf2_to_h2(c.z, keep), bf2_to_h2(c.w, keep));
-                    b = make_uint4(bf2_to_h2(b.x, keep), bf2_to_h2(b.y, keep),
-                                   bf2_to_h2(b.z, keep), bf2_to_h2(b.w, keep));
-                    sts128(sbase + OFF_C + off, c);
-                    sts128(sbase + OFF_B + off, b);
+                    const uint32_t addr = tile + half * HALF + sw128(i, k);
+                    const uint4 r = lds128(addr);
+                    sts128(addr, make_uint4(bf2_to_h2(r.x, keep), bf2_to_h2(r.y, keep),
+                                            bf2_to_h2(r.z, keep), bf2_to_h2(r.w, keep)));
                 }
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
-                const uint32_t off = sw128(tid, k);
-                const uint4 xr = lds128(sbase + OFF_X + off);
-                const uint4 xh = make_uint4(bf2_to_h2(xr.x, keep), bf2_to_h2(xr.y, keep),
-                                            bf2_to_h2(xr.z, keep), bf2_to_h2(xr.w, keep));
-                const uint4 wx = make_uint4(bf2_to_h2(xr.x, w_i), bf2_to_h2(xr.y, w_i),
-                                            bf2_to_h2(xr.z, w_i), bf2_to_h2(xr.w, w_i));
-                sts128(sbase + OFF_X + off, xh);
-                sts128(sbase + OFF_W + off, wx);
+                const uint32_t off = wg * HALF + sw128(i, k);
+                const uint4 r = lds128(sbase + OFF_XR + off);
+                sts128(sbase + OFF_XH + off, make_uint4(bf2_to_h2(r.x, keep), bf2_to_h2(r.y, keep),
+                                                        bf2_to_h2(r.z, keep), bf2_to_h2(r.w, keep)));
+                sts128(sbase + OFF_WM + off, make_uint4(bf2_to_h2(r.x, w_i), bf2_to_h2(r.y, w_i),
+                                                        bf2_to_h2(r.z, w_i), bf2_to_h2(r.w, w_i)));
             }
         }
         tc::fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- G = C B^T,  S^T = B^T (w o X),  Yoff = C H^T ----
         if (tid == 0) {
+            // raw x is consumed: prefetch the next chunk's x
+            if (has_next) {
+                tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
+                tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, h0, (int)c1);
+                tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, h0 + 1, (int)c1);
+            }
             tc::tc_fence_after();
+#pragma unroll
+            for (int hd = 0; hd < 2; ++hd) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ss(tmem + TM_S + hd * 64,
+                                   tc::sdesc_sw128(sbase + OFF_B + kk * 2048, HALF, 1024),
+                                   tc::sdesc_sw128(sbase + OFF_WM + hd * HALF + kk * 2048, HALF, 1024),
+                                   IDESC_S, kk > 0);
+            }
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
                 tc::mma_f16_ss(tmem + TM_G, tc::sdesc_sw128(sbase + OFF_C + koff, 16, 1024),
                                tc::sdesc_sw128(sbase + OFF_B + koff, 16, 1024), IDESC_G, kk > 0);
             }
+            tc::mma_commit(bar_sg);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                tc::mma_f16_ss(tmem + TM_S, tc::sdesc_sw128(sbase + OFF_B + kk * 2048, HALF, 1024),
-                               tc::sdesc_sw128(sbase + OFF_W + kk * 2048, HALF, 1024), IDESC_S, kk > 0);
-            }
+            for (int hd = 0; hd < 2; ++hd) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-                tc::mma_f16_ss(tmem + TM_YO, tc::sdesc_sw128(sbase + OFF_C + koff, 16, 1024),
-                               tc::sdesc_sw128(sbase + OFF_H + kk * 2048, HALF, 1024), IDESC_YO, kk > 0);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
+                    tc::mma_f16_ss(tmem + TM_YO + hd * 64,
+                                   tc::sdesc_sw128(sbase + OFF_C + koff, 16, 1024),
+                                   tc::sdesc_sw128(sbase + OFF_H + hd * HALF + kk * 2048, HALF, 1024),
+                                   IDESC_YO, kk > 0);
+                }
             }
-            tc::mma_commit(bar_mma);
+            tc::mma_commit(bar_yo);
         }
         __syncwarp();
-        tc::mbar_wait_bounded(bar_mma, ph_mma, ok);
-        ph_mma ^= 1;
-        tc::tc_fence_after();
 
-        // ---- M = G o exp(cs_i - cs_j) dt_j for j <= i (row i = tid) ----
+        // ---- decay mask M of this warpgroup's head (row i) ----
+        tc::mbar_wait_bounded(bar_sg, phase, ok);
+        tc::tc_fence_after();
+        {
+            const uint32_t mtile = sbase + (wg == 0 ? OFF_WM : OFF_MB);
 #pragma unroll
-        for (int jc = 0; jc < 4; ++jc) {
-            const uint32_t mrow = sbase + OFF_M + (jc >> 1) * HALF;
-            if (jc <= warp) {
-                uint32_t r[32];
-                tc::tmem_ld32(tmem + tlane + TM_G + jc * 32, r);
-                tc::tmem_ld_wait();
+            for (int jc = 0; jc < 4; ++jc) {
+                const uint32_t mrow = mtile + (jc >> 1) * HALF;
+                if (jc <= wq) {
+                    uint32_t r[32];
+                    tc::tmem_ld32(tmem + tlane + TM_G + jc * 32, r);
+                    tc::tmem_ld_wait();
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float m[8];
+                    for (int q = 0; q < 4; ++q) {
+                        const float4 vd0 = lds128f(smem_offset_f(sbase, OFF_VD, wg, jc * 32 + q * 8));
+                        const float4 vd1 = lds128f(smem_offset_f(sbase, OFF_VD, wg, jc * 32 + q * 8 + 4));
+                        const float vd[8] = {vd0.x, vd0.y, vd0.z, vd0.w, vd1.x, vd1.y, vd1.z, vd1.w};
+                        float m[8];
+                        if (jc < wq) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = jc * 32 + q * 8 + e;
-                        m[e] = (j <= tid) ? __uint_as_float(r[q * 8 + e]) * expf(cs_i - sCS[j]) * sDT[j]
-                                          : 0.f;
+                            for (int e = 0; e < 8; ++e)
+                                m[e] = __uint_as_float(r[q * 8 + e]) * ua[jc] * vd[e];
+                        } else if (block_safe) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int jl = q * 8 + e;   // column within the diagonal block
+                                float mv = (jl <= lane) ? __uint_as_float(r[jl]) * ua[jc] * vd[e] : 0.f;
+                                m[e] = (jl == lane) ? mv + Dh : mv;
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int jl = q * 8 + e;
+                                const float csj = __shfl_sync(0xffffffffu, cs, jl);
+                                const float dtj = __shfl_sync(0xffffffffu, dtv, jl);
+                                float mv = (jl <= lane) ? __uint_as_float(r[jl]) * expf(cs - csj) * dtj : 0.f;
+                                m[e] = (jl == lane) ? mv + Dh : mv;
+                            }
+                        }
+                        sts128(mrow + sw128(i, (jc & 1) * 4 + q),
+                               make_uint4(f2_to_h2(m[0], m[1]), f2_to_h2(m[2], m[3]),
+                                          f2_to_h2(m[4], m[5]), f2_to_h2(m[6], m[7])));
                     }
-                    const uint4 u = make_uint4(f2_to_h2(m[0], m[1]), f2_to_h2(m[2], m[3]),
-                                               f2_to_h2(m[4], m[5]), f2_to_h2(m[6], m[7]));
-                    sts128(mrow + sw128(tid, (jc & 1) * 4 + q), u);
-                }
-            } else {
+                } else {
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    sts128(mrow + sw128(tid, (jc & 1) * 4 + q), make_uint4(0, 0, 0, 0));
+                    for (int q = 0; q < 4; ++q)
+                        sts128(mrow + sw128(i, (jc & 1) * 4 + q), make_uint4(0, 0, 0, 0));
+                }
             }
         }
         tc::fence_proxy_async_smem();
+        tc::mbar_wait_bounded(bar_yo, phase, ok);   // Yoff done: C, B and H^T tiles are free
         tc::tc_fence_before();
         __syncthreads();
 
-        // ---- Y = M X ----
         if (tid == 0) {
+            if (has_next) {
+                tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
+                tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)c1);
+                tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, g, (int)c1);
+                tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)c1);
+                tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)c1);
+            }
             tc::tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-                tc::mma_f16_ss(tmem + TM_Y, tc::sdesc_sw128(sbase + OFF_M + koff, 16, 1024),
-                               tc::sdesc_sw128(sbase + OFF_X + kk * 2048, HALF, 1024), IDESC_Y, kk > 0);
+            for (int hd = 0; hd < 2; ++hd) {
+                const uint32_t mt = sbase + (hd == 0 ? OFF_WM : OFF_MB);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
+                    tc::mma_f16_ss(tmem + TM_Y + hd * 64, tc::sdesc_sw128(mt + koff, 16, 1024),
+                                   tc::sdesc_sw128(sbase + OFF_XH + hd * HALF + kk * 2048, HALF, 1024),
+                                   IDESC_Y, kk > 0);
+                }
             }
-            tc::mma_commit(bar_mma);
+            tc::mma_commit(bar_y);
         }
         __syncwarp();
 
-        // ---- carried state: H <- exp(cs_L) H + S  (this thread: d_state row tid) ----
-        {
-            const float a_last = expf(cs_last);
+        // ---- carried state: H <- exp(cs_L) H + S (d_state row i) ----
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[32];
-                tc::tmem_ld32(tmem + tlane + TM_S + half * 32, r);
-                tc::tmem_ld_wait();
+        for (int half = 0; half < 2; ++half) {
+            uint32_t r[32];
+            tc::tmem_ld32(tmem + tlane + TM_S + wg * 64 + half * 32, r);
+            tc::tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    Hs[half * 32 + e] = fmaf(a_last, Hs[half * 32 + e], __uint_as_float(r[e]));
-            }
-            write_state_tile(sbase + OFF_H, tid, Hs);
+            for (int e = 0; e < 32; ++e)
+                Hs[half * 32 + e] = fmaf(a_last, Hs[half * 32 + e], __uint_as_float(r[e]));
         }
+        write_state_tile(sbase + OFF_H + wg * HALF, i, Hs);
 
-        tc::mbar_wait_bounded(bar_mma, ph_mma, ok);
-        ph_mma ^= 1;
+        // ---- y = Y + exp(cs_i) Yoff (row i; D x is inside Y) ----
+        tc::mbar_wait_bounded(bar_y, phase, ok);
         tc::tc_fence_after();
-
-        // ---- y = Y + exp(cs_i) Yoff + D x  (row i = tid) ----
         {
-            const float e_i = expf(cs_i);
-            TOut *yrow = y + ((size_t)(c0 + tid) * H + h) * kP;
+            TOut *yrow = y + ((size_t)(c0 + i) * H + hh) * kP;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t ry[32], ro[32];
-                tc::tmem_ld32(tmem + tlane + TM_Y + half * 32, ry);
-                tc::tmem_ld32(tmem + tlane + TM_YO + half * 32, ro);
+                tc::tmem_ld32(tmem + tlane + TM_Y + wg * 64 + half * 32, ry);
+                tc::tmem_ld32(tmem + tlane + TM_YO + wg * 64 + half * 32, ro);
                 tc::tmem_ld_wait();
                 float out[32];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 xr = lds128(sbase + OFF_X + sw128(tid, half * 4 + q));
-                    const float2 x01 = h2_to_f2(xr.x), x23 = h2_to_f2(xr.y);
-                    const float2 x45 = h2_to_f2(xr.z), x67 = h2_to_f2(xr.w);
-                    const float xv[8] = {x01.x, x01.y, x23.x, x23.y, x45.x, x45.y, x67.x, x67.y};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int c = q * 8 + e;
-                        out[c] = fmaf(Dh, xv[e], fmaf(e_i, __uint_as_float(ro[c]), __uint_as_float(ry[c])));
-                    }
-                }
+                for (int c = 0; c < 32; ++c)
+                    out[c] = fmaf(e_i, __uint_as_float(ro[c]), __uint_as_float(ry[c]));
                 if (live) store_row(yrow + half * 32, out);
             }
         }
@@ -389,15 +484,15 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     if (a.final_state) {
 #pragma unroll
         for (int p = 0; p < kP; ++p)
-            a.final_state[state_off + (size_t)p * kN + tid] = Hs[p];
+            a.final_state[state_off + (size_t)p * kN + i] = Hs[p];
     }
     tc::tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (tid < 32) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, TM_COLS);
     }
-    if (!ok && tid == 0) report_status(a.status_dev, 5);
+    if (!ok && i == 0) report_status(a.status_dev, 5);
 }
 
 // ------------------------------------------------------------------ host side
@@ -445,7 +540,7 @@ cudaError_t launch_tc_t(const ScanArgs &a, cudaStream_t stream)
     cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<TOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((size_t)a.nseq * a.nheads));
+    dim3 grid((unsigned)((size_t)a.nseq * (a.nheads / 2)));
     scan_tc_kernel<TOut><<<grid, kThreads, SMEM_BYTES, stream>>>(mx, mb, mc, a);
     return cudaGetLastError();
 }
@@ -456,7 +551,7 @@ bool scan_tc_supports(const ScanArgs &a)
 {
     const long long T = a.cu_seqlens ? (long long)a.seqlen : (long long)a.nseq * a.seqlen;
     return a.in_dtype == 1 && a.head_dim == kP && a.d_state == kN && a.chunk_size == kQ &&
-           T > 0 && encode_fn() != nullptr;
+           (a.nheads / a.ngroups) % 2 == 0 && T > 0 && encode_fn() != nullptr;
 }
 
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t stream)
