@@ -19,10 +19,13 @@
 // The diagonal j = i belongs to M because the output reads the updated state.
 //
 // Work decomposition: one CTA per (sequence, pair of heads of one group),
-// sweeping the sequence's chunks in order.  256 threads = two warpgroups; the
-// warpgroup wg owns head 2k+wg: thread i of it owns TMEM lane i (row i of G,
-// M, Y, Yoff; d_state index i of S^T and of the carried state, which lives in
-// 64 fp32 registers for the whole sequence).  Thread 0 issues TMA and MMAs.
+// sweeping the sequence's chunks in order.  512 threads = four warpgroups;
+// warpgroup wg works on head 2k + (wg & 1) and on half (wg >> 1) of the
+// columns: thread i of it owns TMEM lane i (row i of G, M, Y, Yoff; d_state
+// index i of S^T and of the carried state, 32 of whose 64 head_dim entries it
+// keeps in fp32 registers for the whole sequence).  Thread 0 issues TMA and
+// the MMAs; the products shared by both heads (C.B^T, and B^T or C against the
+// two heads' operands side by side) are single N = 128 MMAs.
 //
 // Pipeline per chunk (single-buffered tiles, with prefetch where a buffer
 // frees early):
@@ -56,7 +59,7 @@ namespace {
 constexpr int kQ = 128;       // chunk length
 constexpr int kP = 64;        // head_dim
 constexpr int kN = 128;       // d_state
-constexpr int kThreads = 256;
+constexpr int kThreads = 544;   // 16 compute warps + 1 issuing warp
 
 // Shared memory (bytes from the 1024-aligned dynamic base).  16-bit tiles use
 // the 128B-swizzled layout TMA writes and the MMA descriptors read: rows of 64
@@ -71,10 +74,10 @@ constexpr uint32_t OFF_WM = 131072;      // w o x (2 heads), later M of head 0 [
 constexpr uint32_t OFF_MB = 163840;      // M of head 1
 constexpr uint32_t OFF_H = 196608;       // H^T fp16, 2 heads x [128 n][64 p]
 constexpr uint32_t OFF_MISC = 229376;
-constexpr uint32_t OFF_VD = OFF_MISC;              // float[2][128]
-constexpr uint32_t OFF_CSB = OFF_VD + 1024;        // float[2][8]: block-end cs, cs_last
-constexpr uint32_t OFF_PART = OFF_CSB + 64;        // float[2][4] warp partial sums
-constexpr uint32_t OFF_BAR = OFF_PART + 32;        // 5 mbarriers
+constexpr uint32_t OFF_VD = OFF_MISC;              // float[2 buffers][2 heads][128]
+constexpr uint32_t OFF_CSB = OFF_VD + 2048;        // float[4][8]: block-end cs, cs_last per warpgroup
+constexpr uint32_t OFF_PART = OFF_CSB + 128;       // float[4][4] warp partial sums
+constexpr uint32_t OFF_BAR = OFF_PART + 64;        // 5 mbarriers
 constexpr uint32_t OFF_TM = OFF_BAR + 40;
 constexpr uint32_t SMEM_BYTES = OFF_TM + 16;
 
@@ -83,8 +86,8 @@ constexpr uint32_t TM_G = 0, TM_S = 128, TM_YO = 256, TM_Y = 384;
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_G = tc::idesc_f16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
-constexpr uint32_t IDESC_S = tc::idesc_f16_f32(128, 64, 1, 1);    // B^T (MN-major) x wX (MN-major)
-constexpr uint32_t IDESC_YO = tc::idesc_f16_f32(128, 64, 0, 1);   // C (K-major) x H^T (MN-major)
+constexpr uint32_t IDESC_S2 = tc::idesc_f16_f32(128, 128, 1, 1);  // B^T (MN-major) x [wX_a|wX_b] (MN-major)
+constexpr uint32_t IDESC_YO2 = tc::idesc_f16_f32(128, 128, 0, 1); // C (K-major) x [H_a^T|H_b^T] (MN-major)
 constexpr uint32_t IDESC_Y = tc::idesc_f16_f32(128, 64, 0, 1);    // M (K-major) x X (MN-major)
 
 constexpr float kSafeBlockDecay = 80.f;   // max exp argument taken by the factorised path
@@ -112,72 +115,200 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ float4 lds128f(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-    return v;
-}
-
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};"
                  ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
-
-// Shared address of float element idx of warpgroup wg's 128-entry table at off.
-__device__ __forceinline__ uint32_t smem_offset_f(uint32_t sbase, uint32_t off, int wg, int idx) {
-    return sbase + off + (uint32_t)(wg * 128 + idx) * 4u;
 }
 
 __device__ __forceinline__ void wg_sync(int wg) {
     asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory");
 }
 
-__device__ __forceinline__ void store_row(float *dst, const float (&v)[32]) {
+__device__ __forceinline__ void store16(float *dst, const float (&v)[16]) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
+    for (int q = 0; q < 4; ++q)
         reinterpret_cast<float4 *>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
-__device__ __forceinline__ void store_row(__nv_bfloat16 *dst, const float (&v)[32]) {
+__device__ __forceinline__ void store16(__nv_bfloat16 *dst, const float (&v)[16]) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 u;
+    for (int q = 0; q < 2; ++q) {
         __nv_bfloat162 b0 = __floats2bfloat162_rn(v[8 * q + 0], v[8 * q + 1]);
         __nv_bfloat162 b1 = __floats2bfloat162_rn(v[8 * q + 2], v[8 * q + 3]);
         __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * q + 4], v[8 * q + 5]);
         __nv_bfloat162 b3 = __floats2bfloat162_rn(v[8 * q + 6], v[8 * q + 7]);
-        u.x = *reinterpret_cast<uint32_t *>(&b0);
-        u.y = *reinterpret_cast<uint32_t *>(&b1);
-        u.z = *reinterpret_cast<uint32_t *>(&b2);
-        u.w = *reinterpret_cast<uint32_t *>(&b3);
-        reinterpret_cast<uint4 *>(dst)[q] = u;
+        reinterpret_cast<uint4 *>(dst)[q] =
+            make_uint4(*reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
+                       *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
     }
 }
 
-// This thread's d_state row of the carried state (64 values) as fp16 into the
-// H^T tile (MN-major operand: row n, p contiguous).
-__device__ __forceinline__ void write_state_tile(uint32_t sH, uint32_t n, const float (&Hs)[kP]) {
+// bf16 pair -> fp16 pair (exact for |v| < 65504).
+__device__ __forceinline__ uint32_t bf2h(uint32_t v) {
+    return f2_to_h2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+__device__ __forceinline__ uint4 cvt_chunk(uint4 r) {
+    return make_uint4(bf2h(r.x), bf2h(r.y), bf2h(r.z), bf2h(r.w));
+}
+
+__device__ __forceinline__ uint4 cvt_chunk_scaled(uint4 r, float w) {
+    return make_uint4(bf2_to_h2(r.x, w), bf2_to_h2(r.y, w), bf2_to_h2(r.z, w), bf2_to_h2(r.w, w));
+}
+
+// 32 of this thread's d_state row of the carried state (p in [32 ch, 32 ch + 32))
+// as fp16 into the H^T tile (MN-major operand: row n, p contiguous).
+__device__ __forceinline__ void write_state_half(uint32_t sH, uint32_t n, int ch, const float (&Hs)[32]) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 4; ++k) {
         uint4 u;
         u.x = f2_to_h2(Hs[8 * k + 0], Hs[8 * k + 1]);
         u.y = f2_to_h2(Hs[8 * k + 2], Hs[8 * k + 3]);
         u.z = f2_to_h2(Hs[8 * k + 4], Hs[8 * k + 5]);
         u.w = f2_to_h2(Hs[8 * k + 6], Hs[8 * k + 7]);
-        sts128(sH + sw128(n, k), u);
+        sts128(sH + sw128(n, 4 * ch + k), u);
     }
 }
+
+// One 32-column block jc of row i of the decay mask M (fp16, K-major tile):
+//   off-diagonal (jc < wq):  G[i][j] * exp(cs_i - cs_{r_jc}) * vd[j]
+//   diagonal (jc == wq):     j <= i only, plus D on j == i
+//   above (jc > wq):         zeros
+// with vd[j] = exp(cs_{r_J} - cs_j) dt_j (J = j's block) from shared memory.
+__device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t mtile, const float *sVD,
+                                           int jc, int wq, int i, int lane, float ua,
+                                           bool block_safe, float cs, float dtv, float Dh)
+{
+    const uint32_t mrow = mtile + (jc >> 1) * HALF;
+    if (jc > wq) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sts128(mrow + sw128(i, (jc & 1) * 4 + q), make_uint4(0, 0, 0, 0));
+        return;
+    }
+    const float4 *vd4 = reinterpret_cast<const float4 *>(sVD + jc * 32);
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {   // 16 columns at a time
+        uint32_t r[16];
+        tc::tmem_ld16(g_taddr + jc * 32 + qq * 16, r);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+            const int q = qq * 2 + q2;   // 8-column chunk within the block
+            const float4 v0 = vd4[2 * q], v1 = vd4[2 * q + 1];
+            const float vd[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            float m[8];
+            if (jc < wq) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m[e] = __uint_as_float(r[q2 * 8 + e]) * ua * vd[e];
+            } else if (block_safe) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int jl = q * 8 + e;
+                    const float mv = (jl <= lane) ? __uint_as_float(r[q2 * 8 + e]) * ua * vd[e] : 0.f;
+                    m[e] = (jl == lane) ? mv + Dh : mv;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int jl = q * 8 + e;
+                    const float csj = __shfl_sync(0xffffffffu, cs, jl);
+                    const float dtj = __shfl_sync(0xffffffffu, dtv, jl);
+                    const float mv = (jl <= lane) ? __uint_as_float(r[q2 * 8 + e]) * expf(cs - csj) * dtj : 0.f;
+                    m[e] = (jl == lane) ? mv + Dh : mv;
+                }
+            }
+            sts128(mrow + sw128(i, (jc & 1) * 4 + q),
+                   make_uint4(f2_to_h2(m[0], m[1]), f2_to_h2(m[2], m[3]),
+                              f2_to_h2(m[4], m[5]), f2_to_h2(m[6], m[7])));
+        }
+    }
+}
+
+// 16 bf16 outputs of row i (two 16-byte chunks starting at chunk c) into the
+// y staging tile [128][64] (128B-swizzled, the box the y tensor map stores).
+__device__ __forceinline__ void stage16_bf16(uint32_t stage, int i, int c, const float (&v)[16]) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        __nv_bfloat162 b0 = __floats2bfloat162_rn(v[8 * q + 0], v[8 * q + 1]);
+        __nv_bfloat162 b1 = __floats2bfloat162_rn(v[8 * q + 2], v[8 * q + 3]);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * q + 4], v[8 * q + 5]);
+        __nv_bfloat162 b3 = __floats2bfloat162_rn(v[8 * q + 6], v[8 * q + 7]);
+        sts128(stage + sw128(i, c + q),
+               make_uint4(*reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
+                          *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3)));
+    }
+}
+
+// Per-chunk decay quantities of one head for this thread's row i.
+struct ChunkDecay {
+    float cs;        // inclusive cumulative dt*A at row i
+    float dtv;       // dt of row i (0 past the chunk end)
+    float uaA, uaB;  // exp(cs_i - cs_{r_K}) for this thread's two column blocks
+    float w;         // exp(cs_last - cs_i) dt_i   (weights of the chunk state)
+    float e;         // exp(cs_i)                  (decay of the carried state to row i)
+    float a_last;    // exp(cs_last)               (decay over the whole chunk)
+    bool safe;       // the row block's own decay fits the factorised path
+};
+
+// Cumulative decay of head hh over the chunk starting at c0 with Lc tokens
+// (warpgroup-wide), and this warpgroup's share of the column factors vd,
+// written to vd_out (only the warpgroup with ch == 0 writes).
+__device__ __forceinline__ ChunkDecay chunk_decay(const ScanArgs &a, int H, int hh, float Ah,
+                                                  long c0, int Lc, int i, int wq, int lane, int wg,
+                                                  int ch, float *sPART, float *sCSB, float *vd_out)
+{
+    ChunkDecay d;
+    d.dtv = (i < Lc) ? a.dt[(size_t)(c0 + i) * H + hh] : 0.f;
+    float v = d.dtv * Ah;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    if (lane == 31) sPART[wq] = v;
+    wg_sync(wg);
+    float pre = 0.f;
+    for (int w = 0; w < wq; ++w) pre += sPART[w];
+    d.cs = v + pre;
+    if (lane == 31) sCSB[wq] = d.cs;
+    if (i == Lc - 1) sCSB[4] = d.cs;
+    wg_sync(wg);
+    const float cs_last = sCSB[4];
+    const float cs_own_end = sCSB[wq];
+    d.safe = (__shfl_sync(0xffffffffu, d.cs, 0) - cs_own_end) <= kSafeBlockDecay;
+    const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
+    d.uaA = (kA <= wq) ? expf(d.cs - sCSB[kA]) : 0.f;
+    d.uaB = (kB <= wq) ? expf(d.cs - sCSB[kB]) : 0.f;
+    if (ch == 0) vd_out[i] = expf(cs_own_end - d.cs) * d.dtv;   // <= dt
+    d.w = (i < Lc) ? expf(cs_last - d.cs) * d.dtv : 0.f;
+    d.e = expf(d.cs);
+    d.a_last = expf(cs_last);
+    return d;
+}
+
+// Named barriers: 1..4 per-warpgroup; the compute warps signal the issuing
+// warp with bar.arrive on 5 (operands ready), 6 (decay mask ready) and 7 (y
+// staged); 8 is compute-warps-only.
+constexpr uint32_t BAR_OPERANDS = 5, BAR_MASK = 6, BAR_YSTAGED = 7, BAR_COMPUTE = 8;
+constexpr uint32_t kCompute = 512;
 
 template <typename TOut>
 __global__ void __launch_bounds__(kThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
-               const __grid_constant__ CUtensorMap map_c, const ScanArgs a)
+               const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y,
+               const ScanArgs a)
 {
+    // bf16 y of full chunks is staged in shared memory (the M tile of head 1,
+    // free between the y MMAs and the next chunk's mask) and written by TMA;
+    // fp32 y and partial chunks are stored row by row.
+    constexpr bool kStoreByTma = sizeof(TOut) == 2;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = tc::smem_u32(smem);
     const int tid = threadIdx.x;
-    const int wg = tid >> 7;             // warpgroup = head slot of the pair
+    const bool issuer = tid >= (int)kCompute;  // warp 16: TMA and MMA issue
+    const int wg = (tid >> 7) & 3;       // compute warpgroup 0..3
+    const int hd = wg & 1;               // head slot of the pair
+    const int ch = wg >> 1;              // column half
     const int i = tid & 127;             // row / TMEM lane / d_state index
     const int wq = i >> 5;               // warp within the warpgroup = 32-row block
     const int lane = tid & 31;
@@ -188,7 +319,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     const int s = blockIdx.x / pairs;
     const int h0 = (blockIdx.x - s * pairs) * 2;
     const int g = h0 / hpg;
-    const int hh = h0 + wg;              // this warpgroup's head
+    const int hh = h0 + hd;
 
     if (sbase & 1023u) {                 // the swizzled layouts need 1024-B alignment
         if (tid == 0) report_status(a.status_dev, 5);
@@ -208,7 +339,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         t0 = (long)s * a.seqlen; t1 = t0 + a.seqlen;
     }
 
-    float *sVD = reinterpret_cast<float *>(smem + OFF_VD) + wg * 128;
     float *sCSB = reinterpret_cast<float *>(smem + OFF_CSB) + wg * 8;
     float *sPART = reinterpret_cast<float *>(smem + OFF_PART) + wg * 4;
     const uint32_t bar_x = sbase + OFF_BAR, bar_cb = bar_x + 8, bar_sg = bar_x + 16;
@@ -230,261 +360,209 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_TM);
-    const uint32_t tlane = (uint32_t)(wq * 32) << 16;
-
-    // first chunk's loads
-    if (tid == 0 && t1 > t0) {
-        tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
-        tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, h0, (int)t0);
-        tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, h0 + 1, (int)t0);
-        tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
-        tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)t0);
-        tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, g, (int)t0);
-        tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)t0);
-        tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)t0);
-    }
-
-    const size_t state_off = ((size_t)s * H + hh) * (size_t)(kP * kN);
-    float Hs[kP];
-#pragma unroll
-    for (int p = 0; p < kP; ++p)
-        Hs[p] = a.initial_state ? a.initial_state[state_off + (size_t)p * kN + i] : 0.f;
-    write_state_tile(sbase + OFF_H + wg * HALF, i, Hs);
-
-    const float Ah = a.A[hh];
-    const float Dh = a.D ? a.D[hh] : 0.f;
-    TOut *y = static_cast<TOut *>(a.y);
-    float dt_next = (t0 + i < t1) ? a.dt[(size_t)(t0 + i) * H + hh] : 0.f;
     bool ok = true;
-    uint32_t phase = 0;
-    tc::fence_proxy_async_smem();
-    __syncthreads();
 
-    for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u) {
-        const int Lc = (int)min((long)kQ, t1 - c0);
-        const long c1 = c0 + kQ;
-        const bool has_next = c1 < t1;
-        const bool live = i < Lc;
-
-        // ---- cumulative decay of this warpgroup's head ----
-        const float dtv = dt_next;
-        dt_next = (has_next && c1 + i < t1) ? a.dt[(size_t)(c1 + i) * H + hh] : 0.f;
-        float v = dtv * Ah;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float u = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += u;
+    if (issuer) {
+        // ================= TMA / MMA issuing warp =================
+        const bool leader = lane == 0;
+        // descriptors (start-address field advanced by offset >> 4 per K step)
+        const uint64_t dBmn = tc::sdesc_sw128(sbase + OFF_B, HALF, 1024);   // B^T, MN-major
+        const uint64_t dW = tc::sdesc_sw128(sbase + OFF_WM, HALF, 1024);    // [wX_a | wX_b]
+        const uint64_t dCk = tc::sdesc_sw128(sbase + OFF_C, 16, 1024);      // C, K-major
+        const uint64_t dBk = tc::sdesc_sw128(sbase + OFF_B, 16, 1024);      // B, K-major
+        const uint64_t dH = tc::sdesc_sw128(sbase + OFF_H, HALF, 1024);     // [H_a^T | H_b^T]
+        const uint64_t dMa = tc::sdesc_sw128(sbase + OFF_WM, 16, 1024);
+        const uint64_t dMb = tc::sdesc_sw128(sbase + OFF_MB, 16, 1024);
+        const uint64_t dXa = tc::sdesc_sw128(sbase + OFF_XH, HALF, 1024);
+        const uint64_t dXb = dXa + (HALF >> 4);
+        if (leader && t1 > t0) {
+            tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
+            tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, h0, (int)t0);
+            tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, h0 + 1, (int)t0);
+            tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
+            tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)t0);
+            tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, g, (int)t0);
+            tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)t0);
+            tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)t0);
         }
-        if (lane == 31) sPART[wq] = v;
-        wg_sync(wg);
-        float pre = 0.f;
-        for (int w = 0; w < wq; ++w) pre += sPART[w];
-        const float cs = v + pre;
-        if (lane == 31) sCSB[wq] = cs;
-        if (i == Lc - 1) sCSB[4] = cs;
-        wg_sync(wg);
-        const float cs_last = sCSB[4];
-        float cs_end[4];
-#pragma unroll
-        for (int K = 0; K < 4; ++K) cs_end[K] = sCSB[K];
-        const float cs_own_end = sCSB[wq];
-        const bool block_safe = (__shfl_sync(0xffffffffu, cs, 0) - cs_own_end) <= kSafeBlockDecay;
-        // ua[K] = exp(cs_i - cs_{r_K}): <= 1 for K < wq; for K = wq it is >= 1 and
-        // only used when the block's own decay is bounded (block_safe).
-        float ua[4];
-#pragma unroll
-        for (int K = 0; K < 4; ++K) ua[K] = (K <= wq) ? expf(cs - cs_end[K]) : 0.f;
-        sVD[i] = expf(cs_own_end - cs) * dtv;                  // <= dt
-        const float w_i = live ? expf(cs_last - cs) * dtv : 0.f;
-        const float e_i = expf(cs);
-        const float a_last = expf(cs_last);
-
-        // ---- operands to fp16 (rows past the chunk end zeroed) ----
-        tc::mbar_wait_bounded(bar_x, phase, ok);
-        tc::mbar_wait_bounded(bar_cb, phase, ok);
-        {
-            const float keep = live ? 1.f : 0.f;
-            const uint32_t tile = sbase + (wg == 0 ? OFF_C : OFF_B);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t addr = tile + half * HALF + sw128(i, k);
-                    const uint4 r = lds128(addr);
-                    sts128(addr, make_uint4(bf2_to_h2(r.x, keep), bf2_to_h2(r.y, keep),
-                                            bf2_to_h2(r.z, keep), bf2_to_h2(r.w, keep)));
+        uint32_t phase = 0;
+        for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u) {
+            const long c1 = c0 + kQ;
+            const bool has_next = c1 < t1;
+            tc::named_sync(BAR_OPERANDS, kCompute + 32);
+            if (leader) {
+                tc::bulk_wait_read();   // previous y staging (in the M tiles) was read
+                if (has_next) {
+                    tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
+                    tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, h0, (int)c1);
+                    tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, h0 + 1, (int)c1);
                 }
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t off = wg * HALF + sw128(i, k);
-                const uint4 r = lds128(sbase + OFF_XR + off);
-                sts128(sbase + OFF_XH + off, make_uint4(bf2_to_h2(r.x, keep), bf2_to_h2(r.y, keep),
-                                                        bf2_to_h2(r.z, keep), bf2_to_h2(r.w, keep)));
-                sts128(sbase + OFF_WM + off, make_uint4(bf2_to_h2(r.x, w_i), bf2_to_h2(r.y, w_i),
-                                                        bf2_to_h2(r.z, w_i), bf2_to_h2(r.w, w_i)));
-            }
-        }
-        tc::fence_proxy_async_smem();
-        __syncthreads();
-
-        if (tid == 0) {
-            // raw x is consumed: prefetch the next chunk's x
-            if (has_next) {
-                tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
-                tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, h0, (int)c1);
-                tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, h0 + 1, (int)c1);
-            }
-            tc::tc_fence_after();
-#pragma unroll
-            for (int hd = 0; hd < 2; ++hd) {
+                tc::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16_ss(tmem + TM_S + hd * 64,
-                                   tc::sdesc_sw128(sbase + OFF_B + kk * 2048, HALF, 1024),
-                                   tc::sdesc_sw128(sbase + OFF_WM + hd * HALF + kk * 2048, HALF, 1024),
-                                   IDESC_S, kk > 0);
-            }
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-                tc::mma_f16_ss(tmem + TM_G, tc::sdesc_sw128(sbase + OFF_C + koff, 16, 1024),
-                               tc::sdesc_sw128(sbase + OFF_B + koff, 16, 1024), IDESC_G, kk > 0);
-            }
-            tc::mma_commit(bar_sg);
-#pragma unroll
-            for (int hd = 0; hd < 2; ++hd) {
+                    tc::mma_f16_ss(tmem + TM_S, dBmn + kk * 128, dW + kk * 128, IDESC_S2, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-                    tc::mma_f16_ss(tmem + TM_YO + hd * 64,
-                                   tc::sdesc_sw128(sbase + OFF_C + koff, 16, 1024),
-                                   tc::sdesc_sw128(sbase + OFF_H + hd * HALF + kk * 2048, HALF, 1024),
-                                   IDESC_YO, kk > 0);
+                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
+                    tc::mma_f16_ss(tmem + TM_G, dCk + ko, dBk + ko, IDESC_G, kk > 0);
                 }
+                tc::mma_commit(bar_sg);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
+                    tc::mma_f16_ss(tmem + TM_YO, dCk + ko, dH + kk * 128, IDESC_YO2, kk > 0);
+                }
+                tc::mma_commit(bar_yo);
             }
-            tc::mma_commit(bar_yo);
+            __syncwarp();
+            tc::named_sync(BAR_MASK, kCompute + 32);
+            if (leader) {
+                tc::mbar_wait_bounded(bar_yo, phase, ok);   // C and B tiles free
+                if (has_next) {
+                    tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
+                    tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)c1);
+                    tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, g, (int)c1);
+                    tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)c1);
+                    tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)c1);
+                }
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
+                    tc::mma_f16_ss(tmem + TM_Y, dMa + ko, dXa + kk * 128, IDESC_Y, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
+                    tc::mma_f16_ss(tmem + TM_Y + 64, dMb + ko, dXb + kk * 128, IDESC_Y, kk > 0);
+                }
+                tc::mma_commit(bar_y);
+            }
+            __syncwarp();
+            tc::named_sync(BAR_YSTAGED, kCompute + 32);
+            if (kStoreByTma && leader && c1 <= t1) {   // full chunk: both heads' y tiles by TMA
+                tc::tma_store_3d(&map_y, sbase + OFF_MB, 0, h0, (int)c0);
+                tc::tma_store_3d(&map_y, sbase + OFF_MB + HALF, 0, h0 + 1, (int)c0);
+                tc::bulk_commit();
+            }
+            __syncwarp();
         }
+        if (leader) tc::bulk_wait_all();
         __syncwarp();
+    } else {
+        // ================= compute warpgroups =================
+        const uint32_t tlane = (uint32_t)(wq * 32) << 16;
+        const size_t state_off = ((size_t)s * H + hh) * (size_t)(kP * kN) + (size_t)(32 * ch) * kN + i;
+        float Hs[32];
+#pragma unroll
+        for (int p = 0; p < 32; ++p)
+            Hs[p] = a.initial_state ? a.initial_state[state_off + (size_t)p * kN] : 0.f;
+        write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
 
-        // ---- decay mask M of this warpgroup's head (row i) ----
-        tc::mbar_wait_bounded(bar_sg, phase, ok);
-        tc::tc_fence_after();
-        {
-            const uint32_t mtile = sbase + (wg == 0 ? OFF_WM : OFF_MB);
+        const float Ah = a.A[hh];
+        const float Dh = a.D ? a.D[hh] : 0.f;
+        TOut *y = static_cast<TOut *>(a.y);
+        float *vd_tab = reinterpret_cast<float *>(smem + OFF_VD);   // [2 buffers][2 heads][128]
+        ChunkDecay cur{};
+        if (t1 > t0)
+            cur = chunk_decay(a, H, hh, Ah, t0, (int)min((long)kQ, t1 - t0), i, wq, lane, wg, ch,
+                              sPART, sCSB, vd_tab + hd * 128);
+        tc::named_sync(BAR_COMPUTE, kCompute);
+        uint32_t phase = 0, vb = 0;
+        for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u, vb ^= 1u) {
+            const int Lc = (int)min((long)kQ, t1 - c0);
+            const long c1 = c0 + kQ;
+            const bool has_next = c1 < t1;
+            const bool live = i < Lc;
+
+            // ---- operands to fp16 (rows past the chunk end zeroed) ----
+            tc::mbar_wait_bounded(bar_x, phase, ok);
+            tc::mbar_wait_bounded(bar_cb, phase, ok);
+            {
+                const uint32_t tile = sbase + (hd == 0 ? OFF_C : OFF_B) + ch * HALF;
 #pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
-                const uint32_t mrow = mtile + (jc >> 1) * HALF;
-                if (jc <= wq) {
-                    uint32_t r[32];
-                    tc::tmem_ld32(tmem + tlane + TM_G + jc * 32, r);
-                    tc::tmem_ld_wait();
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t addr = tile + sw128(i, k);
+                    sts128(addr, live ? cvt_chunk(lds128(addr)) : make_uint4(0, 0, 0, 0));
+                }
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float4 vd0 = lds128f(smem_offset_f(sbase, OFF_VD, wg, jc * 32 + q * 8));
-                        const float4 vd1 = lds128f(smem_offset_f(sbase, OFF_VD, wg, jc * 32 + q * 8 + 4));
-                        const float vd[8] = {vd0.x, vd0.y, vd0.z, vd0.w, vd1.x, vd1.y, vd1.z, vd1.w};
-                        float m[8];
-                        if (jc < wq) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                m[e] = __uint_as_float(r[q * 8 + e]) * ua[jc] * vd[e];
-                        } else if (block_safe) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int jl = q * 8 + e;   // column within the diagonal block
-                                float mv = (jl <= lane) ? __uint_as_float(r[jl]) * ua[jc] * vd[e] : 0.f;
-                                m[e] = (jl == lane) ? mv + Dh : mv;
-                            }
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int jl = q * 8 + e;
-                                const float csj = __shfl_sync(0xffffffffu, cs, jl);
-                                const float dtj = __shfl_sync(0xffffffffu, dtv, jl);
-                                float mv = (jl <= lane) ? __uint_as_float(r[jl]) * expf(cs - csj) * dtj : 0.f;
-                                m[e] = (jl == lane) ? mv + Dh : mv;
-                            }
-                        }
-                        sts128(mrow + sw128(i, (jc & 1) * 4 + q),
-                               make_uint4(f2_to_h2(m[0], m[1]), f2_to_h2(m[2], m[3]),
-                                          f2_to_h2(m[4], m[5]), f2_to_h2(m[6], m[7])));
+                for (int k = 4 * ch; k < 4 * ch + 4; ++k) {
+                    const uint32_t off = hd * HALF + sw128(i, k);
+                    if (live) {
+                        const uint4 r = lds128(sbase + OFF_XR + off);
+                        sts128(sbase + OFF_XH + off, cvt_chunk(r));
+                        sts128(sbase + OFF_WM + off, cvt_chunk_scaled(r, cur.w));
+                    } else {
+                        sts128(sbase + OFF_XH + off, make_uint4(0, 0, 0, 0));
+                        sts128(sbase + OFF_WM + off, make_uint4(0, 0, 0, 0));
                     }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        sts128(mrow + sw128(i, (jc & 1) * 4 + q), make_uint4(0, 0, 0, 0));
                 }
             }
-        }
-        tc::fence_proxy_async_smem();
-        tc::mbar_wait_bounded(bar_yo, phase, ok);   // Yoff done: C, B and H^T tiles are free
-        tc::tc_fence_before();
-        __syncthreads();
+            tc::fence_proxy_async_smem();
+            tc::named_arrive(BAR_OPERANDS, kCompute + 32);
 
-        if (tid == 0) {
-            if (has_next) {
-                tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
-                tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)c1);
-                tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, g, (int)c1);
-                tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)c1);
-                tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)c1);
+            // ---- next chunk's decay while the MMAs run ----
+            ChunkDecay nxt{};
+            if (has_next)
+                nxt = chunk_decay(a, H, hh, Ah, c1, (int)min((long)kQ, t1 - c1), i, wq, lane, wg, ch,
+                                  sPART, sCSB, vd_tab + (vb ^ 1u) * 256 + hd * 128);
+            tc::named_sync(BAR_COMPUTE, kCompute);
+
+            // ---- decay mask M of head hd: row i, column blocks kA and kB ----
+            tc::mbar_wait_bounded(bar_sg, phase, ok);
+            tc::tc_fence_after();
+            {
+                const uint32_t mtile = sbase + (hd == 0 ? OFF_WM : OFF_MB);
+                const float *vd = vd_tab + vb * 256 + hd * 128;
+                const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
+                mask_block(tmem + tlane + TM_G, mtile, vd, kA, wq, i, lane, cur.uaA, cur.safe, cur.cs, cur.dtv, Dh);
+                mask_block(tmem + tlane + TM_G, mtile, vd, kB, wq, i, lane, cur.uaB, cur.safe, cur.cs, cur.dtv, Dh);
             }
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            tc::named_arrive(BAR_MASK, kCompute + 32);
+
+            // ---- carried state: H <- exp(cs_L) H + S (d_state row i, p half ch) ----
+            tc::mbar_wait_bounded(bar_yo, phase, ok);   // Yoff read the old H^T
             tc::tc_fence_after();
 #pragma unroll
-            for (int hd = 0; hd < 2; ++hd) {
-                const uint32_t mt = sbase + (hd == 0 ? OFF_WM : OFF_MB);
+            for (int q = 0; q < 2; ++q) {
+                uint32_t r[16];
+                tc::tmem_ld16(tmem + tlane + TM_S + hd * 64 + ch * 32 + q * 16, r);
+                tc::tmem_ld_wait();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t koff = (kk >> 2) * HALF + (kk & 3) * 32;
-                    tc::mma_f16_ss(tmem + TM_Y + hd * 64, tc::sdesc_sw128(mt + koff, 16, 1024),
-                                   tc::sdesc_sw128(sbase + OFF_XH + hd * HALF + kk * 2048, HALF, 1024),
-                                   IDESC_Y, kk > 0);
+                for (int e = 0; e < 16; ++e)
+                    Hs[q * 16 + e] = fmaf(cur.a_last, Hs[q * 16 + e], __uint_as_float(r[e]));
+            }
+            write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+
+            // ---- y = Y + exp(cs_i) Yoff (row i, p half ch; D x is inside Y) ----
+            tc::mbar_wait_bounded(bar_y, phase, ok);
+            tc::tc_fence_after();
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {   // 16 columns at a time
+                uint32_t ry[16], ro[16];
+                tc::tmem_ld16(tmem + tlane + TM_Y + hd * 64 + ch * 32 + q * 16, ry);
+                tc::tmem_ld16(tmem + tlane + TM_YO + hd * 64 + ch * 32 + q * 16, ro);
+                tc::tmem_ld_wait();
+                float out[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) out[c] = fmaf(cur.e, __uint_as_float(ro[c]), __uint_as_float(ry[c]));
+                if (kStoreByTma && Lc == kQ) {
+                    stage16_bf16(sbase + OFF_MB + hd * HALF, i, 4 * ch + 2 * q, out);
+                } else if (live) {
+                    store16(y + ((size_t)(c0 + i) * H + hh) * kP + 32 * ch + 16 * q, out);
                 }
             }
-            tc::mma_commit(bar_y);
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            tc::named_arrive(BAR_YSTAGED, kCompute + 32);
+            cur = nxt;
         }
-        __syncwarp();
-
-        // ---- carried state: H <- exp(cs_L) H + S (d_state row i) ----
+        if (a.final_state) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            uint32_t r[32];
-            tc::tmem_ld32(tmem + tlane + TM_S + wg * 64 + half * 32, r);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-                Hs[half * 32 + e] = fmaf(a_last, Hs[half * 32 + e], __uint_as_float(r[e]));
+            for (int p = 0; p < 32; ++p) a.final_state[state_off + (size_t)p * kN] = Hs[p];
         }
-        write_state_tile(sbase + OFF_H + wg * HALF, i, Hs);
-
-        // ---- y = Y + exp(cs_i) Yoff (row i; D x is inside Y) ----
-        tc::mbar_wait_bounded(bar_y, phase, ok);
-        tc::tc_fence_after();
-        {
-            TOut *yrow = y + ((size_t)(c0 + i) * H + hh) * kP;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t ry[32], ro[32];
-                tc::tmem_ld32(tmem + tlane + TM_Y + wg * 64 + half * 32, ry);
-                tc::tmem_ld32(tmem + tlane + TM_YO + wg * 64 + half * 32, ro);
-                tc::tmem_ld_wait();
-                float out[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    out[c] = fmaf(e_i, __uint_as_float(ro[c]), __uint_as_float(ry[c]));
-                if (live) store_row(yrow + half * 32, out);
-            }
-        }
-        tc::tc_fence_before();
-        tc::fence_proxy_async_smem();
-        __syncthreads();
-    }
-
-    if (a.final_state) {
-#pragma unroll
-        for (int p = 0; p < kP; ++p)
-            a.final_state[state_off + (size_t)p * kN + i] = Hs[p];
     }
     tc::tc_fence_before();
     __syncthreads();
@@ -492,7 +570,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, TM_COLS);
     }
-    if (!ok && i == 0) report_status(a.status_dev, 5);
+    if (!ok) report_status(a.status_dev, 5);
 }
 
 // ------------------------------------------------------------------ host side
@@ -514,8 +592,9 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// 3-D bf16 map over [d2][d1][d0] (d0 contiguous) with a {64, 1, 128} box and
-// 128-byte swizzle.
+// 3-D map over [d2][d1][d0] (d0 contiguous) of 16-bit elements with a
+// {64, 1, 128} box (one 128-token tile of one head or group, 64 elements
+// wide) and 128-byte swizzle.
 bool make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2)
 {
     EncodeTiledFn fn = encode_fn();
@@ -533,15 +612,20 @@ template <typename TOut>
 cudaError_t launch_tc_t(const ScanArgs &a, cudaStream_t stream)
 {
     const uint64_t T = a.cu_seqlens ? (uint64_t)a.seqlen : (uint64_t)a.nseq * a.seqlen;
-    CUtensorMap mx, mb, mc;
+    CUtensorMap mx, mb, mc, my;
     if (!make_map(&mx, a.x, kP, a.nheads, T) || !make_map(&mb, a.B, kN, a.ngroups, T) ||
         !make_map(&mc, a.C, kN, a.ngroups, T))
         return cudaErrorInvalidValue;
+    if (sizeof(TOut) == 2) {
+        if (!make_map(&my, a.y, kP, a.nheads, T)) return cudaErrorInvalidValue;
+    } else {
+        my = mx;   // unused: fp32 y is stored row by row
+    }
     cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<TOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((size_t)a.nseq * (a.nheads / 2)));
-    scan_tc_kernel<TOut><<<grid, kThreads, SMEM_BYTES, stream>>>(mx, mb, mc, a);
+    scan_tc_kernel<TOut><<<grid, kThreads, SMEM_BYTES, stream>>>(mx, mb, mc, my, a);
     return cudaGetLastError();
 }
 
