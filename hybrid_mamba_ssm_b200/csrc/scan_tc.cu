@@ -70,8 +70,8 @@ constexpr uint32_t OFF_C = 0;            // C [128 i][128 n]  (bf16 -> fp16 in p
 constexpr uint32_t OFF_B = 32768;        // B [128 j][128 n]  (bf16 -> fp16 in place)
 constexpr uint32_t OFF_XR = 65536;       // raw x, 2 heads x [128 j][64 p] bf16 (TMA target)
 constexpr uint32_t OFF_XH = 98304;       // x as fp16, 2 heads
-constexpr uint32_t OFF_WM = 131072;      // w o x (2 heads), later M of head 0 [128][128]
-constexpr uint32_t OFF_MB = 163840;      // M of head 1
+constexpr uint32_t OFF_WM = 131072;      // w o x, 2 heads x [128 j][64 p]
+constexpr uint32_t OFF_MB = 163840;      // y staging, 2 heads x [128 t][64 p] bf16
 constexpr uint32_t OFF_H = 196608;       // H^T fp16, 2 heads x [128 n][64 p]
 constexpr uint32_t OFF_MISC = 229376;
 constexpr uint32_t OFF_VD = OFF_MISC;              // float[2 buffers][2 heads][128]
@@ -88,7 +88,7 @@ constexpr uint32_t TM_COLS = 512;
 constexpr uint32_t IDESC_G = tc::idesc_f16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
 constexpr uint32_t IDESC_S2 = tc::idesc_f16_f32(128, 128, 1, 1);  // B^T (MN-major) x [wX_a|wX_b] (MN-major)
 constexpr uint32_t IDESC_YO2 = tc::idesc_f16_f32(128, 128, 0, 1); // C (K-major) x [H_a^T|H_b^T] (MN-major)
-constexpr uint32_t IDESC_Y = tc::idesc_f16_f32(128, 64, 0, 1);    // M (K-major) x X (MN-major)
+constexpr uint32_t IDESC_Y = tc::idesc_f16_f32(128, 64, 0, 1);    // M (TMEM) x X (MN-major)
 
 constexpr float kSafeBlockDecay = 80.f;   // max exp argument taken by the factorised path
 
@@ -170,19 +170,21 @@ __device__ __forceinline__ void write_state_half(uint32_t sH, uint32_t n, int ch
     }
 }
 
-// One 32-column block jc of row i of the decay mask M (fp16, K-major tile):
+// One 32-column block jc of row i of the decay mask M, as fp16 pairs into
+// TMEM (lane i, columns m_taddr + 16 jc ..  + 16: the A operand of the y MMA):
 //   off-diagonal (jc < wq):  G[i][j] * exp(cs_i - cs_{r_jc}) * vd[j]
 //   diagonal (jc == wq):     j <= i only, plus D on j == i
 //   above (jc > wq):         zeros
 // with vd[j] = exp(cs_{r_J} - cs_j) dt_j (J = j's block) from shared memory.
-__device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t mtile, const float *sVD,
-                                           int jc, int wq, int i, int lane, float ua,
+__device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, const float *sVD,
+                                           int jc, int wq, int lane, float ua,
                                            bool block_safe, float cs, float dtv, float Dh)
 {
-    const uint32_t mrow = mtile + (jc >> 1) * HALF;
+    uint32_t pk[16];
     if (jc > wq) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) sts128(mrow + sw128(i, (jc & 1) * 4 + q), make_uint4(0, 0, 0, 0));
+        for (int q = 0; q < 16; ++q) pk[q] = 0u;
+        tc::tmem_st16(m_taddr + jc * 16, pk);
         return;
     }
     const float4 *vd4 = reinterpret_cast<const float4 *>(sVD + jc * 32);
@@ -217,11 +219,11 @@ __device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t mtile, con
                     m[e] = (jl == lane) ? mv + Dh : mv;
                 }
             }
-            sts128(mrow + sw128(i, (jc & 1) * 4 + q),
-                   make_uint4(f2_to_h2(m[0], m[1]), f2_to_h2(m[2], m[3]),
-                              f2_to_h2(m[4], m[5]), f2_to_h2(m[6], m[7])));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pk[q * 4 + e] = f2_to_h2(m[2 * e], m[2 * e + 1]);
         }
     }
+    tc::tmem_st16(m_taddr + jc * 16, pk);
 }
 
 // 16 bf16 outputs of row i (two 16-byte chunks starting at chunk c) into the
@@ -371,8 +373,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         const uint64_t dCk = tc::sdesc_sw128(sbase + OFF_C, 16, 1024);      // C, K-major
         const uint64_t dBk = tc::sdesc_sw128(sbase + OFF_B, 16, 1024);      // B, K-major
         const uint64_t dH = tc::sdesc_sw128(sbase + OFF_H, HALF, 1024);     // [H_a^T | H_b^T]
-        const uint64_t dMa = tc::sdesc_sw128(sbase + OFF_WM, 16, 1024);
-        const uint64_t dMb = tc::sdesc_sw128(sbase + OFF_MB, 16, 1024);
         const uint64_t dXa = tc::sdesc_sw128(sbase + OFF_XH, HALF, 1024);
         const uint64_t dXb = dXa + (HALF >> 4);
         if (leader && t1 > t0) {
@@ -427,15 +427,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 }
                 tc::tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
-                    tc::mma_f16_ss(tmem + TM_Y, dMa + ko, dXa + kk * 128, IDESC_Y, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ts(tmem + TM_Y, tmem + TM_S + kk * 8, dXa + kk * 128, IDESC_Y, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
-                    tc::mma_f16_ss(tmem + TM_Y + 64, dMb + ko, dXb + kk * 128, IDESC_Y, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ts(tmem + TM_Y + 64, tmem + TM_S + 64 + kk * 8, dXb + kk * 128, IDESC_Y, kk > 0);
                 tc::mma_commit(bar_y);
             }
             __syncwarp();
@@ -508,22 +504,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                                   sPART, sCSB, vd_tab + (vb ^ 1u) * 256 + hd * 128);
             tc::named_sync(BAR_COMPUTE, kCompute);
 
-            // ---- decay mask M of head hd: row i, column blocks kA and kB ----
-            tc::mbar_wait_bounded(bar_sg, phase, ok);
-            tc::tc_fence_after();
-            {
-                const uint32_t mtile = sbase + (hd == 0 ? OFF_WM : OFF_MB);
-                const float *vd = vd_tab + vb * 256 + hd * 128;
-                const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
-                mask_block(tmem + tlane + TM_G, mtile, vd, kA, wq, i, lane, cur.uaA, cur.safe, cur.cs, cur.dtv, Dh);
-                mask_block(tmem + tlane + TM_G, mtile, vd, kB, wq, i, lane, cur.uaB, cur.safe, cur.cs, cur.dtv, Dh);
-            }
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
-            tc::named_arrive(BAR_MASK, kCompute + 32);
-
             // ---- carried state: H <- exp(cs_L) H + S (d_state row i, p half ch) ----
-            tc::mbar_wait_bounded(bar_yo, phase, ok);   // Yoff read the old H^T
+            tc::mbar_wait_bounded(bar_sg, phase, ok);
             tc::tc_fence_after();
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
@@ -534,6 +516,24 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 for (int e = 0; e < 16; ++e)
                     Hs[q * 16 + e] = fmaf(cur.a_last, Hs[q * 16 + e], __uint_as_float(r[e]));
             }
+            tc::tc_fence_before();
+            tc::named_sync(BAR_COMPUTE, kCompute);   // every S column read: M may overwrite them
+            tc::tc_fence_after();
+
+            // ---- decay mask M of head hd into TMEM (over S of this head) ----
+            {
+                const float *vd = vd_tab + vb * 256 + hd * 128;
+                const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
+                const uint32_t m_taddr = tmem + tlane + TM_S + hd * 64;
+                mask_block(tmem + tlane + TM_G, m_taddr, vd, kA, wq, lane, cur.uaA, cur.safe, cur.cs, cur.dtv, Dh);
+                mask_block(tmem + tlane + TM_G, m_taddr, vd, kB, wq, lane, cur.uaB, cur.safe, cur.cs, cur.dtv, Dh);
+                tc::tmem_st_wait();
+            }
+            tc::tc_fence_before();
+            tc::named_arrive(BAR_MASK, kCompute + 32);
+
+            // ---- new H^T tile for the next chunk (Yoff of this chunk read the old one) ----
+            tc::mbar_wait_bounded(bar_yo, phase, ok);
             write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
 
             // ---- y = Y + exp(cs_i) Yoff (row i, p half ch; D x is inside Y) ----
