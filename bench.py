@@ -85,8 +85,9 @@ def kernel_source_hash(fname):
 
 
 def measured_traffic(kernel, source_file):
-    """DRAM bytes per launch from a committed ncu summary, or None if the
-    kernel's source changed since the counters were taken."""
+    """DRAM bytes (read + write) per launch of the benchmark's own launch, from
+    the committed ncu summary, or None if the kernel's source changed since the
+    counters were taken."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -444,7 +445,7 @@ def run_ours(args, world, rank, local, pg):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
