@@ -103,6 +103,16 @@ __device__ __forceinline__ uint32_t bf2_to_h2(uint32_t v, float scale) {
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// exp(v) as 2^(v log2 e) with the hardware base-2 exponential (ex2.approx,
+// relative error ~2^-22).  The decay arguments here are cumulative sums of
+// dt A differences (|v| up to a few hundred), so the rounding of v log2 e
+// adds a relative error of about |v| 2^-24, far below the fp16 operands'.
+__device__ __forceinline__ float exp_dec(float v) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v * 1.4426950408889634f));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
@@ -279,12 +289,12 @@ __device__ __forceinline__ ChunkDecay chunk_decay(const ScanArgs &a, int H, int 
     const float cs_own_end = sCSB[wq];
     d.safe = (__shfl_sync(0xffffffffu, d.cs, 0) - cs_own_end) <= kSafeBlockDecay;
     const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
-    d.uaA = (kA <= wq) ? expf(d.cs - sCSB[kA]) : 0.f;
-    d.uaB = (kB <= wq) ? expf(d.cs - sCSB[kB]) : 0.f;
-    if (ch == 0) vd_out[i] = expf(cs_own_end - d.cs) * d.dtv;   // <= dt
-    d.w = (i < Lc) ? expf(cs_last - d.cs) * d.dtv : 0.f;
-    d.e = expf(d.cs);
-    d.a_last = expf(cs_last);
+    d.uaA = (kA <= wq) ? exp_dec(d.cs - sCSB[kA]) : 0.f;
+    d.uaB = (kB <= wq) ? exp_dec(d.cs - sCSB[kB]) : 0.f;
+    if (ch == 0) vd_out[i] = exp_dec(cs_own_end - d.cs) * d.dtv;   // <= dt
+    d.w = (i < Lc) ? exp_dec(cs_last - d.cs) * d.dtv : 0.f;
+    d.e = exp_dec(d.cs);
+    d.a_last = exp_dec(cs_last);
     return d;
 }
 
