@@ -15,7 +15,7 @@ nor the library.
 """
 
 __all__ = ["ssd_chunk_scan", "ssm_state_update", "ssd_chunk_scan_workspace_size",
-           "SSMError"]
+           "ssd_chunk_scan_slots", "ssm_state_update_slots", "SSMError"]
 
 
 def __getattr__(name):

@@ -49,12 +49,12 @@ const char *ssm_status_string(int status)
     case SSM_ERR_MISALIGNED: return "SSM_ERR_MISALIGNED: pointer not 16-byte aligned";
     case SSM_ERR_CUDA: return "SSM_ERR_CUDA: CUDA launch error";
     case SSM_ERR_TIMEOUT: return "SSM_ERR_TIMEOUT: bounded device wait expired";
-    case SSM_ERR_DEVICE_INPUT: return "SSM_ERR_DEVICE_INPUT: inconsistent cu_seqlens";
+    case SSM_ERR_DEVICE_INPUT: return "SSM_ERR_DEVICE_INPUT: inconsistent cu_seqlens or slot index";
     default: return "unknown ssm status";
     }
 }
 
-int ssm_version(void) { return 100; }
+int ssm_version(void) { return 200; }
 
 size_t ssd_chunk_scan_workspace_size(int, int, int, int, int, int, int) { return 0; }
 
@@ -123,6 +123,61 @@ int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
     a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
     a.initial_state = initial_state; a.y = y; a.final_state = final_state;
     a.status_dev = status_dev;
+    a.slot_idx = nullptr; a.has_initial = nullptr; a.max_slots = 0;
+    const cudaError_t e = ssm::scan_tc_supports(a) ? ssm::launch_scan_tc(a, stream)
+                                                   : ssm::launch_scan_simt(a, stream);
+    return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
+                         int nheads, int head_dim, int d_state, int ngroups,
+                         int chunk_size, int in_dtype,
+                         const void *x, const float *dt, const float *A,
+                         const void *B, const void *C, const float *D,
+                         float *state_pool, int max_slots, const int32_t *slot_idx,
+                         const int32_t *has_initial_state,
+                         int y_dtype, void *y, int *status_dev, cudaStream_t stream)
+{
+    if (nseq < 0 || seqlen < 0 || nheads <= 0 || ngroups <= 0 || nheads % ngroups)
+        return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
+    if (!pow2_in(head_dim, 16, 128) || !pow2_in(d_state, 16, 128)) return SSM_ERR_UNSUPPORTED;
+    if (chunk_size != 64 && chunk_size != 128) return SSM_ERR_UNSUPPORTED;
+    if (nseq == 0) return SSM_OK;
+    if (max_slots <= 0 || !state_pool || !slot_idx || !A) return SSM_ERR_INVALID_ARG;
+    const long long T = cu_seqlens ? (long long)seqlen : (long long)nseq * seqlen;
+    if (T > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    if (T > 0 && (!x || !dt || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {cu_seqlens, x, dt, A, B, C, D, state_pool, slot_idx, has_initial_state,
+                          y, status_dev};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+    const size_t es = dtype_size(in_dtype);
+    const Range rpool = range_of(state_pool, (size_t)max_slots * nheads * head_dim * d_state * sizeof(float));
+    const Range ry = range_of(y, (size_t)T * nheads * head_dim * dtype_size(y_dtype));
+    const Range ins[] = {range_of(x, (size_t)T * nheads * head_dim * es),
+                         range_of(dt, (size_t)T * nheads * sizeof(float)),
+                         range_of(A, (size_t)nheads * sizeof(float)),
+                         range_of(B, (size_t)T * ngroups * d_state * es),
+                         range_of(C, (size_t)T * ngroups * d_state * es),
+                         range_of(D, D ? (size_t)nheads * sizeof(float) : 0),
+                         range_of(slot_idx, (size_t)nseq * sizeof(int32_t)),
+                         range_of(has_initial_state, has_initial_state ? (size_t)nseq * sizeof(int32_t) : 0),
+                         range_of(cu_seqlens, cu_seqlens ? (size_t)(nseq + 1) * sizeof(int32_t) : 0)};
+    for (const Range &r : ins)
+        if (overlap(ry, r) || overlap(rpool, r)) return SSM_ERR_INVALID_ARG;
+    if (overlap(ry, rpool)) return SSM_ERR_INVALID_ARG;
+
+    ssm::ScanArgs a;
+    a.nseq = nseq; a.seqlen = seqlen; a.cu_seqlens = cu_seqlens;
+    a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
+    a.ngroups = ngroups; a.chunk_size = chunk_size;
+    a.in_dtype = in_dtype; a.y_dtype = y_dtype;
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.initial_state = state_pool; a.y = y; a.final_state = state_pool;
+    a.status_dev = status_dev;
+    a.slot_idx = slot_idx; a.has_initial = has_initial_state; a.max_slots = max_slots;
+    // empty sequences still run: a slot without an initial state is reset to zero
     const cudaError_t e = ssm::scan_tc_supports(a) ? ssm::launch_scan_tc(a, stream)
                                                    : ssm::launch_scan_simt(a, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
@@ -163,6 +218,47 @@ int ssm_state_update(int batch, int nheads, int head_dim, int d_state,
     a.batch = batch; a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
     a.ngroups = ngroups; a.in_dtype = in_dtype; a.y_dtype = y_dtype;
     a.state = state; a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.y = y;
+    a.slot_idx = nullptr; a.max_slots = 0; a.status_dev = nullptr;
+    return ssm::launch_state_update(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
+                           int ngroups, int in_dtype, float *state_pool, int max_slots,
+                           const int32_t *slot_idx,
+                           const void *x, const float *dt, const float *A,
+                           const void *B, const void *C, const float *D,
+                           int y_dtype, void *y, int *status_dev, cudaStream_t stream)
+{
+    if (batch < 0 || nheads <= 0 || ngroups <= 0 || nheads % ngroups || head_dim <= 0)
+        return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
+    if (head_dim > 256 || !pow2_in(d_state, 16, 256)) return SSM_ERR_UNSUPPORTED;
+    if ((long long)batch * nheads > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    if (batch == 0) return SSM_OK;
+    if (max_slots <= 0 || !state_pool || !slot_idx || !x || !dt || !A || !B || !C || !y)
+        return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {state_pool, slot_idx, x, dt, A, B, C, D, y, status_dev};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+    const size_t es = dtype_size(in_dtype);
+    const Range rs = range_of(state_pool, (size_t)max_slots * nheads * head_dim * d_state * sizeof(float));
+    const Range ry = range_of(y, (size_t)batch * nheads * head_dim * dtype_size(y_dtype));
+    const Range ins[] = {range_of(x, (size_t)batch * nheads * head_dim * es),
+                         range_of(dt, (size_t)batch * nheads * sizeof(float)),
+                         range_of(A, (size_t)nheads * sizeof(float)),
+                         range_of(B, (size_t)batch * ngroups * d_state * es),
+                         range_of(C, (size_t)batch * ngroups * d_state * es),
+                         range_of(D, D ? (size_t)nheads * sizeof(float) : 0),
+                         range_of(slot_idx, (size_t)batch * sizeof(int32_t))};
+    for (const Range &r : ins)
+        if (overlap(ry, r) || overlap(rs, r)) return SSM_ERR_INVALID_ARG;
+    if (overlap(ry, rs)) return SSM_ERR_INVALID_ARG;
+
+    ssm::StateUpdateArgs a;
+    a.batch = batch; a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
+    a.ngroups = ngroups; a.in_dtype = in_dtype; a.y_dtype = y_dtype;
+    a.state = state_pool; a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.y = y;
+    a.slot_idx = slot_idx; a.max_slots = max_slots; a.status_dev = status_dev;
     return ssm::launch_state_update(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

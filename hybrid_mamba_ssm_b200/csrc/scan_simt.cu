@@ -86,11 +86,22 @@ scan_simt_kernel(ScanArgs a)
     TOut *y = static_cast<TOut *>(a.y);
     const float Ah = a.A[h];
     const float Dh = a.D ? a.D[h] : 0.f;
-    const size_t state_off = ((size_t)s * H + h) * (size_t)P * N;
+    size_t srow = (size_t)s;   // state row of this sequence
+    bool load_init = a.initial_state != nullptr;
+    if (a.slot_idx) {
+        const int slot = a.slot_idx[s];
+        if (slot < 0 || slot >= a.max_slots) {
+            if (tid == 0) report_status(a.status_dev, 6);
+            return;
+        }
+        srow = (size_t)slot;
+        if (a.has_initial && a.has_initial[s] == 0) load_init = false;
+    }
+    const size_t state_off = (srow * H + h) * (size_t)P * N;
 
     for (int i = tid; i < P * N; i += kSimtThreads) {
         const int p = i / N, n = i - p * N;
-        Hs[p * N1 + n] = a.initial_state ? a.initial_state[state_off + i] : 0.f;
+        Hs[p * N1 + n] = load_init ? a.initial_state[state_off + i] : 0.f;
     }
 
     for (long c0 = t0; c0 < t1; c0 += Q) {

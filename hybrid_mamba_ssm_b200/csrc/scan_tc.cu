@@ -351,6 +351,18 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         t0 = (long)s * a.seqlen; t1 = t0 + a.seqlen;
     }
 
+    size_t srow = (size_t)s;   // state row of this sequence
+    bool load_init = a.initial_state != nullptr;
+    if (a.slot_idx) {
+        const int slot = a.slot_idx[s];
+        if (slot < 0 || slot >= a.max_slots) {
+            if (tid == 0) report_status(a.status_dev, 6);
+            return;
+        }
+        srow = (size_t)slot;
+        if (a.has_initial && a.has_initial[s] == 0) load_init = false;
+    }
+
     float *sCSB = reinterpret_cast<float *>(smem + OFF_CSB) + wg * 8;
     float *sPART = reinterpret_cast<float *>(smem + OFF_PART) + wg * 4;
     const uint32_t bar_x = sbase + OFF_BAR, bar_cb = bar_x + 8, bar_sg = bar_x + 16;
@@ -458,11 +470,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     } else {
         // ================= compute warpgroups =================
         const uint32_t tlane = (uint32_t)(wq * 32) << 16;
-        const size_t state_off = ((size_t)s * H + hh) * (size_t)(kP * kN) + (size_t)(32 * ch) * kN + i;
+        const size_t state_off = (srow * H + hh) * (size_t)(kP * kN) + (size_t)(32 * ch) * kN + i;
         float Hs[32];
 #pragma unroll
         for (int p = 0; p < 32; ++p)
-            Hs[p] = a.initial_state ? a.initial_state[state_off + (size_t)p * kN] : 0.f;
+            Hs[p] = load_init ? a.initial_state[state_off + (size_t)p * kN] : 0.f;
         write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
 
         const float Ah = a.A[hh];

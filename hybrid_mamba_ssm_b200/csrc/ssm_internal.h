@@ -17,6 +17,10 @@ struct StateUpdateArgs {
     const void *B, *C;
     const float *D;
     void *y;
+    // slot-indexed state pool (nullptr: row b of the state is batch row b)
+    const int32_t *slot_idx;      // device [batch]; < 0 skips the row
+    int max_slots;
+    int *status_dev;
 };
 
 struct ScanArgs {
@@ -32,6 +36,12 @@ struct ScanArgs {
     void *y;
     float *final_state;           // nullptr = not written
     int *status_dev;              // nullptr = not reported
+    // slot-indexed state pool: sequence s reads and writes state row
+    // slot_idx[s] of initial_state / final_state (the same pool); nullptr
+    // means row s.  has_initial[s] == 0 starts sequence s from zero.
+    const int32_t *slot_idx;
+    const int32_t *has_initial;
+    int max_slots;
 };
 
 cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);

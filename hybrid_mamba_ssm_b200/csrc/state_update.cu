@@ -29,7 +29,8 @@ state_update_kernel(int nheads, int head_dim, int heads_per_group, int ngroups,
                     float *__restrict__ state, const TIn *__restrict__ x,
                     const float *__restrict__ dt, const float *__restrict__ A,
                     const TIn *__restrict__ B, const TIn *__restrict__ C,
-                    const float *__restrict__ D, TOut *__restrict__ y)
+                    const float *__restrict__ D, TOut *__restrict__ y,
+                    const int32_t *__restrict__ slot_idx, int max_slots, int *status)
 {
     constexpr int LPR = (N / 4 < 32) ? N / 4 : 32;   // lanes per state row
     constexpr int VEC = N / (4 * LPR);               // float4s per lane
@@ -40,6 +41,16 @@ state_update_kernel(int nheads, int head_dim, int heads_per_group, int ngroups,
     const int b = bh / nheads;
     const int h = bh - b * nheads;
     const int g = h / heads_per_group;
+    size_t srow = (size_t)b;   // state row of this batch row
+    if (slot_idx) {
+        const int slot = __ldg(slot_idx + b);
+        if (slot < 0) return;                        // padding row: nothing to do
+        if (slot >= max_slots) {
+            if (threadIdx.x == 0) report_status(status, 6);
+            return;
+        }
+        srow = (size_t)slot;
+    }
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int li = lane % LPR;
@@ -59,7 +70,7 @@ state_update_kernel(int nheads, int head_dim, int heads_per_group, int ngroups,
         cv[v] = load4(Cp + n0);
     }
 
-    float *st = state + (size_t)bh * head_dim * N;
+    float *st = state + (srow * nheads + h) * (size_t)head_dim * N;
     const TIn *xp = x + (size_t)bh * head_dim;
     TOut *yp = y + (size_t)bh * head_dim;
 
@@ -113,7 +124,8 @@ static cudaError_t launch_state_update_t(const StateUpdateArgs &a, cudaStream_t 
     state_update_kernel<N, TIn, TOut><<<grid, kDecodeWarps * 32, 0, stream>>>(
         a.nheads, a.head_dim, a.nheads / a.ngroups, a.ngroups, a.state,
         static_cast<const TIn *>(a.x), a.dt, a.A, static_cast<const TIn *>(a.B),
-        static_cast<const TIn *>(a.C), a.D, static_cast<TOut *>(a.y));
+        static_cast<const TIn *>(a.C), a.D, static_cast<TOut *>(a.y), a.slot_idx, a.max_slots,
+        a.status_dev);
     return cudaGetLastError();
 }
 

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED",
                 3: "SSM_ERR_MISALIGNED", 4: "SSM_ERR_CUDA", 5: "SSM_ERR_TIMEOUT",
                 6: "SSM_ERR_DEVICE_INPUT"}
 EXPORTS = ("ssd_chunk_scan", "ssd_chunk_scan_workspace_size", "ssm_state_update",
-           "ssm_status_string", "ssm_version")
+           "ssd_chunk_scan_slots", "ssm_state_update_slots", "ssm_status_string", "ssm_version")
 
 
 def _load():
@@ -37,6 +37,12 @@ def _load():
     lib.ssm_state_update.restype = i
     lib.ssm_state_update.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, i,
                                      vp, vp]
+    lib.ssd_chunk_scan_slots.restype = i
+    lib.ssd_chunk_scan_slots.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp,
+                                         vp, i, vp, vp, i, vp, vp, vp]
+    lib.ssm_state_update_slots.restype = i
+    lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp, vp,
+                                           i, vp, vp, vp]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_status_string.argtypes = [i]
     lib.ssm_version.restype = i
@@ -168,4 +174,80 @@ def ssm_state_update(state, x, dt, A, B, C, D=None, y=None, y_dtype=None, stream
                               _ptr(A), _ptr(B), _ptr(C), _ptr(D), _dtype_code(y.dtype),
                               _ptr(y), _stream(stream))
     _check(st, "ssm_state_update")
+    return y
+
+
+def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_state=None,
+                         cu_seqlens=None, chunk_size: int = 128, y=None, y_dtype=None,
+                         status=None, stream=None):
+    """Chunked SSD prefill whose states live in a pool, updated in place.
+
+    state_pool : [max_slots, H, P, N] fp32; sequence s starts from
+        state_pool[slot_idx[s]] (or zero where has_initial_state[s] == 0) and
+        its final state is written back to the same row.
+    slot_idx, has_initial_state : int32 CUDA tensors [nseq].
+    Other arguments as for ssd_chunk_scan.  Returns y.
+    """
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens", torch.int32)
+        T, H, P = x.shape
+        nseq = cu_seqlens.shape[0] - 1
+        seqlen = T
+    else:
+        nseq, L, H, P = x.shape
+        seqlen = L
+    G, N = B.shape[-2], B.shape[-1]
+    _dev(dt, "dt", torch.float32)
+    _dev(A, "A", torch.float32)
+    _dev(B, "B", x.dtype)
+    _dev(C, "C", x.dtype)
+    _dev(D, "D", torch.float32)
+    _dev(state_pool, "state_pool", torch.float32)
+    _dev(slot_idx, "slot_idx", torch.int32)
+    _dev(has_initial_state, "has_initial_state", torch.int32)
+    _dev(status, "status", torch.int32)
+    if y_dtype is None:
+        y_dtype = x.dtype if y is None else y.dtype
+    if y is None:
+        y = torch.empty(x.shape, dtype=y_dtype, device=x.device)
+    _dev(y, "y", y_dtype)
+    st = lib.ssd_chunk_scan_slots(nseq, seqlen, _ptr(cu_seqlens), H, P, N, G, int(chunk_size),
+                                  in_code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                  _ptr(state_pool), state_pool.shape[0], _ptr(slot_idx),
+                                  _ptr(has_initial_state), _dtype_code(y.dtype), _ptr(y),
+                                  _ptr(status), _stream(stream))
+    _check(st, "ssd_chunk_scan_slots")
+    return y
+
+
+def ssm_state_update_slots(state_pool, slot_idx, x, dt, A, B, C, D=None, y=None, y_dtype=None,
+                           status=None, stream=None):
+    """One-token decode update of pool rows: batch row b updates
+    state_pool[slot_idx[b]] in place (slot_idx[b] < 0: padding row, skipped).
+    Returns y [batch, H, P] (padding rows left as they were)."""
+    _dev(state_pool, "state_pool", torch.float32)
+    _dev(slot_idx, "slot_idx", torch.int32)
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    batch, H, P = x.shape
+    N = state_pool.shape[-1]
+    G = B.shape[-2]
+    _dev(dt, "dt", torch.float32)
+    _dev(A, "A", torch.float32)
+    _dev(B, "B", x.dtype)
+    _dev(C, "C", x.dtype)
+    _dev(D, "D", torch.float32)
+    _dev(status, "status", torch.int32)
+    if y_dtype is None:
+        y_dtype = x.dtype if y is None else y.dtype
+    if y is None:
+        y = torch.zeros((batch, H, P), dtype=y_dtype, device=x.device)
+    _dev(y, "y", y_dtype)
+    st = lib.ssm_state_update_slots(batch, H, P, N, G, in_code, _ptr(state_pool),
+                                    state_pool.shape[0], _ptr(slot_idx), _ptr(x), _ptr(dt),
+                                    _ptr(A), _ptr(B), _ptr(C), _ptr(D), _dtype_code(y.dtype),
+                                    _ptr(y), _ptr(status), _stream(stream))
+    _check(st, "ssm_state_update_slots")
     return y

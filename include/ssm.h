@@ -59,7 +59,7 @@ typedef enum {
     SSM_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
     SSM_ERR_CUDA = 4,          /* the CUDA runtime reported a launch error */
     SSM_ERR_TIMEOUT = 5,       /* reserved: a bounded device wait expired */
-    SSM_ERR_DEVICE_INPUT = 6   /* written to status_dev: bad cu_seqlens */
+    SSM_ERR_DEVICE_INPUT = 6   /* written to status_dev: bad cu_seqlens or slot index */
 } ssm_status;
 
 typedef enum {
@@ -70,7 +70,7 @@ typedef enum {
 /* Human-readable name of a status code (static string, never NULL). */
 SSM_API const char *ssm_status_string(int status);
 
-/* Library version as major*10000 + minor*100 + patch. */
+/* Library version as major*10000 + minor*100 + patch (200 = 0.2.0). */
 SSM_API int ssm_version(void);
 
 /*
@@ -152,6 +152,57 @@ SSM_API int ssm_state_update(int batch, int nheads, int head_dim, int d_state,
                      const void *x, const float *dt, const float *A,
                      const void *B, const void *C, const float *D,
                      int y_dtype, void *y, cudaStream_t stream);
+
+/*
+ * Slot-indexed state pools.  A serving engine keeps every live request's
+ * recurrent state in one pool [max_slots][nheads][head_dim][d_state] (fp32)
+ * and hands each call the pool slot of each sequence or batch row, so that no
+ * gather/scatter of states around the call is needed: the kernels read and
+ * write the slots in place.  This is the slot_idx -> ssm_pool design of the
+ * MAX nemotron_h article, section 8 (state pools and request lifecycle), with
+ * its has_initial_state flag (section 5.5).
+ */
+
+/*
+ * ssd_chunk_scan_slots -- ssd_chunk_scan whose initial and final states are
+ * rows of a state pool.
+ *   state_pool         device fp32 [max_slots][nheads][head_dim][d_state], read
+ *                      and written in place (only the rows named in slot_idx)
+ *   max_slots          number of rows of the pool (> 0)
+ *   slot_idx           device int32 [nseq]: pool row of sequence s.  Rows must
+ *                      be distinct; an index outside [0, max_slots) skips that
+ *                      sequence (no output written) and sets
+ *                      SSM_ERR_DEVICE_INPUT in *status_dev.
+ *   has_initial_state  device int32 [nseq] or NULL (all true): 0 starts the
+ *                      sequence from a zero state (a freshly claimed slot)
+ *                      instead of the slot's contents.
+ * Every other argument is as for ssd_chunk_scan.  A zero-length sequence
+ * leaves its slot unchanged, or zeroes it when it has no initial state.  The
+ * pool must not overlap any input or y.
+ */
+SSM_API int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
+                                 int nheads, int head_dim, int d_state, int ngroups,
+                                 int chunk_size, int in_dtype,
+                                 const void *x, const float *dt, const float *A,
+                                 const void *B, const void *C, const float *D,
+                                 float *state_pool, int max_slots, const int32_t *slot_idx,
+                                 const int32_t *has_initial_state,
+                                 int y_dtype, void *y, int *status_dev, cudaStream_t stream);
+
+/*
+ * ssm_state_update_slots -- ssm_state_update on pool rows: batch row b updates
+ * state_pool[slot_idx[b]] in place.  A negative slot index marks a padding row
+ * (no state update, y not written); an index >= max_slots skips the row and
+ * sets SSM_ERR_DEVICE_INPUT in *status_dev (status_dev may be NULL).  Slot
+ * indices of non-padding rows must be distinct.  Other arguments as for
+ * ssm_state_update.
+ */
+SSM_API int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
+                                   int ngroups, int in_dtype, float *state_pool, int max_slots,
+                                   const int32_t *slot_idx,
+                                   const void *x, const float *dt, const float *A,
+                                   const void *B, const void *C, const float *D,
+                                   int y_dtype, void *y, int *status_dev, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -158,3 +158,43 @@ def state_update(state, x, dt, A, B, C, D=None):
     if rc != 0:
         raise ValueError(f"oracle_state_update rejected its arguments ({rc})")
     return y, st
+
+
+def scan_slots(pool, slot_idx, has_initial, x, dt, A, B, C, D=None, cu_seqlens=None):
+    """The scan over sequences whose states are rows of a pool (the slot_idx ->
+    ssm_pool design of the MAX nemotron_h article, section 8): sequence s
+    starts from pool[slot_idx[s]] (zero where has_initial[s] == 0) and writes
+    its final state back to that row; other rows are untouched.
+
+    Returns (y, new_pool), fp64.  Pure gather / scan / scatter around scan().
+    """
+    pool = _f64(pool)
+    slots = np.asarray(slot_idx, dtype=np.int64)
+    h0 = pool[slots].copy()
+    if has_initial is not None:
+        h0[np.asarray(has_initial) == 0] = 0.0
+    y, hT = scan(x, dt, A, B, C, D, h0, cu_seqlens=cu_seqlens)
+    out = pool.copy()
+    out[slots] = hT
+    return y, out
+
+
+def state_update_slots(pool, slot_idx, x, dt, A, B, C, D=None):
+    """One decode step on pool rows: batch row b updates pool[slot_idx[b]];
+    rows with a negative slot are padding (no update, y row NaN).
+
+    Returns (y, new_pool), fp64.
+    """
+    pool = _f64(pool)
+    slots = np.asarray(slot_idx, dtype=np.int64)
+    live = slots >= 0
+    out = pool.copy()
+    batch = slots.shape[0]
+    H, P = pool.shape[1], pool.shape[2]
+    y = np.full((batch, H, P), np.nan)
+    if live.any():
+        yl, st = state_update(pool[slots[live]], _f64(x)[live], _f64(dt)[live], A,
+                              _f64(B)[live], _f64(C)[live], D)
+        y[live] = yl
+        out[slots[live]] = st
+    return y, out

@@ -131,3 +131,56 @@ def test_update_rejects(lib, kw, code):
 
 def test_update_batch_zero_is_noop(lib):
     assert update(lib, batch=0, state=None, x=None) == OK
+
+
+@pytest.fixture(scope="module")
+def slib(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.ssd_chunk_scan_slots.restype = i
+    lib.ssd_chunk_scan_slots.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp,
+                                         vp, i, vp, vp, i, vp, vp, vp]
+    lib.ssm_state_update_slots.restype = i
+    lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp, vp,
+                                           i, vp, vp, vp]
+    return lib
+
+
+def scan_slots(lib, nseq=2, seqlen=128, H=4, P=64, N=128, G=1, pool=0x200000, max_slots=8,
+               slots=0x300000, has=None, x=A16, y=0x60000):
+    return lib.ssd_chunk_scan_slots(nseq, seqlen, None, H, P, N, G, 128, BF16, x, A16b, A16c,
+                                    0x40000, 0x50000, None, pool, max_slots, slots, has, BF16,
+                                    y, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(max_slots=0), INVALID),
+    (dict(pool=None), INVALID),
+    (dict(slots=None), INVALID),
+    (dict(slots=0x300004), MISALIGNED),
+    (dict(y=0x200000 + 4096), INVALID),     # y inside the pool
+    (dict(P=96), UNSUPPORTED),
+])
+def test_scan_slots_rejects(slib, kw, code):
+    assert scan_slots(slib, **kw) == code
+
+
+def test_scan_slots_nseq_zero_is_noop(slib):
+    assert scan_slots(slib, nseq=0, pool=None, slots=None, x=None, y=None) == OK
+
+
+def update_slots(lib, batch=2, H=4, P=64, N=128, G=2, pool=0x200000, max_slots=8,
+                 slots=0x300000, x=A16, y=0x60000):
+    return lib.ssm_state_update_slots(batch, H, P, N, G, BF16, pool, max_slots, slots, x, A16b,
+                                      A16c, 0x40000, 0x50000, None, F32, y, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(max_slots=-1), INVALID),
+    (dict(slots=None), INVALID),
+    (dict(x=None), INVALID),
+    (dict(pool=0x200008), MISALIGNED),
+    (dict(x=0x200000 + 512), INVALID),      # x inside the pool
+    (dict(N=48), UNSUPPORTED),
+])
+def test_update_slots_rejects(slib, kw, code):
+    assert update_slots(slib, **kw) == code

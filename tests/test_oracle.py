@@ -296,3 +296,42 @@ def test_pins_reject_planted_mistakes(tmp_path, name, monkeypatch):
             caught.append(pin)
     monkeypatch.setattr(oracle, "_lib", saved)
     assert caught, f"no pin rejects the planted mistake {name!r}"
+
+
+# ---------------------------------------------------------------------------
+# Slot-indexed state pools (gather / scan / scatter around the recurrence)
+# ---------------------------------------------------------------------------
+def test_slot_pool_scan_identity_and_permutation():
+    rng = np.random.default_rng(12)
+    lens = [7, 0, 12]
+    T = sum(lens)
+    x, dt, A, B, C, D, _ = rand_problem(rng, T, 4, 3, 5, 2, h0=False)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    pool = rng.standard_normal((6, 4, 3, 5))
+    slots = [4, 1, 0]
+    has = [1, 1, 0]
+    y, new_pool = oracle.scan_slots(pool, slots, has, x, dt, A, B, C, D, cu_seqlens=cu)
+    h0 = np.stack([pool[4], pool[1], np.zeros_like(pool[0])])
+    y_ref, hT_ref = oracle.scan(x, dt, A, B, C, D, h0, cu_seqlens=cu)
+    np.testing.assert_array_equal(y, y_ref)
+    np.testing.assert_array_equal(new_pool[[4, 1, 0]], hT_ref)
+    np.testing.assert_array_equal(new_pool[[2, 3, 5]], pool[[2, 3, 5]])   # untouched rows
+    np.testing.assert_array_equal(new_pool[1], pool[1])   # empty sequence keeps its slot
+
+
+def test_slot_pool_decode_padding_rows():
+    rng = np.random.default_rng(13)
+    pool = rng.standard_normal((5, 2, 3, 4))
+    slots = np.array([3, -1, 0])
+    x = rng.standard_normal((3, 2, 3))
+    dt = rng.uniform(0.01, 0.1, (3, 2))
+    A = -rng.uniform(0.5, 2, 2)
+    B = rng.standard_normal((3, 1, 4))
+    C = rng.standard_normal((3, 1, 4))
+    D = rng.standard_normal(2)
+    y, new_pool = oracle.state_update_slots(pool, slots, x, dt, A, B, C, D)
+    yr, st = oracle.state_update(pool[[3, 0]], x[[0, 2]], dt[[0, 2]], A, B[[0, 2]], C[[0, 2]], D)
+    np.testing.assert_array_equal(y[[0, 2]], yr)
+    assert np.isnan(y[1]).all()
+    np.testing.assert_array_equal(new_pool[[3, 0]], st)
+    np.testing.assert_array_equal(new_pool[[1, 2, 4]], pool[[1, 2, 4]])
