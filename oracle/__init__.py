@@ -67,6 +67,10 @@ def _load():
             lib.oracle_state_update.argtypes = [
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp]
+            lib.oracle_causal_conv1d.restype = ctypes.c_int
+            lib.oracle_causal_conv1d.argtypes = [
+                ctypes.c_int, _i64p, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, ctypes.c_int,
+                _dp, _dp]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -198,3 +202,43 @@ def state_update_slots(pool, slot_idx, x, dt, A, B, C, D=None):
         y[live] = yl
         out[slots[live]] = st
     return y, out
+
+
+def causal_conv1d(x, weight, bias=None, activation="silu", state=None, cu_seqlens=None):
+    """Causal depthwise conv1d over (packed) sequences, channels-last, in fp64.
+
+    x : [T, dim]; weight : [dim, K]; bias : [dim] or None;
+    activation : "silu" or None; state : [nseq, dim, K-1] or None (zeros
+    before each sequence start, and no state returned).
+    Returns (y [T, dim], new_state [nseq, dim, K-1] or None).
+    """
+    xf = _f64(x)
+    T, dim = xf.shape
+    wf = _f64(weight)
+    K = wf.shape[1]
+    if K - 1 > 64:
+        raise ValueError("conv width above 65 is not supported by the oracle")
+    cu = (np.array([0, T], dtype=np.int64) if cu_seqlens is None
+          else np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64)))
+    nseq = cu.shape[0] - 1
+    bf = None if bias is None else _f64(bias)
+    st = None if state is None else _f64(state).reshape(nseq, dim, K - 1).copy()
+    y = np.zeros((T, dim), dtype=np.float64)
+    rc = _load().oracle_causal_conv1d(nseq, cu.ctypes.data_as(_i64p), dim, K, _ptr(xf),
+                                      _ptr(wf), _ptr(bf), 1 if activation == "silu" else 0,
+                                      _ptr(st), _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle_causal_conv1d rejected its arguments ({rc})")
+    return y, st
+
+
+def causal_conv1d_update(x, weight, bias, state, activation="silu"):
+    """One decode token per row: window = [state (K-1 values), x] -> y; the
+    state rolls by one (drops its oldest value, appends x).
+
+    x : [batch, dim]; state : [batch, dim, K-1].  Returns (y, new_state), fp64.
+    """
+    xf = _f64(x)
+    batch = xf.shape[0]
+    cu = np.arange(batch + 1, dtype=np.int64)
+    return causal_conv1d(xf, weight, bias, activation, state, cu_seqlens=cu)

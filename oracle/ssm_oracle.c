@@ -162,3 +162,65 @@ int oracle_state_update(int batch, int H, int P, int N, int G,
     }
     return ORACLE_OK;
 }
+
+/*
+ * Causal depthwise conv1d with optional SiLU, over packed sequences in the
+ * channels-last layout ("Depthwise SiLU 卷积" of the MAX nemotron_h article,
+ * section 5.4 item 2; causal_conv1d_fn / causal_conv1d_update and the conv
+ * state of the modeling_nemotron_h.py walk-through, "Prefill 阶段" /
+ * "Decode 阶段").  For channel c, width K, token t of a sequence:
+ *
+ *   pre[t][c] = bias[c] + sum_{k=0}^{K-1} w[c][k] * in[t - (K-1) + k][c]
+ *   y[t][c]   = act(pre[t][c]),  act = identity or SiLU (v / (1 + exp(-v)))
+ *
+ * where in[t'] for t' < 0 is taken from the sequence's conv state
+ * (state[s][c][K-1+t'], its K-1 most recent earlier inputs, oldest first) or
+ * zero when no state is given.  Afterwards the state holds the K-1 most
+ * recent inputs (earlier state entries shift in when the sequence is short).
+ *
+ *   x [T][dim], w [dim][K], bias [dim] or NULL, state [nseq][dim][K-1] or
+ *   NULL (in/out), y [T][dim].
+ */
+static double conv_act(double v, int act)
+{
+    return act ? v / (1.0 + exp(-v)) : v;
+}
+
+int oracle_causal_conv1d(int nseq, const int64_t *cu_seqlens, int dim, int K,
+                         const double *x, const double *w, const double *bias, int act,
+                         double *state, double *y)
+{
+    if (nseq < 0 || dim <= 0 || K < 1) return ORACLE_BAD_ARG;
+    if (nseq == 0) return ORACLE_OK;
+    if (!cu_seqlens || !w) return ORACLE_BAD_ARG;
+
+#pragma omp parallel for schedule(static)
+    for (long sc = 0; sc < (long)nseq * dim; ++sc) {
+        const int s = (int)(sc / dim), c = (int)(sc % dim);
+        const int64_t t0 = cu_seqlens[s], t1 = cu_seqlens[s + 1];
+        double *st = state ? state + ((size_t)s * dim + c) * (size_t)(K - 1) : NULL;
+        for (int64_t t = t0; t < t1; ++t) {
+            double acc = bias ? bias[c] : 0.0;
+            for (int k = 0; k < K; ++k) {
+                const int64_t src = t - (K - 1) + k;        /* absolute token */
+                double v;
+                if (src >= t0) v = x[(size_t)src * dim + c];
+                else if (st) v = st[(K - 1) + (src - t0)];   /* src - t0 in [-(K-1), -1] */
+                else v = 0.0;
+                acc += w[(size_t)c * K + k] * v;
+            }
+            y[(size_t)t * dim + c] = conv_act(acc, act);
+        }
+        if (st && K > 1) {
+            /* new state: the K-1 most recent inputs (old state entries first) */
+            double win[64];
+            const int64_t L = t1 - t0;
+            for (int k = 0; k < K - 1; ++k) {
+                const int64_t src = L - (K - 1) + k;         /* relative to t0 */
+                win[k] = src >= 0 ? x[(size_t)(t0 + src) * dim + c] : st[(K - 1) + src];
+            }
+            for (int k = 0; k < K - 1; ++k) st[k] = win[k];
+        }
+    }
+    return ORACLE_OK;
+}
