@@ -227,6 +227,81 @@ def oracle_step_sample(rank_seed, prefill_tokens, prefill_heads, decode_rows):
     return step_s, desc, oracle.num_threads()
 
 
+CONV_PREFILL = dict(nseq=4, seqlen=4096, dim=128 * 64 + 2 * 8 * 128, width=4)
+CONV_DECODE = dict(batch=64, dim=256 * 64 + 2 * 8 * 128, width=4, ring=32)
+
+
+def conv_prefill_work(c=CONV_PREFILL):
+    """Algorithmic bytes of one causal_conv1d_fwd call (bf16 x and y, bf16
+    state read and written, fp32 weight and bias)."""
+    T = c["nseq"] * c["seqlen"]
+    W = c["width"]
+    return T * c["dim"] * 4 + 2 * c["nseq"] * c["dim"] * (W - 1) * 2 + c["dim"] * (W + 1) * 4, T
+
+
+def conv_decode_work(c=CONV_DECODE):
+    """Algorithmic bytes of one causal_conv1d_update call: x, y, the state
+    window read and written (bf16), weight, bias, slot indices."""
+    b, dim, W = c["batch"], c["dim"], c["width"]
+    return b * dim * (4 + 4 * (W - 1)) + dim * (W + 1) * 4 + b * 4, b
+
+
+def time_conv(dev, stream, seed, iters=50):
+    """Device time of the conv1d entry points at the benchmark shapes (run
+    beside the step, not inside it).  Prefill inputs exceed L2; decode cycles
+    through a ring of pool rows and inputs larger than L2."""
+    import torch
+    from hybrid_mamba_ssm_b200 import inputs as synth
+    from hybrid_mamba_ssm_b200 import ssm
+
+    def bf16(t):
+        return torch.from_numpy(np.ascontiguousarray(t.bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    cp, cd = CONV_PREFILL, CONV_DECODE
+    inp = synth.make_conv_inputs(seed, [cp["seqlen"]] * cp["nseq"], cp["dim"], cp["width"])
+    x = bf16(inp.x).view(cp["nseq"], cp["seqlen"], cp["dim"])
+    w = torch.from_numpy(inp.weight).to(dev)
+    b = torch.from_numpy(inp.bias).to(dev)
+    st = bf16(inp.state)
+    y = torch.empty_like(x)
+    rng = np.random.Generator(np.random.PCG64(seed + 1))
+    rows = cd["batch"] * cd["ring"]
+    pool = torch.from_numpy(rng.standard_normal((rows, cd["dim"], cd["width"] - 1),
+                                                dtype=np.float32)).to(dev).to(torch.bfloat16)
+    dx = torch.from_numpy(rng.standard_normal((cd["ring"], cd["batch"], cd["dim"]),
+                                              dtype=np.float32)).to(dev).to(torch.bfloat16)
+    dw = torch.from_numpy(rng.uniform(-0.5, 0.5, (cd["dim"], cd["width"])).astype(np.float32)).to(dev)
+    db = torch.from_numpy(rng.uniform(-0.5, 0.5, cd["dim"]).astype(np.float32)).to(dev)
+    slots = torch.arange(rows, dtype=torch.int32, device=dev).view(cd["ring"], cd["batch"])
+    dy = torch.empty((cd["batch"], cd["dim"]), dtype=torch.bfloat16, device=dev)
+
+    def pre():
+        ssm.causal_conv1d_fwd(x, w, b, conv_state=st, y=y, stream=stream)
+
+    def dec(k):
+        ssm.causal_conv1d_update(dx[k % cd["ring"]], dw, db, pool, slot_idx=slots[k % cd["ring"]],
+                                 y=dy, stream=stream)
+
+    out = {}
+    for name, fn, (nbytes, units) in (("conv1d_prefill", lambda k: pre(), conv_prefill_work()),
+                                      ("conv1d_decode", dec, conv_decode_work())):
+        for k in range(5):
+            fn(k)
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(iters)]
+        for k in range(iters):
+            ev[k][0].record(stream)
+            fn(k)
+            ev[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
+        out[name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "bytes_per_launch": nbytes,
+                     "tokens_per_s": units / (ms * 1e-3), "launches": iters}
+    return out
+
+
 def run_reference(args, world, rank, pg):
     if rank != 0:
         return 0
@@ -410,8 +485,12 @@ def run_ours(args, world, rank, local, pg):
     barrier(pg, dev)
     e2e_ms = max_over_ranks(pg, s2.elapsed_time(e2), dev)
 
+    conv = time_conv(dev, stream, seed + 17)
+
     # ---- numbers ----
     peaks, peak_kind = load_peaks()
+    for part in conv.values():
+        part["hbm_frac"] = part["gbs"] / peaks["hbm_gbs"]
     tok_step = p["nseq"] * p["seqlen"] + d["batch"]
     value = world * tok_step * K / (ms * 1e-3)
     e2e_value = world * tok_step * e2e_steps / (e2e_ms * 1e-3)
@@ -456,7 +535,7 @@ def run_ours(args, world, rank, local, pg):
                        "decode": dict(DECODE, in_dtype="bf16", y_dtype="bf16", ring=RING),
                        "l2": "inputs larger than L2 (about 1.7 GB touched per step)",
                        "parallelism": f"replicas x{world} (independent batches per GPU)"},
-            "parts": {"prefill": pre, "decode": dec},
+            "parts": {"prefill": pre, "decode": dec, **conv},
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,

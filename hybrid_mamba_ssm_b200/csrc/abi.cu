@@ -262,4 +262,87 @@ int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
     return ssm::launch_state_update(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
+int causal_conv1d_fwd(int nseq, int seqlen, const int32_t *cu_seqlens, int dim, int width,
+                      int in_dtype, const void *x, const float *weight, const float *bias,
+                      int activation, void *conv_state, int max_slots, const int32_t *slot_idx,
+                      const int32_t *has_initial_state, int y_dtype, void *y, int *status_dev,
+                      cudaStream_t stream)
+{
+    if (nseq < 0 || seqlen < 0 || dim <= 0) return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
+    if (activation != 0 && activation != 1) return SSM_ERR_INVALID_ARG;
+    if (width < 1) return SSM_ERR_INVALID_ARG;
+    if (width > 8 || nseq > 0x7fffffff / 2) return SSM_ERR_UNSUPPORTED;
+    if (cu_seqlens && nseq == 0 && seqlen != 0) return SSM_ERR_INVALID_ARG;
+    const long long T = cu_seqlens ? (long long)seqlen : (long long)nseq * seqlen;
+    if (nseq == 0 || (T == 0 && !conv_state)) return SSM_OK;
+    if (!weight || (T > 0 && (!x || !y))) return SSM_ERR_INVALID_ARG;
+    if (slot_idx && (!conv_state || max_slots <= 0)) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {cu_seqlens, x, weight, bias, conv_state, slot_idx, has_initial_state,
+                          y, status_dev};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+    const size_t es = dtype_size(in_dtype);
+    const long long rows = slot_idx ? max_slots : nseq;
+    const Range rs = range_of(conv_state, conv_state ? (size_t)rows * dim * (width - 1) * es : 0);
+    const Range ry = range_of(y, (size_t)T * dim * dtype_size(y_dtype));
+    const Range ins[] = {range_of(x, (size_t)T * dim * es),
+                         range_of(weight, (size_t)dim * width * sizeof(float)),
+                         range_of(bias, bias ? (size_t)dim * sizeof(float) : 0),
+                         range_of(cu_seqlens, cu_seqlens ? (size_t)(nseq + 1) * sizeof(int32_t) : 0),
+                         range_of(slot_idx, slot_idx ? (size_t)nseq * sizeof(int32_t) : 0),
+                         range_of(has_initial_state,
+                                  has_initial_state ? (size_t)nseq * sizeof(int32_t) : 0)};
+    for (const Range &r : ins)
+        if (overlap(ry, r) || overlap(rs, r)) return SSM_ERR_INVALID_ARG;
+    if (overlap(ry, rs)) return SSM_ERR_INVALID_ARG;
+
+    ssm::ConvArgs a{};
+    a.update = 0; a.nseq = nseq; a.seqlen = seqlen; a.cu_seqlens = cu_seqlens;
+    a.dim = dim; a.width = width; a.activation = activation;
+    a.in_dtype = in_dtype; a.y_dtype = y_dtype;
+    a.x = x; a.weight = weight; a.bias = bias; a.state = conv_state;
+    a.slot_idx = slot_idx; a.has_initial = has_initial_state; a.max_slots = max_slots;
+    a.y = y; a.status_dev = status_dev;
+    return ssm::launch_conv1d(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int causal_conv1d_update(int batch, int dim, int width, int in_dtype, const void *x,
+                         const float *weight, const float *bias, int activation,
+                         void *conv_state, int max_slots, const int32_t *slot_idx,
+                         int y_dtype, void *y, int *status_dev, cudaStream_t stream)
+{
+    if (batch < 0 || dim <= 0) return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
+    if (activation != 0 && activation != 1) return SSM_ERR_INVALID_ARG;
+    if (width < 1) return SSM_ERR_INVALID_ARG;
+    if (width > 8) return SSM_ERR_UNSUPPORTED;
+    if (batch == 0) return SSM_OK;
+    if (!x || !weight || !y || (width > 1 && !conv_state)) return SSM_ERR_INVALID_ARG;
+    if (slot_idx && max_slots <= 0) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, weight, bias, conv_state, slot_idx, y, status_dev};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+    const size_t es = dtype_size(in_dtype);
+    const long long rows = slot_idx ? max_slots : batch;
+    const Range rs = range_of(conv_state, conv_state ? (size_t)rows * dim * (width - 1) * es : 0);
+    const Range ry = range_of(y, (size_t)batch * dim * dtype_size(y_dtype));
+    const Range ins[] = {range_of(x, (size_t)batch * dim * es),
+                         range_of(weight, (size_t)dim * width * sizeof(float)),
+                         range_of(bias, bias ? (size_t)dim * sizeof(float) : 0),
+                         range_of(slot_idx, slot_idx ? (size_t)batch * sizeof(int32_t) : 0)};
+    for (const Range &r : ins)
+        if (overlap(ry, r) || overlap(rs, r)) return SSM_ERR_INVALID_ARG;
+    if (overlap(ry, rs)) return SSM_ERR_INVALID_ARG;
+
+    ssm::ConvArgs a{};
+    a.update = 1; a.nseq = batch; a.seqlen = 1;
+    a.dim = dim; a.width = width; a.activation = activation;
+    a.in_dtype = in_dtype; a.y_dtype = y_dtype;
+    a.x = x; a.weight = weight; a.bias = bias; a.state = conv_state;
+    a.slot_idx = slot_idx; a.max_slots = max_slots;
+    a.y = y; a.status_dev = status_dev;
+    return ssm::launch_conv1d(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -1,0 +1,545 @@
+// conv1d.cu -- causal depthwise conv1d (+ optional SiLU) in the channels-last
+// layout, the short convolution that produces the scan's x, B and C
+// ("Depthwise SiLU 卷积" of the MAX nemotron_h article, section 5.4 item 2;
+// causal_conv1d_fn / causal_conv1d_update of the modeling_nemotron_h.py
+// walk-through).  For channel c, width K and token t of a sequence:
+//
+//   y[t][c] = act(bias[c] + sum_{k<K} w[c][k] * in[t - (K-1) + k][c])
+//
+// where the inputs before the sequence start come from its conv state (the
+// K-1 most recent earlier inputs, oldest first) or are zero.  Afterwards the
+// state holds the sequence's K-1 most recent inputs.
+//
+// Prefill runs as two launches: the convolution over 64-token tiles of the
+// packed stream (several tiles of one sequence read its old state
+// concurrently), then one pass per (sequence, channel) that rolls the state.
+// Decode is one launch per token batch; the window rolls in place.
+// All three are bound by HBM: each input and output is touched once.
+#include "common.cuh"
+#include "ssm_internal.h"
+
+namespace ssm {
+
+constexpr int kConvThreads = 256;   // channels per CTA
+constexpr int kConvTile = 64;       // tokens per CTA
+constexpr int kMaxWidth = 8;
+
+// SiLU as v * (1 / (1 + e^-v)) with the hardware approximate reciprocal
+// (rcp of +inf is 0, so large negative v gives -0 as the limit does).
+__device__ __forceinline__ float rcp_approx(float v) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+__device__ __forceinline__ float conv_act(float v, int act) {
+    return act ? v * rcp_approx(1.f + __expf(-v)) : v;
+}
+
+__device__ __forceinline__ float ld_in(const float *p) { return *p; }
+__device__ __forceinline__ float ld_in(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void st_in(float *p, float v) { *p = v; }
+__device__ __forceinline__ void st_in(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+// Prefill state row of sequence s: >= 0 a row of the state (or pool), -1 no
+// state given, -2 a slot index outside [0, max_slots) (reported; the sequence
+// is skipped, as the scan does).
+__device__ __forceinline__ long conv_state_row(const ConvArgs &a, int s, bool &load_init) {
+    load_init = a.state != nullptr;
+    if (!a.state) return -1;
+    if (a.has_initial && a.has_initial[s] == 0) load_init = false;
+    if (!a.slot_idx) return s;
+    const int slot = a.slot_idx[s];
+    if (slot < 0 || slot >= a.max_slots) {
+        report_status(a.status_dev, 6);
+        return -2;
+    }
+    return slot;
+}
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kConvThreads)
+conv1d_fwd_kernel(ConvArgs a)
+{
+    const int c = blockIdx.y * kConvThreads + threadIdx.x;
+    const long tok0 = (long)blockIdx.x * kConvTile;
+    const long T = a.cu_seqlens ? (long)a.seqlen : (long)a.nseq * a.seqlen;
+    if (tok0 >= T) return;
+    const long tok1 = min(tok0 + kConvTile, T);
+    const int K = a.width, dim = a.dim;
+    const TIn *x = static_cast<const TIn *>(a.x);
+    const TIn *st = static_cast<const TIn *>(a.state);
+    TOut *y = static_cast<TOut *>(a.y);
+
+    // sequence holding tok0 (last s with start <= tok0 and end > tok0)
+    __shared__ int s_seq;
+    if (threadIdx.x == 0) {
+        int s;
+        if (a.cu_seqlens) {
+            int lo = 0, hi = a.nseq - 1;
+            while (lo < hi) {   // largest s with cu[s] <= tok0
+                const int mid = (lo + hi + 1) >> 1;
+                if (a.cu_seqlens[mid] <= tok0) lo = mid; else hi = mid - 1;
+            }
+            s = lo;
+            while (s + 1 < a.nseq && a.cu_seqlens[s + 1] <= tok0) ++s;
+        } else {
+            s = (int)(tok0 / a.seqlen);
+        }
+        s_seq = s;
+    }
+    __syncthreads();
+    if (c >= dim) return;
+
+    float w[kMaxWidth];
+#pragma unroll
+    for (int k = 0; k < kMaxWidth; ++k) w[k] = (k < K) ? a.weight[(size_t)c * K + k] : 0.f;
+    const float bias = a.bias ? a.bias[c] : 0.f;
+
+    int s = s_seq;
+    auto seq_start = [&](int q) -> long { return a.cu_seqlens ? (long)a.cu_seqlens[q] : (long)q * a.seqlen; };
+    auto seq_end = [&](int q) -> long { return a.cu_seqlens ? (long)a.cu_seqlens[q + 1] : (long)(q + 1) * a.seqlen; };
+
+    // window: win[K-2] is the input just before the current token
+    float win[kMaxWidth - 1];
+    bool skip = false;
+    auto load_window = [&](long t) {
+        const long ts = seq_start(s);
+        bool load_init;
+        const long row = conv_state_row(a, s, load_init);
+        skip = row == -2;
+#pragma unroll
+        for (int j = 0; j < kMaxWidth - 1; ++j) {
+            float v = 0.f;
+            if (j < K - 1) {
+                const long src = t - (K - 1) + j;   // absolute token of window slot j
+                if (src >= ts && src >= 0) v = ld_in(x + (size_t)src * dim + c);
+                else if (row >= 0 && load_init && src - ts >= -(K - 1))
+                    v = ld_in(st + ((size_t)row * dim + c) * (K - 1) + (K - 1) + (src - ts));
+            }
+            win[j] = v;
+        }
+    };
+    load_window(tok0);
+    long te = seq_end(s);
+    for (long t = tok0; t < tok1; ++t) {
+        if (t >= te) {   // next sequence (skipping empty ones)
+            do { ++s; } while (s + 1 < a.nseq && seq_end(s) <= t);
+            if (s >= a.nseq) {   // offsets end before T: reported by the state pass
+                report_status(a.status_dev, 6);
+                return;
+            }
+            te = seq_end(s);
+            load_window(t);
+        }
+        const float cur = ld_in(x + (size_t)t * dim + c);
+        float acc = bias;
+#pragma unroll
+        for (int j = 0; j < kMaxWidth - 1; ++j)
+            if (j < K - 1) acc = fmaf(w[j], win[j], acc);
+        acc = fmaf(w[K - 1], cur, acc);
+        if (!skip) store_out(y + (size_t)t * dim + c, conv_act(acc, a.activation));
+#pragma unroll
+        for (int j = 0; j < kMaxWidth - 1; ++j) {
+            if (j < K - 2) win[j] = win[j + 1];
+            else if (j == K - 2) win[j] = cur;
+        }
+    }
+}
+
+// Vectorised form for dim % V == 0: each thread owns V adjacent channels
+// (one 16-byte load per token row: 8 bf16 or 4 fp32), the width is a
+// template constant, and tiles whose whole window lies inside one sequence
+// (all but the tiles at a sequence start) issue 8 row loads before using
+// any, so every warp keeps 4 KB of loads in flight.
+template <typename T> struct ConvVec;
+template <> struct ConvVec<__nv_bfloat16> { static constexpr int V = 8; using Raw = uint4; };
+template <> struct ConvVec<float> { static constexpr int V = 4; using Raw = float4; };
+
+constexpr int kVecThreads = 128;
+constexpr int kVecUnroll = 8;
+
+__device__ __forceinline__ void unpack_row(const uint4 &r, float (&f)[8]) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 v = __bfloat1622float2(h[i]);
+        f[2 * i] = v.x;
+        f[2 * i + 1] = v.y;
+    }
+}
+__device__ __forceinline__ void unpack_row(const float4 &r, float (&f)[4]) {
+    f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w;
+}
+
+template <int V>
+__device__ __forceinline__ void store_row(float *p, const float (&v)[V]) {
+#pragma unroll
+    for (int i = 0; i < V / 4; ++i)
+        reinterpret_cast<float4 *>(p)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+template <int V>
+__device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float (&v)[V]) {
+    uint32_t w[V / 2];
+#pragma unroll
+    for (int i = 0; i < V / 2; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    if constexpr (V == 8) *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    else *reinterpret_cast<uint2 *>(p) = make_uint2(w[0], w[1]);
+}
+
+template <typename TIn>
+__device__ __forceinline__ typename ConvVec<TIn>::Raw load_row(const TIn *p) {
+    return __ldg(reinterpret_cast<const typename ConvVec<TIn>::Raw *>(p));
+}
+
+template <typename TIn, typename TOut, int K>
+__global__ void __launch_bounds__(kVecThreads)
+conv1d_fwd_vec_kernel(ConvArgs a)
+{
+    constexpr int V = ConvVec<TIn>::V;
+    constexpr int W = K > 1 ? K - 1 : 1;        // window slots (at least one)
+    using Raw = typename ConvVec<TIn>::Raw;
+    const int c0 = (blockIdx.y * kVecThreads + threadIdx.x) * V;
+    const long tok0 = (long)blockIdx.x * kConvTile;
+    const long T = a.cu_seqlens ? (long)a.seqlen : (long)a.nseq * a.seqlen;
+    if (tok0 >= T) return;
+    const long tok1 = min(tok0 + kConvTile, T);
+    const int dim = a.dim;
+    const TIn *x = static_cast<const TIn *>(a.x);
+    TOut *y = static_cast<TOut *>(a.y);
+
+    __shared__ int s_seq;
+    if (threadIdx.x == 0) {
+        int s;
+        if (a.cu_seqlens) {
+            int lo = 0, hi = a.nseq - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (a.cu_seqlens[mid] <= tok0) lo = mid; else hi = mid - 1;
+            }
+            s = lo;
+        } else {
+            s = (int)(tok0 / a.seqlen);
+        }
+        s_seq = s;
+    }
+    __syncthreads();
+    if (c0 >= dim) return;
+
+    float w[V][K], bias[V];
+#pragma unroll
+    for (int i = 0; i < V * K / 4; ++i) {
+        const float4 q = __ldg(reinterpret_cast<const float4 *>(a.weight + (size_t)c0 * K) + i);
+        const float e[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[(4 * i + j) / K][(4 * i + j) % K] = e[j];
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v) bias[v] = a.bias ? __ldg(a.bias + c0 + v) : 0.f;
+
+    int s = s_seq;
+    auto seq_start = [&](int q) -> long { return a.cu_seqlens ? (long)a.cu_seqlens[q] : (long)q * a.seqlen; };
+    auto seq_end = [&](int q) -> long { return a.cu_seqlens ? (long)a.cu_seqlens[q + 1] : (long)(q + 1) * a.seqlen; };
+    long ts = seq_start(s), te = seq_end(s);
+
+    float win[W][V];   // win[j] = inputs of token t-(K-1)+j
+    auto step = [&](long t, const float (&cur)[V], bool write) {
+        float out[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            float acc = bias[v];
+#pragma unroll
+            for (int j = 0; j < K - 1; ++j) acc = fmaf(w[v][j], win[j][v], acc);
+            acc = fmaf(w[v][K - 1], cur[v], acc);
+            out[v] = conv_act(acc, a.activation);
+        }
+        if (write) store_row<V>(y + (size_t)t * dim + c0, out);
+#pragma unroll
+        for (int j = 0; j < K - 2; ++j)
+#pragma unroll
+            for (int v = 0; v < V; ++v) win[j][v] = win[j + 1][v];
+        if (K > 1)
+#pragma unroll
+            for (int v = 0; v < V; ++v) win[W - 1][v] = cur[v];
+    };
+
+    if (tok0 - (K - 1) >= ts && tok0 - (K - 1) >= 0 && tok1 <= te) {
+        // fast path: the window and the tile lie inside one sequence
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) {
+            float f[V];
+            unpack_row(load_row(x + (size_t)(tok0 - (K - 1) + j) * dim + c0), f);
+#pragma unroll
+            for (int v = 0; v < V; ++v) win[j][v] = f[v];
+        }
+        for (long t = tok0; t < tok1; t += kVecUnroll) {
+            Raw r[kVecUnroll];
+#pragma unroll
+            for (int u = 0; u < kVecUnroll; ++u)
+                if (t + u < tok1) r[u] = load_row(x + (size_t)(t + u) * dim + c0);
+#pragma unroll
+            for (int u = 0; u < kVecUnroll; ++u) {
+                if (t + u < tok1) {
+                    float cur[V];
+                    unpack_row(r[u], cur);
+                    step(t + u, cur, true);
+                }
+            }
+        }
+        return;
+    }
+
+    // general path: sequence starts (state or zeros) inside the tile
+    const TIn *st = static_cast<const TIn *>(a.state);
+    bool skip = false;
+    auto load_window = [&](long t) {
+        bool load_init;
+        const long row = conv_state_row(a, s, load_init);
+        skip = row == -2;
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) {
+            const long src = t - (K - 1) + j;
+            if (src >= ts && src >= 0) {
+                float f[V];
+                unpack_row(load_row(x + (size_t)src * dim + c0), f);
+#pragma unroll
+                for (int v = 0; v < V; ++v) win[j][v] = f[v];
+            } else {
+#pragma unroll
+                for (int v = 0; v < V; ++v)
+                    win[j][v] = (row >= 0 && load_init)
+                        ? ld_in(st + ((size_t)row * dim + c0 + v) * (K - 1) + (K - 1) + (src - ts))
+                        : 0.f;
+            }
+        }
+    };
+    load_window(tok0);
+    for (long t = tok0; t < tok1; ++t) {
+        if (t >= te) {
+            do { ++s; } while (s + 1 < a.nseq && seq_end(s) <= t);
+            if (s >= a.nseq) {
+                report_status(a.status_dev, 6);
+                return;
+            }
+            ts = seq_start(s);
+            te = seq_end(s);
+            load_window(t);
+        }
+        float cur[V];
+        unpack_row(load_row(x + (size_t)t * dim + c0), cur);
+        step(t, cur, !skip);
+    }
+}
+
+// New conv state of each sequence: its K-1 most recent inputs, with older
+// state entries (or zeros) shifting in when the sequence is shorter.
+template <typename TIn>
+__global__ void __launch_bounds__(kConvThreads)
+conv1d_state_kernel(ConvArgs a)
+{
+    const int c = blockIdx.y * kConvThreads + threadIdx.x;
+    const int s = blockIdx.x;
+    if (c >= a.dim) return;
+    const int K = a.width, dim = a.dim;
+    long t0, t1;
+    if (a.cu_seqlens) {
+        t0 = a.cu_seqlens[s]; t1 = a.cu_seqlens[s + 1];
+        if (a.cu_seqlens[0] != 0 || t1 < t0 || t0 < 0 || t1 > a.seqlen ||
+            a.cu_seqlens[a.nseq] != a.seqlen) {
+            if (c == 0) report_status(a.status_dev, 6);
+            return;
+        }
+    } else {
+        t0 = (long)s * a.seqlen; t1 = t0 + a.seqlen;
+    }
+    bool load_init;
+    const long row = conv_state_row(a, s, load_init);
+    if (row < 0) return;
+    const TIn *x = static_cast<const TIn *>(a.x);
+    TIn *st = static_cast<TIn *>(a.state) + ((size_t)row * dim + c) * (K - 1);
+    float nw[kMaxWidth - 1];
+    const long L = t1 - t0;
+#pragma unroll
+    for (int k = 0; k < kMaxWidth - 1; ++k) {
+        if (k >= K - 1) break;
+        const long src = L - (K - 1) + k;
+        nw[k] = src >= 0 ? ld_in(x + (size_t)(t0 + src) * dim + c)
+                         : (load_init ? ld_in(st + (K - 1) + src) : 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxWidth - 1; ++k)
+        if (k < K - 1) st_in(st + k, nw[k]);
+}
+
+// Decode: one token per batch row; the window rolls in place.
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kConvThreads)
+conv1d_update_kernel(ConvArgs a)
+{
+    const int c = blockIdx.y * kConvThreads + threadIdx.x;
+    const int b = blockIdx.x;
+    if (c >= a.dim) return;
+    const int K = a.width, dim = a.dim;
+    long row = b;
+    if (a.slot_idx) {
+        const int slot = a.slot_idx[b];
+        if (slot < 0) return;                   // padding row
+        if (slot >= a.max_slots) {
+            if (c == 0) report_status(a.status_dev, 6);
+            return;
+        }
+        row = slot;
+    }
+    TIn *st = static_cast<TIn *>(a.state) + ((size_t)row * dim + c) * (K - 1);
+    const float cur = ld_in(static_cast<const TIn *>(a.x) + (size_t)b * dim + c);
+    float acc = a.bias ? a.bias[c] : 0.f;
+    float win[kMaxWidth - 1];
+#pragma unroll
+    for (int j = 0; j < kMaxWidth - 1; ++j) {
+        win[j] = (j < K - 1) ? ld_in(st + j) : 0.f;
+        if (j < K - 1) acc = fmaf(a.weight[(size_t)c * K + j], win[j], acc);
+    }
+    acc = fmaf(a.weight[(size_t)c * K + K - 1], cur, acc);
+    store_out(static_cast<TOut *>(a.y) + (size_t)b * dim + c, conv_act(acc, a.activation));
+#pragma unroll
+    for (int j = 0; j < kMaxWidth - 1; ++j) {
+        if (j < K - 2) st_in(st + j, win[j + 1]);
+        else if (j == K - 2) st_in(st + j, cur);
+    }
+}
+
+// Vectorised decode for dim % V == 0: V adjacent channels per thread, whose
+// state windows are (K-1) consecutive 16-byte vectors of the state row.
+template <typename TIn, typename TOut, int K>
+__global__ void __launch_bounds__(kVecThreads)
+conv1d_update_vec_kernel(ConvArgs a)
+{
+    constexpr int V = ConvVec<TIn>::V;
+    constexpr int W = K > 1 ? K - 1 : 1;
+    using Raw = typename ConvVec<TIn>::Raw;
+    const int c0 = (blockIdx.y * kVecThreads + threadIdx.x) * V;
+    const int b = blockIdx.x;
+    const int dim = a.dim;
+    if (c0 >= dim) return;
+    long row = b;
+    if (a.slot_idx) {
+        const int slot = __ldg(a.slot_idx + b);
+        if (slot < 0) return;                   // padding row
+        if (slot >= a.max_slots) {
+            if (c0 == 0) report_status(a.status_dev, 6);
+            return;
+        }
+        row = slot;
+    }
+    float cur[V];
+    unpack_row(load_row(static_cast<const TIn *>(a.x) + (size_t)b * dim + c0), cur);
+    // state of channels c0..c0+V-1: V*(K-1) values, channel-major
+    TIn *st = static_cast<TIn *>(a.state) + ((size_t)row * dim + c0) * (K - 1);
+    float sv[W * V];
+#pragma unroll
+    for (int i = 0; i < K - 1; ++i) {
+        float f[V];
+        unpack_row(*reinterpret_cast<const Raw *>(st + (size_t)i * V), f);
+#pragma unroll
+        for (int j = 0; j < V; ++j) sv[i * V + j] = f[j];
+    }
+    float w[V * K], out[V];
+#pragma unroll
+    for (int i = 0; i < V * K / 4; ++i) {
+        const float4 q = __ldg(reinterpret_cast<const float4 *>(a.weight + (size_t)c0 * K) + i);
+        w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        float acc = a.bias ? __ldg(a.bias + c0 + v) : 0.f;
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) acc = fmaf(w[v * K + j], sv[v * (K - 1) + j], acc);
+        acc = fmaf(w[v * K + K - 1], cur[v], acc);
+        out[v] = conv_act(acc, a.activation);
+    }
+    store_row<V>(static_cast<TOut *>(a.y) + (size_t)b * dim + c0, out);
+    if (K > 1) {
+        // roll: channel v keeps its last K-2 entries and appends cur[v]
+        float nv[W * V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+#pragma unroll
+            for (int j = 0; j < K - 2; ++j) nv[v * (K - 1) + j] = sv[v * (K - 1) + j + 1];
+            nv[v * (K - 1) + K - 2] = cur[v];
+        }
+#pragma unroll
+        for (int i = 0; i < K - 1; ++i) {
+            float f[V];
+#pragma unroll
+            for (int j = 0; j < V; ++j) f[j] = nv[i * V + j];
+            store_row<V>(st + (size_t)i * V, f);
+        }
+    }
+}
+
+template <typename TIn, typename TOut>
+static cudaError_t launch_conv_t(const ConvArgs &a, cudaStream_t stream)
+{
+    const unsigned cblocks = (unsigned)((a.dim + kConvThreads - 1) / kConvThreads);
+    constexpr int V = ConvVec<TIn>::V;
+    if (a.update) {
+        if (a.dim % V == 0) {
+            const dim3 grid((unsigned)a.nseq, (unsigned)((a.dim / V + kVecThreads - 1) / kVecThreads));
+            switch (a.width) {
+            case 1: conv1d_update_vec_kernel<TIn, TOut, 1><<<grid, kVecThreads, 0, stream>>>(a); break;
+            case 2: conv1d_update_vec_kernel<TIn, TOut, 2><<<grid, kVecThreads, 0, stream>>>(a); break;
+            case 3: conv1d_update_vec_kernel<TIn, TOut, 3><<<grid, kVecThreads, 0, stream>>>(a); break;
+            case 4: conv1d_update_vec_kernel<TIn, TOut, 4><<<grid, kVecThreads, 0, stream>>>(a); break;
+            case 5: conv1d_update_vec_kernel<TIn, TOut, 5><<<grid, kVecThreads, 0, stream>>>(a); break;
+            case 6: conv1d_update_vec_kernel<TIn, TOut, 6><<<grid, kVecThreads, 0, stream>>>(a); break;
+            case 7: conv1d_update_vec_kernel<TIn, TOut, 7><<<grid, kVecThreads, 0, stream>>>(a); break;
+            default: conv1d_update_vec_kernel<TIn, TOut, 8><<<grid, kVecThreads, 0, stream>>>(a); break;
+            }
+        } else {
+            conv1d_update_kernel<TIn, TOut><<<dim3((unsigned)a.nseq, cblocks), kConvThreads, 0, stream>>>(a);
+        }
+        return cudaGetLastError();
+    }
+    const long T = a.cu_seqlens ? (long)a.seqlen : (long)a.nseq * a.seqlen;
+    if (T > 0 && a.dim % V == 0) {
+        const unsigned tiles = (unsigned)((T + kConvTile - 1) / kConvTile);
+        const unsigned vblocks = (unsigned)((a.dim / V + kVecThreads - 1) / kVecThreads);
+        const dim3 grid(tiles, vblocks);
+        switch (a.width) {
+        case 1: conv1d_fwd_vec_kernel<TIn, TOut, 1><<<grid, kVecThreads, 0, stream>>>(a); break;
+        case 2: conv1d_fwd_vec_kernel<TIn, TOut, 2><<<grid, kVecThreads, 0, stream>>>(a); break;
+        case 3: conv1d_fwd_vec_kernel<TIn, TOut, 3><<<grid, kVecThreads, 0, stream>>>(a); break;
+        case 4: conv1d_fwd_vec_kernel<TIn, TOut, 4><<<grid, kVecThreads, 0, stream>>>(a); break;
+        case 5: conv1d_fwd_vec_kernel<TIn, TOut, 5><<<grid, kVecThreads, 0, stream>>>(a); break;
+        case 6: conv1d_fwd_vec_kernel<TIn, TOut, 6><<<grid, kVecThreads, 0, stream>>>(a); break;
+        case 7: conv1d_fwd_vec_kernel<TIn, TOut, 7><<<grid, kVecThreads, 0, stream>>>(a); break;
+        default: conv1d_fwd_vec_kernel<TIn, TOut, 8><<<grid, kVecThreads, 0, stream>>>(a); break;
+        }
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    } else if (T > 0) {
+        const unsigned tiles = (unsigned)((T + kConvTile - 1) / kConvTile);
+        conv1d_fwd_kernel<TIn, TOut><<<dim3(tiles, cblocks), kConvThreads, 0, stream>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (a.state && a.width > 1) {
+        conv1d_state_kernel<TIn><<<dim3((unsigned)a.nseq, cblocks), kConvThreads, 0, stream>>>(a);
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_conv1d(const ConvArgs &a, cudaStream_t stream)
+{
+    const bool in_bf16 = a.in_dtype == 1, out_bf16 = a.y_dtype == 1;
+    if (in_bf16 && out_bf16) return launch_conv_t<__nv_bfloat16, __nv_bfloat16>(a, stream);
+    if (in_bf16) return launch_conv_t<__nv_bfloat16, float>(a, stream);
+    if (out_bf16) return launch_conv_t<float, __nv_bfloat16>(a, stream);
+    return launch_conv_t<float, float>(a, stream);
+}
+
+}  // namespace ssm

@@ -44,7 +44,27 @@ struct ScanArgs {
     int max_slots;
 };
 
+// Causal depthwise conv1d (prefill over packed sequences, or one decode token
+// per batch row when update != 0; then nseq is the batch).
+struct ConvArgs {
+    int update;
+    int nseq, seqlen;             // seqlen = T when cu_seqlens is given
+    const int32_t *cu_seqlens;
+    int dim, width, activation;   // activation: 0 none, 1 SiLU
+    int in_dtype, y_dtype;
+    const void *x;
+    const float *weight;          // [dim][width]
+    const float *bias;            // [dim] or nullptr
+    void *state;                  // [rows][dim][width-1], in_dtype, or nullptr
+    const int32_t *slot_idx;      // rows map, or nullptr
+    const int32_t *has_initial;
+    int max_slots;
+    void *y;
+    int *status_dev;
+};
+
 cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);
+cudaError_t launch_conv1d(const ConvArgs &a, cudaStream_t stream);
 
 // General chunked scan on the CUDA cores: any supported shape and dtype.
 cudaError_t launch_scan_simt(const ScanArgs &a, cudaStream_t stream);

@@ -152,6 +152,38 @@ def make_state(seed: int, shape, std: float = 0.1) -> np.ndarray:
     return (std * rng.standard_normal(shape, dtype=np.float32)).astype(np.float32)
 
 
+@dataclass
+class ConvInputs:
+    """Inputs of one causal depthwise conv1d call over packed sequences."""
+    x: Tensor16              # [T, dim]
+    weight: np.ndarray       # fp32 [dim, width]
+    bias: np.ndarray         # fp32 [dim]
+    state: Tensor16          # [nseq, dim, width-1], same storage as x
+    cu_seqlens: np.ndarray   # int32 [nseq+1]
+
+
+def conv_dim(nheads: int, head_dim: int, ngroups: int, d_state: int) -> int:
+    """Channels of the short convolution: x (nheads*head_dim), B and C
+    (ngroups*d_state each) side by side."""
+    return nheads * head_dim + 2 * ngroups * d_state
+
+
+def make_conv_inputs(seed: int, seqlens, dim: int, width: int = 4,
+                     dtype: str = "bf16") -> ConvInputs:
+    """x, state ~ N(0, 1); weight, bias ~ U(-1/sqrt(width), 1/sqrt(width))."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lens = [int(v) for v in seqlens]
+    T = sum(lens)
+    cu = np.zeros(len(lens) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lens)
+    x = _store(rng.standard_normal((T, dim), dtype=np.float32), dtype)
+    bound = 1.0 / np.sqrt(width)
+    weight = rng.uniform(-bound, bound, (dim, width)).astype(np.float32)
+    bias = rng.uniform(-bound, bound, dim).astype(np.float32)
+    state = _store(rng.standard_normal((len(lens), dim, width - 1), dtype=np.float32), dtype)
+    return ConvInputs(x=x, weight=weight, bias=bias, state=state, cu_seqlens=cu)
+
+
 def mixed_seqlens(seed: int, nseq: int = 8, lo: int = 512, hi: int = 16384):
     """Sequence lengths drawn uniformly from the integers lo..hi."""
     rng = np.random.Generator(np.random.PCG64(seed))

@@ -2,6 +2,8 @@
 
     python -m hybrid_mamba_ssm_b200.profile_cases prefill --nseq 1 --seqlen 4096 --heads 128
     python -m hybrid_mamba_ssm_b200.profile_cases decode --batch 16 --heads 256
+    python -m hybrid_mamba_ssm_b200.profile_cases conv --nseq 1 --seqlen 8192
+    python -m hybrid_mamba_ssm_b200.profile_cases conv_update --batch 64
 
 Each case draws seeded inputs, runs ``--warmup`` untimed launches and then
 ``--launches`` more, and prints the device time of the last ones.  Inputs are
@@ -54,9 +56,32 @@ def decode(args, dev):
     return lambda: ssm.ssm_state_update(state, x, dt, A, Bt, Ct, D, y=y)
 
 
+def conv(args, dev):
+    dim = synth.conv_dim(args.heads, args.head_dim, args.groups, args.d_state)
+    inp = synth.make_conv_inputs(81, [args.seqlen] * args.nseq, dim, args.width)
+    x = _bf16(inp.x, dev).view(args.nseq, args.seqlen, dim)
+    w, b = _f32(inp.weight, dev), _f32(inp.bias, dev)
+    st = _bf16(inp.state, dev)
+    y = torch.empty_like(x)
+    return lambda: ssm.causal_conv1d_fwd(x, w, b, conv_state=st, y=y)
+
+
+def conv_update(args, dev):
+    dim = synth.conv_dim(args.heads, args.head_dim, args.groups, args.d_state)
+    inp = synth.make_conv_inputs(82, [1] * args.batch, dim, args.width)
+    x = _bf16(inp.x, dev)
+    w, b = _f32(inp.weight, dev), _f32(inp.bias, dev)
+    st = _bf16(inp.state, dev)
+    y = torch.empty_like(x)
+    return lambda: ssm.causal_conv1d_update(x, w, b, st, y=y)
+
+
+CASES = {"prefill": prefill, "decode": decode, "conv": conv, "conv_update": conv_update}
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["prefill", "decode"])
+    ap.add_argument("case", choices=sorted(CASES))
     ap.add_argument("--nseq", type=int, default=1)
     ap.add_argument("--seqlen", type=int, default=4096)
     ap.add_argument("--batch", type=int, default=16)
@@ -65,13 +90,14 @@ def main():
     ap.add_argument("--d-state", type=int, default=128)
     ap.add_argument("--groups", type=int, default=8)
     ap.add_argument("--chunk", type=int, default=128)
+    ap.add_argument("--width", type=int, default=4)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--launches", type=int, default=1)
     args = ap.parse_args()
     if args.heads is None:
-        args.heads = 128 if args.case == "prefill" else 256
+        args.heads = 128 if args.case in ("prefill", "conv") else 256
     dev = torch.device("cuda", 0)
-    run = prefill(args, dev) if args.case == "prefill" else decode(args, dev)
+    run = CASES[args.case](args, dev)
     for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()

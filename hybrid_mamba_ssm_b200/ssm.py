@@ -20,7 +20,9 @@ STATUS_NAMES = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED",
                 3: "SSM_ERR_MISALIGNED", 4: "SSM_ERR_CUDA", 5: "SSM_ERR_TIMEOUT",
                 6: "SSM_ERR_DEVICE_INPUT"}
 EXPORTS = ("ssd_chunk_scan", "ssd_chunk_scan_workspace_size", "ssm_state_update",
-           "ssd_chunk_scan_slots", "ssm_state_update_slots", "ssm_status_string", "ssm_version")
+           "ssd_chunk_scan_slots", "ssm_state_update_slots", "causal_conv1d_fwd",
+           "causal_conv1d_update", "ssm_status_string", "ssm_version")
+ACTIVATIONS = {None: 0, "none": 0, "silu": 1}
 
 
 def _load():
@@ -43,6 +45,11 @@ def _load():
     lib.ssm_state_update_slots.restype = i
     lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp, vp,
                                            i, vp, vp, vp]
+    lib.causal_conv1d_fwd.restype = i
+    lib.causal_conv1d_fwd.argtypes = [i, i, vp, i, i, i, vp, vp, vp, i, vp, i, vp, vp, i, vp,
+                                      vp, vp]
+    lib.causal_conv1d_update.restype = i
+    lib.causal_conv1d_update.argtypes = [i, i, i, i, vp, vp, vp, i, vp, i, vp, i, vp, vp, vp]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_status_string.argtypes = [i]
     lib.ssm_version.restype = i
@@ -250,4 +257,82 @@ def ssm_state_update_slots(state_pool, slot_idx, x, dt, A, B, C, D=None, y=None,
                                     _ptr(A), _ptr(B), _ptr(C), _ptr(D), _dtype_code(y.dtype),
                                     _ptr(y), _ptr(status), _stream(stream))
     _check(st, "ssm_state_update_slots")
+    return y
+
+
+def _activation(activation) -> int:
+    if activation not in ACTIVATIONS:
+        raise ValueError(f"activation must be one of {sorted(map(str, ACTIVATIONS))}")
+    return ACTIVATIONS[activation]
+
+
+def causal_conv1d_fwd(x, weight, bias=None, conv_state=None, cu_seqlens=None,
+                      activation="silu", slot_idx=None, has_initial_state=None, y=None,
+                      y_dtype=None, status=None, stream=None):
+    """Causal depthwise conv1d over whole sequences (prefill), channels-last.
+
+    x : [nseq, L, dim] or, with cu_seqlens (int32 [nseq+1]), packed [T, dim];
+        bf16 or fp32.
+    weight : [dim, width] fp32 (width <= 8); bias : [dim] fp32 or None.
+    conv_state : [rows, dim, width-1] in x's dtype, or None; read as the
+        history before each sequence and overwritten with its last width-1
+        inputs.  rows = nseq, or the pool size when slot_idx is given.
+    slot_idx, has_initial_state : int32 [nseq] or None.
+    Returns y shaped like x.
+    """
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens", torch.int32)
+        T, dim = x.shape
+        nseq, seqlen = cu_seqlens.shape[0] - 1, T
+    else:
+        nseq, seqlen, dim = x.shape
+    _dev(weight, "weight", torch.float32)
+    width = weight.shape[-1]
+    _dev(bias, "bias", torch.float32)
+    _dev(conv_state, "conv_state", x.dtype)
+    _dev(slot_idx, "slot_idx", torch.int32)
+    _dev(has_initial_state, "has_initial_state", torch.int32)
+    _dev(status, "status", torch.int32)
+    if y_dtype is None:
+        y_dtype = x.dtype if y is None else y.dtype
+    if y is None:
+        y = torch.empty(x.shape, dtype=y_dtype, device=x.device)
+    _dev(y, "y", y_dtype)
+    max_slots = conv_state.shape[0] if (conv_state is not None and slot_idx is not None) else 0
+    st = lib.causal_conv1d_fwd(nseq, seqlen, _ptr(cu_seqlens), dim, width, in_code, _ptr(x),
+                               _ptr(weight), _ptr(bias), _activation(activation),
+                               _ptr(conv_state), max_slots, _ptr(slot_idx),
+                               _ptr(has_initial_state), _dtype_code(y.dtype), _ptr(y),
+                               _ptr(status), _stream(stream))
+    _check(st, "causal_conv1d_fwd")
+    return y
+
+
+def causal_conv1d_update(x, weight, bias, conv_state, activation="silu", slot_idx=None,
+                         y=None, y_dtype=None, status=None, stream=None):
+    """One decode token per batch row; conv_state [rows, dim, width-1] rolls in
+    place (rows = batch, or the pool size when slot_idx is given; a negative
+    slot marks a padding row).  x : [batch, dim].  Returns y [batch, dim]."""
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    batch, dim = x.shape
+    _dev(weight, "weight", torch.float32)
+    width = weight.shape[-1]
+    _dev(bias, "bias", torch.float32)
+    _dev(conv_state, "conv_state", x.dtype)
+    _dev(slot_idx, "slot_idx", torch.int32)
+    _dev(status, "status", torch.int32)
+    if y_dtype is None:
+        y_dtype = x.dtype if y is None else y.dtype
+    if y is None:
+        y = torch.zeros((batch, dim), dtype=y_dtype, device=x.device)
+    _dev(y, "y", y_dtype)
+    max_slots = conv_state.shape[0] if (conv_state is not None and slot_idx is not None) else 0
+    st = lib.causal_conv1d_update(batch, dim, width, in_code, _ptr(x), _ptr(weight), _ptr(bias),
+                                  _activation(activation), _ptr(conv_state), max_slots,
+                                  _ptr(slot_idx), _dtype_code(y.dtype), _ptr(y), _ptr(status),
+                                  _stream(stream))
+    _check(st, "causal_conv1d_update")
     return y

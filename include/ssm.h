@@ -204,6 +204,69 @@ SSM_API int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_st
                                    const void *B, const void *C, const float *D,
                                    int y_dtype, void *y, int *status_dev, cudaStream_t stream);
 
+/*
+ * Causal depthwise conv1d, the short convolution in front of the scan that
+ * mixes each channel of the concatenated (x, B, C) projection over the last
+ * `width` tokens ("Depthwise SiLU 卷积" of the MAX nemotron_h article,
+ * section 5.4 item 2; causal_conv1d_fn for prefill and causal_conv1d_update
+ * for decode in the modeling_nemotron_h.py walk-through, sections
+ * "Prefill 阶段" and "Decode 阶段").  For channel c and token t of a sequence:
+ *
+ *     y[t][c] = act(bias[c] + sum_{k<width} weight[c][k] * in[t-(width-1)+k][c])
+ *
+ * where the inputs before the sequence start are its conv state (its
+ * width-1 most recent earlier inputs, oldest first) or zero.  Afterwards the
+ * conv state holds the width-1 most recent inputs of the sequence (for a
+ * sequence shorter than width-1, the newest old entries shift down).
+ *
+ * Layouts (channels-last, row-major, contiguous):
+ *   x, y        [T][dim]              (in_dtype / y_dtype)
+ *   weight      [dim][width]          fp32
+ *   bias        [dim]                 fp32 or NULL
+ *   conv_state  [rows][dim][width-1]  in_dtype (the inputs' own type)
+ * activation: 0 = identity, 1 = SiLU (v * sigmoid(v)).  width in [1, 8].
+ * Accumulation is fp32; y rounds to nearest even when bf16, the conv state
+ * holds inputs verbatim.  All device pointers must be 16-byte aligned; y must
+ * not overlap x, the state or any other input.
+ */
+enum { SSM_ACT_NONE = 0, SSM_ACT_SILU = 1 };
+
+/*
+ * causal_conv1d_fwd -- prefill over whole sequences.
+ *   nseq, seqlen, cu_seqlens   as for ssd_chunk_scan (cu_seqlens device int32
+ *                              [nseq+1] for packed sequences, or NULL)
+ *   conv_state   device [rows][dim][width-1] or NULL (zero history; no state
+ *                written).  rows = nseq when slot_idx is NULL, else max_slots.
+ *   slot_idx     device int32 [nseq] or NULL: conv-state row of each sequence;
+ *                an index outside [0, max_slots) skips that sequence (no y,
+ *                no state written) and sets SSM_ERR_DEVICE_INPUT.
+ *   has_initial_state  device int32 [nseq] or NULL: 0 = zero history for that
+ *                sequence (its state row is still written).
+ * Two launches (the convolution, then the state roll) on `stream`.
+ */
+SSM_API int causal_conv1d_fwd(int nseq, int seqlen, const int32_t *cu_seqlens, int dim,
+                              int width, int in_dtype, const void *x, const float *weight,
+                              const float *bias, int activation, void *conv_state,
+                              int max_slots, const int32_t *slot_idx,
+                              const int32_t *has_initial_state, int y_dtype, void *y,
+                              int *status_dev, cudaStream_t stream);
+
+/*
+ * causal_conv1d_update -- decode: one token per batch row; the window is
+ * [conv_state row, x] and the state row rolls by one in place.
+ *   x, y         device [batch][dim]
+ *   conv_state   device [rows][dim][width-1] (rows = batch without slot_idx,
+ *                else max_slots); may be NULL only when width == 1.
+ *   slot_idx     device int32 [batch] or NULL: a negative index marks a
+ *                padding row (y and state untouched); an index >= max_slots
+ *                skips the row and sets SSM_ERR_DEVICE_INPUT.  Indices of
+ *                non-padding rows must be distinct.
+ */
+SSM_API int causal_conv1d_update(int batch, int dim, int width, int in_dtype, const void *x,
+                                 const float *weight, const float *bias, int activation,
+                                 void *conv_state, int max_slots, const int32_t *slot_idx,
+                                 int y_dtype, void *y, int *status_dev, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -184,3 +184,67 @@ def update_slots(lib, batch=2, H=4, P=64, N=128, G=2, pool=0x200000, max_slots=8
 ])
 def test_update_slots_rejects(slib, kw, code):
     assert update_slots(slib, **kw) == code
+
+
+@pytest.fixture(scope="module")
+def clib(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.causal_conv1d_fwd.restype = i
+    lib.causal_conv1d_fwd.argtypes = [i, i, vp, i, i, i, vp, vp, vp, i, vp, i, vp, vp, i, vp,
+                                      vp, vp]
+    lib.causal_conv1d_update.restype = i
+    lib.causal_conv1d_update.argtypes = [i, i, i, i, vp, vp, vp, i, vp, i, vp, i, vp, vp, vp]
+    return lib
+
+
+def conv_fwd(lib, nseq=2, seqlen=64, cu=None, dim=256, width=4, ind=BF16, x=0x100000,
+             w=0x200000, bias=None, act=1, state=0x300000, max_slots=0, slots=None, has=None,
+             yd=BF16, y=0x400000):
+    return lib.causal_conv1d_fwd(nseq, seqlen, cu, dim, width, ind, x, w, bias, act, state,
+                                 max_slots, slots, has, yd, y, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dim=0), INVALID),
+    (dict(width=0), INVALID),
+    (dict(width=9), UNSUPPORTED),
+    (dict(act=2), INVALID),
+    (dict(ind=5), INVALID),
+    (dict(w=None), INVALID),
+    (dict(x=None), INVALID),
+    (dict(y=0x400002), MISALIGNED),
+    (dict(y=0x100000 + 64), INVALID),           # y overlaps x
+    (dict(state=0x100000 + 4096), INVALID),     # state inside x
+    (dict(slots=0x500000, state=None), INVALID),
+    (dict(slots=0x500000, max_slots=0), INVALID),
+    (dict(nseq=0, seqlen=5, cu=0x600000), INVALID),
+])
+def test_conv_fwd_rejects(clib, kw, code):
+    assert conv_fwd(clib, **kw) == code
+
+
+def test_conv_fwd_noops(clib):
+    assert conv_fwd(clib, nseq=0, x=None, y=None, state=None) == OK
+    assert conv_fwd(clib, seqlen=0, x=None, y=None, state=None) == OK
+
+
+def conv_update(lib, batch=4, dim=256, width=4, x=0x100000, w=0x200000, state=0x300000,
+                max_slots=0, slots=None, y=0x400000):
+    return lib.causal_conv1d_update(batch, dim, width, BF16, x, w, None, 1, state, max_slots,
+                                    slots, BF16, y, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=-1), INVALID),
+    (dict(width=9), UNSUPPORTED),
+    (dict(state=None), INVALID),
+    (dict(slots=0x500000), INVALID),            # slot map without a pool size
+    (dict(x=0x100008), MISALIGNED),
+    (dict(y=0x300000 + 256), INVALID),          # y inside the state
+])
+def test_conv_update_rejects(clib, kw, code):
+    assert conv_update(clib, **kw) == code
+
+
+def test_conv_update_batch_zero_is_noop(clib):
+    assert conv_update(clib, batch=0, x=None, y=None, state=None) == OK
