@@ -11,7 +11,9 @@ One step = one pass of the whole hot path over one batch of synthetic input:
     a ring of 8 seeded input sets.
 ``value`` is tokens/s over both (16384 prefill + 64 decode tokens per step and
 per GPU); the per-kernel numbers the metric names (prefill tokens/s and % of
-tensor peak, decode GB/s and % of HBM peak) are under ``parts``.
+tensor peak, decode GB/s and % of HBM peak) are under ``parts``, with the
+causal conv1d that feeds the scan timed beside the step (``conv1d_prefill``:
+4 x 4096 tokens x 10240 channels; ``conv1d_decode``: 64 rows x 18432 channels).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun each rank runs its own batch (weak scaling, no data-path
@@ -284,21 +286,48 @@ def time_conv(dev, stream, seed, iters=50):
                                  y=dy, stream=stream)
 
     out = {}
-    for name, fn, (nbytes, units) in (("conv1d_prefill", lambda k: pre(), conv_prefill_work()),
-                                      ("conv1d_decode", dec, conv_decode_work())):
-        for k in range(5):
-            fn(k)
-        torch.cuda.synchronize(dev)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(iters)]
-        for k in range(iters):
-            ev[k][0].record(stream)
-            fn(k)
-            ev[k][1].record(stream)
-        torch.cuda.synchronize(dev)
-        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
-        out[name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "bytes_per_launch": nbytes,
-                     "tokens_per_s": units / (ms * 1e-3), "launches": iters}
+    # prefill: per-launch events (two kernels per call: convolution, state roll)
+    for k in range(5):
+        pre()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    for k in range(iters):
+        ev[k][0].record(stream)
+        pre()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
+    nbytes, units = conv_prefill_work()
+    out["conv1d_prefill"] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                             "bytes_per_launch": nbytes, "tokens_per_s": units / (ms * 1e-3),
+                             "launches": iters}
+    # decode: a few microseconds per launch, so the launches are replayed from
+    # a CUDA graph (the host's launch rate would otherwise set the time)
+    for k in range(5):
+        dec(k)
+    torch.cuda.synchronize(dev)
+    gs = torch.cuda.Stream(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(gs):
+        with torch.cuda.graph(graph, stream=gs):
+            for k in range(cd["ring"]):
+                ssm.causal_conv1d_update(dx[k], dw, db, pool, slot_idx=slots[k], y=dy, stream=gs)
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(1, iters // 10)
+    g0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = g0.elapsed_time(g1) / (reps * cd["ring"])
+    nbytes, units = conv_decode_work()
+    out["conv1d_decode"] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                            "bytes_per_launch": nbytes, "tokens_per_s": units / (ms * 1e-3),
+                            "launches": reps * cd["ring"], "timing": "CUDA graph replay"}
+    del graph
     return out
 
 

@@ -17,6 +17,7 @@
 // All three are bound by HBM: each input and output is touched once.
 #include "common.cuh"
 #include "ssm_internal.h"
+#include "tc_ptx.cuh"
 
 namespace ssm {
 
@@ -157,7 +158,6 @@ template <> struct ConvVec<__nv_bfloat16> { static constexpr int V = 8; using Ra
 template <> struct ConvVec<float> { static constexpr int V = 4; using Raw = float4; };
 
 constexpr int kVecThreads = 128;
-constexpr int kVecUnroll = 8;
 
 __device__ __forceinline__ void unpack_row(const uint4 &r, float (&f)[8]) {
     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r);
@@ -190,111 +190,146 @@ __device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float (&v)[V])
     else *reinterpret_cast<uint2 *>(p) = make_uint2(w[0], w[1]);
 }
 
+// The same rows as channel pairs (fp32x2 lanes).
+__device__ __forceinline__ void unpack_row2(const uint4 &r, float2 (&f)[4]) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = __bfloat1622float2(h[i]);
+}
+__device__ __forceinline__ void unpack_row2(const float4 &r, float2 (&f)[2]) {
+    f[0] = make_float2(r.x, r.y);
+    f[1] = make_float2(r.z, r.w);
+}
+template <int P2>
+__device__ __forceinline__ void store_row2(float *p, const float2 (&v)[P2]) {
+#pragma unroll
+    for (int i = 0; i < P2 / 2; ++i)
+        reinterpret_cast<float4 *>(p)[i] = make_float4(v[2 * i].x, v[2 * i].y, v[2 * i + 1].x, v[2 * i + 1].y);
+}
+template <int P2>
+__device__ __forceinline__ void store_row2(__nv_bfloat16 *p, const float2 (&v)[P2]) {
+    uint32_t w[P2];
+#pragma unroll
+    for (int i = 0; i < P2; ++i) {
+        const __nv_bfloat162 h = __float22bfloat162_rn(v[i]);
+        w[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    if constexpr (P2 == 4) *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    else *reinterpret_cast<uint2 *>(p) = make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ float ex2_approx(float v) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+// SiLU of two lanes: v / (1 + 2^(-v log2 e)), the exponential and the
+// reciprocal on the special-function unit, the rest as fp32x2 arithmetic.
+__device__ __forceinline__ float2 silu2(float2 v) {
+    constexpr float kNegLog2e = -1.4426950408889634f;
+    const float2 e = __fmul2_rn(v, make_float2(kNegLog2e, kNegLog2e));
+    float2 d = make_float2(ex2_approx(e.x), ex2_approx(e.y));
+    d = __fadd2_rn(d, make_float2(1.f, 1.f));
+    return __fmul2_rn(v, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
 template <typename TIn>
 __device__ __forceinline__ typename ConvVec<TIn>::Raw load_row(const TIn *p) {
     return __ldg(reinterpret_cast<const typename ConvVec<TIn>::Raw *>(p));
 }
 
-template <typename TIn, typename TOut, int K>
+// Pipelined prefill for dim % V == 0.  A CTA owns one strip of
+// kPipeThreads*V channels (2 KB of a token row) and a contiguous range of
+// tokens; one thread streams the strip's rows into a ring of shared-memory
+// stages with bulk copies (kPipeRows rows per stage, completion on an
+// mbarrier) while all threads convolve the stage before.  The window carries
+// across rows in registers; at the range start and at every sequence start
+// inside the range it is reloaded from x, the conv state or zeros.
+constexpr int kPipeRows = 8;
+constexpr int kPipeStages = 3;
+constexpr int kPipeRowBytes = kVecThreads * 16;
+constexpr int kPipeSmem = kPipeStages * kPipeRows * kPipeRowBytes + kPipeStages * 8;
+
+template <typename TIn, typename TOut, int K, bool ACT>
 __global__ void __launch_bounds__(kVecThreads)
-conv1d_fwd_vec_kernel(ConvArgs a)
+conv1d_fwd_pipe_kernel(ConvArgs a, int ncta)
 {
     constexpr int V = ConvVec<TIn>::V;
-    constexpr int W = K > 1 ? K - 1 : 1;        // window slots (at least one)
+    constexpr int W = K > 1 ? K - 1 : 1;
     using Raw = typename ConvVec<TIn>::Raw;
-    const int c0 = (blockIdx.y * kVecThreads + threadIdx.x) * V;
-    const long tok0 = (long)blockIdx.x * kConvTile;
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_seq;
+    const uint32_t ring = tc::smem_u32(smem);
+    const uint32_t bar0 = ring + kPipeStages * kPipeRows * kPipeRowBytes;
+    const int tid = threadIdx.x, dim = a.dim;
+    const int c_base = blockIdx.y * kVecThreads * V;
+    const uint32_t strip_bytes = (uint32_t)min(kVecThreads * V, dim - c_base) * sizeof(TIn);
+    const int c0 = c_base + tid * V;
+    const bool active = c0 < dim;
     const long T = a.cu_seqlens ? (long)a.seqlen : (long)a.nseq * a.seqlen;
-    if (tok0 >= T) return;
-    const long tok1 = min(tok0 + kConvTile, T);
-    const int dim = a.dim;
+    const long t_begin = T * blockIdx.x / ncta, t_end = T * (blockIdx.x + 1) / ncta;
+    if (t_begin >= t_end) return;                       // uniform over the CTA
+    const int groups = (int)((t_end - t_begin + kPipeRows - 1) / kPipeRows);
     const TIn *x = static_cast<const TIn *>(a.x);
     TOut *y = static_cast<TOut *>(a.y);
 
-    __shared__ int s_seq;
-    if (threadIdx.x == 0) {
-        int s;
+    auto issue = [&](int g) {
+        const int slot = g % kPipeStages;
+        const long r0 = t_begin + (long)g * kPipeRows;
+        const int n = (int)min((long)kPipeRows, t_end - r0);
+        const uint32_t bar = bar0 + 8 * slot;
+        tc::mbar_arrive_expect_tx(bar, n * strip_bytes);
+        for (int r = 0; r < n; ++r)
+            tc::bulk_load_1d(ring + (slot * kPipeRows + r) * kPipeRowBytes,
+                             x + (size_t)(r0 + r) * dim + c_base, strip_bytes, bar);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < kPipeStages; ++i) tc::mbar_init(bar0 + 8 * i, 1);
+        tc::fence_mbar_init();
+        for (int g = 0; g < min(kPipeStages, groups); ++g) issue(g);
+        int s = 0;
         if (a.cu_seqlens) {
             int lo = 0, hi = a.nseq - 1;
-            while (lo < hi) {
+            while (lo < hi) {   // last sequence starting at or before t_begin
                 const int mid = (lo + hi + 1) >> 1;
-                if (a.cu_seqlens[mid] <= tok0) lo = mid; else hi = mid - 1;
+                if (a.cu_seqlens[mid] <= t_begin) lo = mid; else hi = mid - 1;
             }
             s = lo;
         } else {
-            s = (int)(tok0 / a.seqlen);
+            s = (int)(t_begin / a.seqlen);
         }
         s_seq = s;
     }
     __syncthreads();
-    if (c0 >= dim) return;
 
-    float w[V][K], bias[V];
+    // channels in pairs: the products and the SiLU run on packed fp32x2
+    constexpr int P2 = V / 2;
+    float2 w2[K][P2], b2[P2];
+    if (active) {
+        float wv[V * K];
 #pragma unroll
-    for (int i = 0; i < V * K / 4; ++i) {
-        const float4 q = __ldg(reinterpret_cast<const float4 *>(a.weight + (size_t)c0 * K) + i);
-        const float e[4] = {q.x, q.y, q.z, q.w};
+        for (int i = 0; i < V * K / 4; ++i) {
+            const float4 q = __ldg(reinterpret_cast<const float4 *>(a.weight + (size_t)c0 * K) + i);
+            wv[4 * i] = q.x; wv[4 * i + 1] = q.y; wv[4 * i + 2] = q.z; wv[4 * i + 3] = q.w;
+        }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) w[(4 * i + j) / K][(4 * i + j) % K] = e[j];
+        for (int k = 0; k < K; ++k)
+#pragma unroll
+            for (int p = 0; p < P2; ++p) w2[k][p] = make_float2(wv[(2 * p) * K + k], wv[(2 * p + 1) * K + k]);
+#pragma unroll
+        for (int p = 0; p < P2; ++p)
+            b2[p] = a.bias ? make_float2(__ldg(a.bias + c0 + 2 * p), __ldg(a.bias + c0 + 2 * p + 1))
+                           : make_float2(0.f, 0.f);
     }
-#pragma unroll
-    for (int v = 0; v < V; ++v) bias[v] = a.bias ? __ldg(a.bias + c0 + v) : 0.f;
 
     int s = s_seq;
     auto seq_start = [&](int q) -> long { return a.cu_seqlens ? (long)a.cu_seqlens[q] : (long)q * a.seqlen; };
     auto seq_end = [&](int q) -> long { return a.cu_seqlens ? (long)a.cu_seqlens[q + 1] : (long)(q + 1) * a.seqlen; };
     long ts = seq_start(s), te = seq_end(s);
-
-    float win[W][V];   // win[j] = inputs of token t-(K-1)+j
-    auto step = [&](long t, const float (&cur)[V], bool write) {
-        float out[V];
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-            float acc = bias[v];
-#pragma unroll
-            for (int j = 0; j < K - 1; ++j) acc = fmaf(w[v][j], win[j][v], acc);
-            acc = fmaf(w[v][K - 1], cur[v], acc);
-            out[v] = conv_act(acc, a.activation);
-        }
-        if (write) store_row<V>(y + (size_t)t * dim + c0, out);
-#pragma unroll
-        for (int j = 0; j < K - 2; ++j)
-#pragma unroll
-            for (int v = 0; v < V; ++v) win[j][v] = win[j + 1][v];
-        if (K > 1)
-#pragma unroll
-            for (int v = 0; v < V; ++v) win[W - 1][v] = cur[v];
-    };
-
-    if (tok0 - (K - 1) >= ts && tok0 - (K - 1) >= 0 && tok1 <= te) {
-        // fast path: the window and the tile lie inside one sequence
-#pragma unroll
-        for (int j = 0; j < K - 1; ++j) {
-            float f[V];
-            unpack_row(load_row(x + (size_t)(tok0 - (K - 1) + j) * dim + c0), f);
-#pragma unroll
-            for (int v = 0; v < V; ++v) win[j][v] = f[v];
-        }
-        for (long t = tok0; t < tok1; t += kVecUnroll) {
-            Raw r[kVecUnroll];
-#pragma unroll
-            for (int u = 0; u < kVecUnroll; ++u)
-                if (t + u < tok1) r[u] = load_row(x + (size_t)(t + u) * dim + c0);
-#pragma unroll
-            for (int u = 0; u < kVecUnroll; ++u) {
-                if (t + u < tok1) {
-                    float cur[V];
-                    unpack_row(r[u], cur);
-                    step(t + u, cur, true);
-                }
-            }
-        }
-        return;
-    }
-
-    // general path: sequence starts (state or zeros) inside the tile
     const TIn *st = static_cast<const TIn *>(a.state);
-    bool skip = false;
+    bool skip = false, dead = false;
+    float2 win[W][P2];   // win[j] = inputs of token t-(K-1)+j
     auto load_window = [&](long t) {
         bool load_init;
         const long row = conv_state_row(a, s, load_init);
@@ -303,34 +338,79 @@ conv1d_fwd_vec_kernel(ConvArgs a)
         for (int j = 0; j < K - 1; ++j) {
             const long src = t - (K - 1) + j;
             if (src >= ts && src >= 0) {
-                float f[V];
-                unpack_row(load_row(x + (size_t)src * dim + c0), f);
-#pragma unroll
-                for (int v = 0; v < V; ++v) win[j][v] = f[v];
+                unpack_row2(load_row(x + (size_t)src * dim + c0), win[j]);
             } else {
+                auto sv = [&](int c) {
+                    return (row >= 0 && load_init)
+                        ? ld_in(st + ((size_t)row * dim + c) * (K - 1) + (K - 1) + (src - ts)) : 0.f;
+                };
 #pragma unroll
-                for (int v = 0; v < V; ++v)
-                    win[j][v] = (row >= 0 && load_init)
-                        ? ld_in(st + ((size_t)row * dim + c0 + v) * (K - 1) + (K - 1) + (src - ts))
-                        : 0.f;
+                for (int p = 0; p < P2; ++p) win[j][p] = make_float2(sv(c0 + 2 * p), sv(c0 + 2 * p + 1));
             }
         }
     };
-    load_window(tok0);
-    for (long t = tok0; t < tok1; ++t) {
-        if (t >= te) {
-            do { ++s; } while (s + 1 < a.nseq && seq_end(s) <= t);
-            if (s >= a.nseq) {
-                report_status(a.status_dev, 6);
-                return;
-            }
-            ts = seq_start(s);
-            te = seq_end(s);
-            load_window(t);
+    if (active) load_window(t_begin);
+
+    // one token: y row from the window and the staged row, then roll the window
+    auto token = [&](long t, const uint8_t *rowp, bool write) {
+        float2 cur[P2], out[P2];
+        unpack_row2(*reinterpret_cast<const Raw *>(rowp), cur);
+#pragma unroll
+        for (int p = 0; p < P2; ++p) {
+            float2 acc = b2[p];
+#pragma unroll
+            for (int j = 0; j < K - 1; ++j) acc = __ffma2_rn(w2[j][p], win[j][p], acc);
+            acc = __ffma2_rn(w2[K - 1][p], cur[p], acc);
+            out[p] = ACT ? silu2(acc) : acc;
         }
-        float cur[V];
-        unpack_row(load_row(x + (size_t)t * dim + c0), cur);
-        step(t, cur, !skip);
+        if (write) store_row2<P2>(y + (size_t)t * dim + c0, out);
+#pragma unroll
+        for (int j = 0; j < K - 2; ++j)
+#pragma unroll
+            for (int p = 0; p < P2; ++p) win[j][p] = win[j + 1][p];
+        if (K > 1)
+#pragma unroll
+            for (int p = 0; p < P2; ++p) win[W - 1][p] = cur[p];
+    };
+
+    bool ok = true;
+    for (int g = 0; g < groups; ++g) {
+        const int slot = g % kPipeStages;
+        if (!tc::mbar_wait_bounded(bar0 + 8 * slot, (uint32_t)((g / kPipeStages) & 1), ok)) {
+            if (tid == 0) report_status(a.status_dev, 5);
+            return;   // a bulk copy that never lands: nothing in flight can be waited for
+        }
+        const long r0 = t_begin + (long)g * kPipeRows;
+        const int n = (int)min((long)kPipeRows, t_end - r0);
+        const uint8_t *base = smem + slot * kPipeRows * kPipeRowBytes + tid * 16;
+        if (active && !dead) {
+            if (n == kPipeRows && r0 + kPipeRows <= te) {
+                // whole stage inside the current sequence
+#pragma unroll
+                for (int r = 0; r < kPipeRows; ++r) token(r0 + r, base + r * kPipeRowBytes, !skip);
+            } else {
+                for (int r = 0; r < n; ++r) {
+                    const long t = r0 + r;
+                    if (t >= te) {   // next sequence (skipping empty ones)
+                        do { ++s; } while (s + 1 < a.nseq && seq_end(s) <= t);
+                        if (s >= a.nseq) {   // offsets end before T
+                            report_status(a.status_dev, 6);
+                            dead = true;
+                            break;
+                        }
+                        ts = seq_start(s);
+                        te = seq_end(s);
+                        load_window(t);
+                    }
+                    token(t, base + r * kPipeRowBytes, !skip);
+                }
+            }
+        }
+        __syncthreads();                 // every thread is done with this slot
+        if (tid == 0 && g + kPipeStages < groups) {
+            tc::fence_proxy_async_smem();
+            issue(g + kPipeStages);
+        }
     }
 }
 
@@ -480,6 +560,47 @@ conv1d_update_vec_kernel(ConvArgs a)
     }
 }
 
+static int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+// Resident pipelined CTAs per SM: shared memory allows 4 of kPipeSmem.
+static int pipe_ctas_per_sm() { return 4; }
+
+template <typename TIn, typename TOut, int K, bool ACT>
+static cudaError_t launch_pipe_k(const ConvArgs &a, dim3 grid, int ncta, cudaStream_t stream) {
+    auto kern = conv1d_fwd_pipe_kernel<TIn, TOut, K, ACT>;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPipeSmem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    kern<<<grid, kVecThreads, kPipeSmem, stream>>>(a, ncta);
+    return cudaGetLastError();
+}
+
+template <typename TIn, typename TOut, bool ACT>
+static cudaError_t launch_pipe(const ConvArgs &a, dim3 grid, int ncta, cudaStream_t stream) {
+    switch (a.width) {
+    case 1: return launch_pipe_k<TIn, TOut, 1, ACT>(a, grid, ncta, stream);
+    case 2: return launch_pipe_k<TIn, TOut, 2, ACT>(a, grid, ncta, stream);
+    case 3: return launch_pipe_k<TIn, TOut, 3, ACT>(a, grid, ncta, stream);
+    case 4: return launch_pipe_k<TIn, TOut, 4, ACT>(a, grid, ncta, stream);
+    case 5: return launch_pipe_k<TIn, TOut, 5, ACT>(a, grid, ncta, stream);
+    case 6: return launch_pipe_k<TIn, TOut, 6, ACT>(a, grid, ncta, stream);
+    case 7: return launch_pipe_k<TIn, TOut, 7, ACT>(a, grid, ncta, stream);
+    default: return launch_pipe_k<TIn, TOut, 8, ACT>(a, grid, ncta, stream);
+    }
+}
+
 template <typename TIn, typename TOut>
 static cudaError_t launch_conv_t(const ConvArgs &a, cudaStream_t stream)
 {
@@ -505,20 +626,14 @@ static cudaError_t launch_conv_t(const ConvArgs &a, cudaStream_t stream)
     }
     const long T = a.cu_seqlens ? (long)a.seqlen : (long)a.nseq * a.seqlen;
     if (T > 0 && a.dim % V == 0) {
-        const unsigned tiles = (unsigned)((T + kConvTile - 1) / kConvTile);
-        const unsigned vblocks = (unsigned)((a.dim / V + kVecThreads - 1) / kVecThreads);
-        const dim3 grid(tiles, vblocks);
-        switch (a.width) {
-        case 1: conv1d_fwd_vec_kernel<TIn, TOut, 1><<<grid, kVecThreads, 0, stream>>>(a); break;
-        case 2: conv1d_fwd_vec_kernel<TIn, TOut, 2><<<grid, kVecThreads, 0, stream>>>(a); break;
-        case 3: conv1d_fwd_vec_kernel<TIn, TOut, 3><<<grid, kVecThreads, 0, stream>>>(a); break;
-        case 4: conv1d_fwd_vec_kernel<TIn, TOut, 4><<<grid, kVecThreads, 0, stream>>>(a); break;
-        case 5: conv1d_fwd_vec_kernel<TIn, TOut, 5><<<grid, kVecThreads, 0, stream>>>(a); break;
-        case 6: conv1d_fwd_vec_kernel<TIn, TOut, 6><<<grid, kVecThreads, 0, stream>>>(a); break;
-        case 7: conv1d_fwd_vec_kernel<TIn, TOut, 7><<<grid, kVecThreads, 0, stream>>>(a); break;
-        default: conv1d_fwd_vec_kernel<TIn, TOut, 8><<<grid, kVecThreads, 0, stream>>>(a); break;
-        }
-        cudaError_t e = cudaGetLastError();
+        const int strips = (a.dim / V + kVecThreads - 1) / kVecThreads;
+        // enough CTAs to fill the GPU once, each with at least 4 stages of rows
+        const long fill = (long)pipe_ctas_per_sm() * sm_count() / strips;
+        const long by_rows = (T + 4 * kPipeRows - 1) / (4 * kPipeRows);
+        const int ncta = (int)(fill < by_rows ? (fill > 0 ? fill : 1) : by_rows);
+        const dim3 grid((unsigned)ncta, (unsigned)strips);
+        cudaError_t e = a.activation ? launch_pipe<TIn, TOut, true>(a, grid, ncta, stream)
+                                     : launch_pipe<TIn, TOut, false>(a, grid, ncta, stream);
         if (e != cudaSuccess) return e;
     } else if (T > 0) {
         const unsigned tiles = (unsigned)((T + kConvTile - 1) / kConvTile);

@@ -93,6 +93,7 @@ def main():
     ap.add_argument("--width", type=int, default=4)
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--launches", type=int, default=1)
+    ap.add_argument("--graph", action="store_true")
     args = ap.parse_args()
     if args.heads is None:
         args.heads = 128 if args.case in ("prefill", "conv") else 256
@@ -102,10 +103,25 @@ def main():
         run()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(args.launches):
-        run()
-    e.record()
+    if args.graph:
+        # launch-bound kernels: replay the launches from a CUDA graph so the
+        # device time is not bounded by the host's launch rate
+        stream = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(graph, stream=stream):
+                for _ in range(args.launches):
+                    run()
+        graph.replay()
+        torch.cuda.synchronize()
+        s.record()
+        graph.replay()
+        e.record()
+    else:
+        s.record()
+        for _ in range(args.launches):
+            run()
+        e.record()
     torch.cuda.synchronize()
     print(json.dumps({"case": args.case, "ms_per_launch": s.elapsed_time(e) / args.launches,
                       "args": vars(args)}))
