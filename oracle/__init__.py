@@ -16,10 +16,13 @@ restated for decode in the modeling_nemotron_h.py walk-through (section
 ``h <- exp(dt*A_h) * h + dt * x (outer) B`` and ``y = h . C + D_h * x``, the
 output reading the updated state.
 
-Every function here is pinned by tests/test_oracle.py against results that do
-not come from this code: a brute-force evaluation of the structured
+Every function here is pinned against results that do not come from this
+code: tests/test_oracle.py (a brute-force evaluation of the structured
 semiseparable (SSD) matrix form, closed forms for dt = 0, A = 0, d_state = 1
-and time-invariant inputs, split-and-carry, and linearity.
+and time-invariant inputs, split-and-carry, and linearity),
+tests/test_oracle_conv.py (numpy's correlate, the logistic function) and
+tests/test_oracle_mtp.py (the matrix form over each draft prefix, correlate
+over [conv state, draft inputs]).
 """
 from __future__ import annotations
 
@@ -242,3 +245,64 @@ def causal_conv1d_update(x, weight, bias, state, activation="silu"):
     batch = xf.shape[0]
     cu = np.arange(batch + 1, dtype=np.int64)
     return causal_conv1d(xf, weight, bias, activation, state, cu_seqlens=cu)
+
+
+def state_update_multi(state, x, dt, A, B, C, D=None, accept_len=None):
+    """Speculative (multi-token) decode: each batch row runs its ntok draft
+    tokens in order from its state (the MTP / speculative-decoding item of
+    the deep-research note, "MTP / speculative decoding": candidate tokens
+    produce intermediate states, and the accepted count decides which one
+    becomes the row's state).
+
+    state : [batch, H, P, N]; x : [batch, ntok, H, P]; dt : [batch, ntok, H];
+    B, C : [batch, ntok, G, N]; accept_len : [batch] ints in [0, ntok] or None.
+    Returns (y [batch, ntok, H, P], inter [batch, ntok, H, P, N] -- the state
+    after each draft token --, new_state [batch, H, P, N]: the state after
+    accept_len[b] tokens, i.e. the input state where accept_len[b] == 0 or
+    where accept_len is None).  fp64; a loop of state_update calls.
+    """
+    st = _f64(state).copy()
+    xf, dtf, Bf, Cf = _f64(x), _f64(dt), _f64(B), _f64(C)
+    batch, ntok = xf.shape[0], xf.shape[1]
+    ys, inter = [], []
+    cur = st.copy()
+    for k in range(ntok):
+        yk, cur = state_update(cur, xf[:, k], dtf[:, k], A, Bf[:, k], Cf[:, k], D)
+        ys.append(yk)
+        inter.append(cur.copy())
+    y = np.stack(ys, axis=1) if ntok else np.zeros(xf.shape)
+    inter = (np.stack(inter, axis=1) if ntok
+             else np.zeros((batch, 0) + st.shape[1:]))
+    new = st.copy()
+    if accept_len is not None:
+        acc = np.asarray(accept_len, dtype=np.int64)
+        for b in range(batch):
+            if acc[b] > 0:
+                new[b] = inter[b, acc[b] - 1]
+    return y, inter, new
+
+
+def causal_conv1d_update_multi(x, weight, bias, state, activation="silu", accept_len=None):
+    """ntok draft tokens per batch row through the causal conv1d, in order
+    from the row's conv state.  x : [batch, ntok, dim]; state : [batch, dim,
+    K-1].  Returns (y [batch, ntok, dim], new_state): the conv state after
+    accept_len[b] tokens (unchanged where 0, or everywhere when accept_len is
+    None).  fp64; a loop of causal_conv1d_update calls.
+    """
+    xf = _f64(x)
+    batch, ntok = xf.shape[0], xf.shape[1]
+    st = _f64(state).copy()
+    cur = st.copy()
+    ys, states = [], []
+    for k in range(ntok):
+        yk, cur = causal_conv1d_update(xf[:, k], weight, bias, cur, activation)
+        ys.append(yk)
+        states.append(cur.copy())
+    y = np.stack(ys, axis=1) if ntok else np.zeros(xf.shape)
+    new = st.copy()
+    if accept_len is not None:
+        acc = np.asarray(accept_len, dtype=np.int64)
+        for b in range(batch):
+            if acc[b] > 0:
+                new[b] = states[acc[b] - 1][b]
+    return y, new
