@@ -331,6 +331,80 @@ def time_conv(dev, stream, seed, iters=50):
     return out
 
 
+MTP = dict(batch=64, ntok=4, H=256, P=64, N=128, G=8)
+
+
+def mtp_work(kind, m=MTP):
+    """Algorithmic bytes of one speculative-decode call at the Ultra decode
+    shape: the state (fp32) read once, plus per draft token x, B, C (bf16), dt
+    (fp32) and y (bf16); the intermediate states written (``verify_inter``);
+    the state read and written once (``replay``); or the accepted
+    intermediate state read and the state written (``scatter``)."""
+    b, n, H, P, N, G = m["batch"], m["ntok"], m["H"], m["P"], m["N"], m["G"]
+    state = b * H * P * N * 4
+    per_tok = b * (H * P * 2 + 2 * G * N * 2 + H * 4)
+    y = b * n * H * P * 2
+    if kind == "verify":
+        return state + n * per_tok + y
+    if kind == "verify_inter":
+        return state + n * per_tok + y + n * state
+    if kind == "replay":
+        return 2 * state + n * per_tok
+    return 2 * state + b * 4                                    # scatter
+
+
+def time_mtp(dev, stream, seed, iters=20):
+    """Device time of the speculative-decode entry points (beside the step)."""
+    import torch
+    from hybrid_mamba_ssm_b200 import inputs as synth
+    from hybrid_mamba_ssm_b200 import ssm
+
+    m = MTP
+    b, n, H, P, N, G = m["batch"], m["ntok"], m["H"], m["P"], m["N"], m["G"]
+    A, D = synth.make_head_params(seed, H)
+    A, D = torch.from_numpy(A).to(dev), torch.from_numpy(D).to(dev)
+    state = torch.from_numpy(synth.make_state(seed + 1, (b, H, P, N))).to(dev)
+    steps = [synth.make_decode_step(seed + 2 + k, b, H, P, N, G) for k in range(n)]
+
+    def stack16(f):
+        return torch.stack([torch.from_numpy(np.ascontiguousarray(f(s).bits).view(np.int16))
+                            for s in steps], dim=1).view(torch.bfloat16).contiguous().to(dev)
+
+    x, B, C = stack16(lambda s: s.x), stack16(lambda s: s.B), stack16(lambda s: s.C)
+    dt = torch.from_numpy(np.stack([s.dt for s in steps], axis=1)).contiguous().to(dev)
+    y = torch.empty((b, n, H, P), dtype=torch.bfloat16, device=dev)
+    inter = torch.empty((b, n, H, P, N), dtype=torch.float32, device=dev)
+    # every row accepts at least one token, so every row's state is written
+    acc = torch.from_numpy(np.random.default_rng(seed).integers(1, n + 1, b).astype(np.int32)).to(dev)
+    calls = {
+        "verify": lambda: ssm.ssm_state_update_multi(state, x, dt, A, B, C, D, y=y, stream=stream),
+        "verify_inter": lambda: ssm.ssm_state_update_multi(state, x, dt, A, B, C, D, y=y,
+                                                           inter_states=inter, stream=stream),
+        "replay": lambda: ssm.ssm_state_update_multi(state, x, dt, A, B, C, D, accept_len=acc,
+                                                     want_y=False, stream=stream),
+        "scatter": lambda: ssm.ssm_state_commit(inter, acc, state, stream=stream),
+    }
+    out = {}
+    for name, fn in calls.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(iters)]
+        for e0, e1 in ev:
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
+        nbytes = mtp_work(name)
+        out["mtp_" + name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                              "bytes_per_launch": nbytes, "launches": iters,
+                              "draft": f"batch {b} x {n} tokens"}
+    del inter
+    return out
+
+
 def run_reference(args, world, rank, pg):
     if rank != 0:
         return 0
@@ -515,6 +589,7 @@ def run_ours(args, world, rank, local, pg):
     e2e_ms = max_over_ranks(pg, s2.elapsed_time(e2), dev)
 
     conv = time_conv(dev, stream, seed + 17)
+    conv.update(time_mtp(dev, stream, seed + 29))
 
     # ---- numbers ----
     peaks, peak_kind = load_peaks()

@@ -336,13 +336,135 @@ int causal_conv1d_update(int batch, int dim, int width, int in_dtype, const void
     if (overlap(ry, rs)) return SSM_ERR_INVALID_ARG;
 
     ssm::ConvArgs a{};
-    a.update = 1; a.nseq = batch; a.seqlen = 1;
+    a.update = 1; a.nseq = batch; a.seqlen = 1; a.ntok = 1; a.commit_all = 1;
     a.dim = dim; a.width = width; a.activation = activation;
     a.in_dtype = in_dtype; a.y_dtype = y_dtype;
     a.x = x; a.weight = weight; a.bias = bias; a.state = conv_state;
     a.slot_idx = slot_idx; a.max_slots = max_slots;
     a.y = y; a.status_dev = status_dev;
     return ssm::launch_conv1d(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int causal_conv1d_update_multi(int batch, int ntok, int dim, int width, int in_dtype,
+                               const void *x, const float *weight, const float *bias,
+                               int activation, void *conv_state, int max_slots,
+                               const int32_t *slot_idx, const int32_t *accept_len, int y_dtype,
+                               void *y, int *status_dev, cudaStream_t stream)
+{
+    if (batch < 0 || ntok < 0 || dim <= 0) return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
+    if (activation != 0 && activation != 1) return SSM_ERR_INVALID_ARG;
+    if (width < 1) return SSM_ERR_INVALID_ARG;
+    if (width > 8) return SSM_ERR_UNSUPPORTED;
+    if (batch == 0 || ntok == 0) return SSM_OK;
+    if (!x || !weight || (width > 1 && !conv_state)) return SSM_ERR_INVALID_ARG;
+    if (!y && !accept_len) return SSM_ERR_INVALID_ARG;        // nothing would be produced
+    if (slot_idx && max_slots <= 0) return SSM_ERR_INVALID_ARG;
+    if ((long long)batch * ntok > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    const void *ptrs[] = {x, weight, bias, conv_state, slot_idx, accept_len, y, status_dev};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+    const size_t es = dtype_size(in_dtype);
+    const long long rows = slot_idx ? max_slots : batch;
+    const Range rs = range_of(conv_state, conv_state ? (size_t)rows * dim * (width - 1) * es : 0);
+    const Range ry = range_of(y, y ? (size_t)batch * ntok * dim * dtype_size(y_dtype) : 0);
+    const Range ins[] = {range_of(x, (size_t)batch * ntok * dim * es),
+                         range_of(weight, (size_t)dim * width * sizeof(float)),
+                         range_of(bias, bias ? (size_t)dim * sizeof(float) : 0),
+                         range_of(slot_idx, slot_idx ? (size_t)batch * sizeof(int32_t) : 0),
+                         range_of(accept_len, accept_len ? (size_t)batch * sizeof(int32_t) : 0)};
+    for (const Range &r : ins)
+        if (overlap(ry, r) || overlap(rs, r)) return SSM_ERR_INVALID_ARG;
+    if (overlap(ry, rs)) return SSM_ERR_INVALID_ARG;
+
+    ssm::ConvArgs a{};
+    a.update = 1; a.nseq = batch; a.seqlen = 1; a.ntok = ntok; a.commit_all = 0;
+    a.accept_len = accept_len;
+    a.dim = dim; a.width = width; a.activation = activation;
+    a.in_dtype = in_dtype; a.y_dtype = y_dtype;
+    a.x = x; a.weight = weight; a.bias = bias; a.state = conv_state;
+    a.slot_idx = slot_idx; a.max_slots = max_slots;
+    a.y = y; a.status_dev = status_dev;
+    return ssm::launch_conv1d(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_state_update_multi(int batch, int ntok, int nheads, int head_dim, int d_state,
+                           int ngroups, int in_dtype, float *state, int max_slots,
+                           const int32_t *slot_idx, const void *x, const float *dt,
+                           const float *A, const void *B, const void *C, const float *D,
+                           const int32_t *accept_len, float *inter_states, int y_dtype, void *y,
+                           int *status_dev, cudaStream_t stream)
+{
+    if (batch < 0 || ntok < 0 || nheads <= 0 || ngroups <= 0 || nheads % ngroups ||
+        head_dim <= 0)
+        return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
+    if (head_dim > 256 || !pow2_in(d_state, 16, 256)) return SSM_ERR_UNSUPPORTED;
+    if ((long long)batch * nheads > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    if (batch == 0 || ntok == 0) return SSM_OK;
+    if (!state || !x || !dt || !A || !B || !C) return SSM_ERR_INVALID_ARG;
+    if (!y && !inter_states && !accept_len) return SSM_ERR_INVALID_ARG;
+    if (slot_idx && max_slots <= 0) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {state, slot_idx, x, dt, A, B, C, D, accept_len, inter_states, y,
+                          status_dev};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+    const size_t es = dtype_size(in_dtype);
+    const size_t bt = (size_t)batch * ntok;
+    const size_t rows = slot_idx ? (size_t)max_slots : (size_t)batch;
+    const size_t slice = (size_t)nheads * head_dim * d_state * sizeof(float);
+    const Range rs = range_of(state, rows * slice);
+    const Range ri = range_of(inter_states, inter_states ? bt * slice : 0);
+    const Range ry = range_of(y, y ? bt * nheads * head_dim * dtype_size(y_dtype) : 0);
+    const Range ins[] = {range_of(x, bt * nheads * head_dim * es),
+                         range_of(dt, bt * nheads * sizeof(float)),
+                         range_of(A, (size_t)nheads * sizeof(float)),
+                         range_of(B, bt * ngroups * d_state * es),
+                         range_of(C, bt * ngroups * d_state * es),
+                         range_of(D, D ? (size_t)nheads * sizeof(float) : 0),
+                         range_of(slot_idx, slot_idx ? (size_t)batch * sizeof(int32_t) : 0),
+                         range_of(accept_len, accept_len ? (size_t)batch * sizeof(int32_t) : 0)};
+    for (const Range &r : ins)
+        if (overlap(ry, r) || overlap(rs, r) || overlap(ri, r)) return SSM_ERR_INVALID_ARG;
+    if (overlap(ry, rs) || overlap(ri, rs) || overlap(ri, ry)) return SSM_ERR_INVALID_ARG;
+
+    ssm::MultiUpdateArgs a;
+    a.batch = batch; a.ntok = ntok; a.nheads = nheads; a.head_dim = head_dim;
+    a.d_state = d_state; a.ngroups = ngroups; a.in_dtype = in_dtype; a.y_dtype = y_dtype;
+    a.state = state; a.slot_idx = slot_idx; a.max_slots = max_slots;
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
+    a.accept_len = accept_len; a.inter = inter_states; a.y = y; a.status_dev = status_dev;
+    return ssm::launch_state_update_multi(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_state_commit(int batch, int ntok, int nheads, int head_dim, int d_state,
+                     const float *inter_states, const int32_t *accept_len, float *state,
+                     int max_slots, const int32_t *slot_idx, int *status_dev,
+                     cudaStream_t stream)
+{
+    if (batch < 0 || ntok < 0 || nheads <= 0 || head_dim <= 0) return SSM_ERR_INVALID_ARG;
+    if (head_dim > 256 || !pow2_in(d_state, 16, 256)) return SSM_ERR_UNSUPPORTED;
+    if ((long long)batch * nheads > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    if (batch == 0 || ntok == 0) return SSM_OK;
+    if (!inter_states || !accept_len || !state) return SSM_ERR_INVALID_ARG;
+    if (slot_idx && max_slots <= 0) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {inter_states, accept_len, state, slot_idx, status_dev};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
+    const size_t slice = (size_t)nheads * head_dim * d_state * sizeof(float);
+    const size_t rows = slot_idx ? (size_t)max_slots : (size_t)batch;
+    const Range rs = range_of(state, rows * slice);
+    const Range ins[] = {range_of(inter_states, (size_t)batch * ntok * slice),
+                         range_of(accept_len, (size_t)batch * sizeof(int32_t)),
+                         range_of(slot_idx, slot_idx ? (size_t)batch * sizeof(int32_t) : 0)};
+    for (const Range &r : ins)
+        if (overlap(rs, r)) return SSM_ERR_INVALID_ARG;
+
+    ssm::CommitArgs a;
+    a.batch = batch; a.ntok = ntok; a.nheads = nheads; a.head_dim = head_dim;
+    a.d_state = d_state; a.inter = inter_states; a.accept_len = accept_len; a.state = state;
+    a.slot_idx = slot_idx; a.max_slots = max_slots; a.status_dev = status_dev;
+    return ssm::launch_state_commit(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 }  // extern "C"

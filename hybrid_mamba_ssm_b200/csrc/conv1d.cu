@@ -250,9 +250,14 @@ constexpr int kPipeRows = 8;
 constexpr int kPipeStages = 3;
 constexpr int kPipeRowBytes = kVecThreads * 16;
 constexpr int kPipeSmem = kPipeStages * kPipeRows * kPipeRowBytes + kPipeStages * 8;
+// Resident pipelined CTAs per SM: shared memory allows 4; the register cap
+// that keeps 4 (128) only fits the narrow windows of 8-channel threads.
+__host__ __device__ constexpr int pipe_ctas(int V, int K) {
+    return V * K <= 32 ? 4 : (V * K <= 48 ? 3 : 2);
+}
 
 template <typename TIn, typename TOut, int K, bool ACT>
-__global__ void __launch_bounds__(kVecThreads)
+__global__ void __launch_bounds__(kVecThreads, pipe_ctas(ConvVec<TIn>::V, K))
 conv1d_fwd_pipe_kernel(ConvArgs a, int ncta)
 {
     constexpr int V = ConvVec<TIn>::V;
@@ -454,7 +459,23 @@ conv1d_state_kernel(ConvArgs a)
         if (k < K - 1) st_in(st + k, nw[k]);
 }
 
-// Decode: one token per batch row; the window rolls in place.
+// Tokens after which decode row b writes its state back: all ntok for the
+// plain update, accept_len[b] for a speculative commit, none otherwise; -1
+// for a bad row (reported).
+__device__ __forceinline__ int conv_commit_count(const ConvArgs &a, int b) {
+    if (a.accept_len) {
+        const int n = a.accept_len[b];
+        if (n < 0 || n > a.ntok) {
+            report_status(a.status_dev, 6);
+            return -1;
+        }
+        return n;
+    }
+    return a.commit_all ? a.ntok : 0;
+}
+
+// Decode: ntok tokens per batch row (x, y [batch][ntok][dim]) from the row's
+// window; the state row is rewritten after the committed tokens.
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_update_kernel(ConvArgs a)
@@ -473,21 +494,32 @@ conv1d_update_kernel(ConvArgs a)
         }
         row = slot;
     }
+    const int commit = conv_commit_count(a, b);
+    if (commit < 0) return;
     TIn *st = static_cast<TIn *>(a.state) + ((size_t)row * dim + c) * (K - 1);
-    const float cur = ld_in(static_cast<const TIn *>(a.x) + (size_t)b * dim + c);
-    float acc = a.bias ? a.bias[c] : 0.f;
     float win[kMaxWidth - 1];
 #pragma unroll
-    for (int j = 0; j < kMaxWidth - 1; ++j) {
-        win[j] = (j < K - 1) ? ld_in(st + j) : 0.f;
-        if (j < K - 1) acc = fmaf(a.weight[(size_t)c * K + j], win[j], acc);
-    }
-    acc = fmaf(a.weight[(size_t)c * K + K - 1], cur, acc);
-    store_out(static_cast<TOut *>(a.y) + (size_t)b * dim + c, conv_act(acc, a.activation));
+    for (int j = 0; j < kMaxWidth - 1; ++j) win[j] = (j < K - 1) ? ld_in(st + j) : 0.f;
+    const float bias = a.bias ? a.bias[c] : 0.f;
+    for (int t = 0; t < a.ntok; ++t) {
+        const size_t xi = ((size_t)b * a.ntok + t) * dim + c;
+        const float cur = ld_in(static_cast<const TIn *>(a.x) + xi);
+        float acc = bias;
 #pragma unroll
-    for (int j = 0; j < kMaxWidth - 1; ++j) {
-        if (j < K - 2) st_in(st + j, win[j + 1]);
-        else if (j == K - 2) st_in(st + j, cur);
+        for (int j = 0; j < kMaxWidth - 1; ++j)
+            if (j < K - 1) acc = fmaf(a.weight[(size_t)c * K + j], win[j], acc);
+        acc = fmaf(a.weight[(size_t)c * K + K - 1], cur, acc);
+        if (a.y) store_out(static_cast<TOut *>(a.y) + xi, conv_act(acc, a.activation));
+#pragma unroll
+        for (int j = 0; j < kMaxWidth - 1; ++j) {
+            if (j < K - 2) win[j] = win[j + 1];
+            else if (j == K - 2) win[j] = cur;
+        }
+        if (t + 1 == commit) {
+#pragma unroll
+            for (int j = 0; j < kMaxWidth - 1; ++j)
+                if (j < K - 1) st_in(st + j, win[j]);
+        }
     }
 }
 
@@ -514,48 +546,54 @@ conv1d_update_vec_kernel(ConvArgs a)
         }
         row = slot;
     }
-    float cur[V];
-    unpack_row(load_row(static_cast<const TIn *>(a.x) + (size_t)b * dim + c0), cur);
+    const int commit = conv_commit_count(a, b);
+    if (commit < 0) return;
     // state of channels c0..c0+V-1: V*(K-1) values, channel-major
     TIn *st = static_cast<TIn *>(a.state) + ((size_t)row * dim + c0) * (K - 1);
-    float sv[W * V];
+    float win[W][V];   // win[j][v]: channel c0+v, window slot j (oldest first)
 #pragma unroll
     for (int i = 0; i < K - 1; ++i) {
         float f[V];
         unpack_row(*reinterpret_cast<const Raw *>(st + (size_t)i * V), f);
 #pragma unroll
-        for (int j = 0; j < V; ++j) sv[i * V + j] = f[j];
+        for (int e = 0; e < V; ++e) win[(i * V + e) % W][(i * V + e) / W] = f[e];
     }
-    float w[V * K], out[V];
+    float w[V * K], bias[V];
 #pragma unroll
     for (int i = 0; i < V * K / 4; ++i) {
         const float4 q = __ldg(reinterpret_cast<const float4 *>(a.weight + (size_t)c0 * K) + i);
         w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
     }
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-        float acc = a.bias ? __ldg(a.bias + c0 + v) : 0.f;
-#pragma unroll
-        for (int j = 0; j < K - 1; ++j) acc = fmaf(w[v * K + j], sv[v * (K - 1) + j], acc);
-        acc = fmaf(w[v * K + K - 1], cur[v], acc);
-        out[v] = conv_act(acc, a.activation);
-    }
-    store_row<V>(static_cast<TOut *>(a.y) + (size_t)b * dim + c0, out);
-    if (K > 1) {
-        // roll: channel v keeps its last K-2 entries and appends cur[v]
-        float nv[W * V];
+    for (int v = 0; v < V; ++v) bias[v] = a.bias ? __ldg(a.bias + c0 + v) : 0.f;
+    for (int t = 0; t < a.ntok; ++t) {
+        const size_t xi = ((size_t)b * a.ntok + t) * dim + c0;
+        float cur[V], out[V];
+        unpack_row(load_row(static_cast<const TIn *>(a.x) + xi), cur);
 #pragma unroll
         for (int v = 0; v < V; ++v) {
+            float acc = bias[v];
 #pragma unroll
-            for (int j = 0; j < K - 2; ++j) nv[v * (K - 1) + j] = sv[v * (K - 1) + j + 1];
-            nv[v * (K - 1) + K - 2] = cur[v];
+            for (int j = 0; j < K - 1; ++j) acc = fmaf(w[v * K + j], win[j][v], acc);
+            acc = fmaf(w[v * K + K - 1], cur[v], acc);
+            out[v] = conv_act(acc, a.activation);
         }
+        if (a.y) store_row<V>(static_cast<TOut *>(a.y) + xi, out);
 #pragma unroll
-        for (int i = 0; i < K - 1; ++i) {
-            float f[V];
+        for (int j = 0; j < K - 2; ++j)
 #pragma unroll
-            for (int j = 0; j < V; ++j) f[j] = nv[i * V + j];
-            store_row<V>(st + (size_t)i * V, f);
+            for (int v = 0; v < V; ++v) win[j][v] = win[j + 1][v];
+        if (K > 1)
+#pragma unroll
+            for (int v = 0; v < V; ++v) win[W - 1][v] = cur[v];
+        if (t + 1 == commit) {
+#pragma unroll
+            for (int i = 0; i < K - 1; ++i) {
+                float f[V];
+#pragma unroll
+                for (int e = 0; e < V; ++e) f[e] = win[(i * V + e) % W][(i * V + e) / W];
+                store_row<V>(st + (size_t)i * V, f);
+            }
         }
     }
 }
@@ -570,9 +608,6 @@ static int sm_count() {
     }
     return n;
 }
-
-// Resident pipelined CTAs per SM: shared memory allows 4 of kPipeSmem.
-static int pipe_ctas_per_sm() { return 4; }
 
 template <typename TIn, typename TOut, int K, bool ACT>
 static cudaError_t launch_pipe_k(const ConvArgs &a, dim3 grid, int ncta, cudaStream_t stream) {
@@ -628,7 +663,7 @@ static cudaError_t launch_conv_t(const ConvArgs &a, cudaStream_t stream)
     if (T > 0 && a.dim % V == 0) {
         const int strips = (a.dim / V + kVecThreads - 1) / kVecThreads;
         // enough CTAs to fill the GPU once, each with at least 4 stages of rows
-        const long fill = (long)pipe_ctas_per_sm() * sm_count() / strips;
+        const long fill = (long)pipe_ctas(V, a.width) * sm_count() / strips;
         const long by_rows = (T + 4 * kPipeRows - 1) / (4 * kPipeRows);
         const int ncta = (int)(fill < by_rows ? (fill > 0 ? fill : 1) : by_rows);
         const dim3 grid((unsigned)ncta, (unsigned)strips);

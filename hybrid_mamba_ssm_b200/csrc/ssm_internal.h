@@ -23,6 +23,35 @@ struct StateUpdateArgs {
     int *status_dev;
 };
 
+// Speculative (multi-token) decode: ntok draft tokens per batch row, in
+// order, from the row's state; optional outputs per token.
+struct MultiUpdateArgs {
+    int batch, ntok, nheads, head_dim, d_state, ngroups;
+    int in_dtype, y_dtype;
+    float *state;                 // [rows][H][P][N] (rows = batch, or max_slots)
+    const int32_t *slot_idx;      // device [batch] or nullptr; < 0 = padding
+    int max_slots;
+    const void *x;                // [batch][ntok][H][P]
+    const float *dt, *A;          // dt [batch][ntok][H]
+    const void *B, *C;            // [batch][ntok][G][N]
+    const float *D;
+    const int32_t *accept_len;    // device [batch] or nullptr (state not written)
+    float *inter;                 // [batch][ntok][H][P][N] or nullptr
+    void *y;                      // [batch][ntok][H][P] or nullptr
+    int *status_dev;
+};
+
+// Scatter of accepted intermediate states into the state rows.
+struct CommitArgs {
+    int batch, ntok, nheads, head_dim, d_state;
+    const float *inter;           // [batch][ntok][H][P][N]
+    const int32_t *accept_len;    // device [batch]
+    float *state;
+    const int32_t *slot_idx;
+    int max_slots;
+    int *status_dev;
+};
+
 struct ScanArgs {
     int nseq, seqlen;             // seqlen = T when cu_seqlens is given
     const int32_t *cu_seqlens;    // device [nseq+1] or nullptr
@@ -48,6 +77,11 @@ struct ScanArgs {
 // per batch row when update != 0; then nseq is the batch).
 struct ConvArgs {
     int update;
+    // decode only: ntok tokens per row (x, y [batch][ntok][dim]); the state
+    // row is rewritten after accept_len[b] tokens, after all of them when
+    // commit_all is set, or not at all.
+    int ntok, commit_all;
+    const int32_t *accept_len;
     int nseq, seqlen;             // seqlen = T when cu_seqlens is given
     const int32_t *cu_seqlens;
     int dim, width, activation;   // activation: 0 none, 1 SiLU
@@ -65,6 +99,8 @@ struct ConvArgs {
 
 cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);
 cudaError_t launch_conv1d(const ConvArgs &a, cudaStream_t stream);
+cudaError_t launch_state_update_multi(const MultiUpdateArgs &a, cudaStream_t stream);
+cudaError_t launch_state_commit(const CommitArgs &a, cudaStream_t stream);
 
 // General chunked scan on the CUDA cores: any supported shape and dtype.
 cudaError_t launch_scan_simt(const ScanArgs &a, cudaStream_t stream);

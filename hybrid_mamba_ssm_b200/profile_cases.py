@@ -4,6 +4,7 @@
     python -m hybrid_mamba_ssm_b200.profile_cases decode --batch 16 --heads 256
     python -m hybrid_mamba_ssm_b200.profile_cases conv --nseq 1 --seqlen 8192
     python -m hybrid_mamba_ssm_b200.profile_cases conv_update --batch 64
+    python -m hybrid_mamba_ssm_b200.profile_cases mtp --batch 16 --ntok 4 --mode verify
 
 Each case draws seeded inputs, runs ``--warmup`` untimed launches and then
 ``--launches`` more, and prints the device time of the last ones.  Inputs are
@@ -76,7 +77,25 @@ def conv_update(args, dev):
     return lambda: ssm.causal_conv1d_update(x, w, b, st, y=y)
 
 
-CASES = {"prefill": prefill, "decode": decode, "conv": conv, "conv_update": conv_update}
+def mtp(args, dev):
+    b, n, H, P, N, G = args.batch, args.ntok, args.heads, args.head_dim, args.d_state, args.groups
+    A, D = synth.make_head_params(83, H)
+    A, D = _f32(A, dev), _f32(D, dev)
+    state = _f32(synth.make_state(84, (b, H, P, N)), dev)
+    steps = [synth.make_decode_step(85 + k, b, H, P, N, G) for k in range(n)]
+    x = torch.stack([_bf16(s.x, dev) for s in steps], dim=1).contiguous()
+    Bt = torch.stack([_bf16(s.B, dev) for s in steps], dim=1).contiguous()
+    Ct = torch.stack([_bf16(s.C, dev) for s in steps], dim=1).contiguous()
+    dt = torch.stack([_f32(s.dt, dev) for s in steps], dim=1).contiguous()
+    acc = torch.full((b,), n, dtype=torch.int32, device=dev)
+    y = torch.empty((b, n, H, P), dtype=torch.bfloat16, device=dev)
+    if args.mode == "replay":
+        return lambda: ssm.ssm_state_update_multi(state, x, dt, A, Bt, Ct, D, accept_len=acc,
+                                                  want_y=False)
+    return lambda: ssm.ssm_state_update_multi(state, x, dt, A, Bt, Ct, D, y=y)
+
+
+CASES = {"mtp": mtp, "prefill": prefill, "decode": decode, "conv": conv, "conv_update": conv_update}
 
 
 def main():
@@ -91,6 +110,8 @@ def main():
     ap.add_argument("--groups", type=int, default=8)
     ap.add_argument("--chunk", type=int, default=128)
     ap.add_argument("--width", type=int, default=4)
+    ap.add_argument("--ntok", type=int, default=4)
+    ap.add_argument("--mode", choices=["verify", "replay"], default="verify")
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--launches", type=int, default=1)
     ap.add_argument("--graph", action="store_true")

@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED",
                 6: "SSM_ERR_DEVICE_INPUT"}
 EXPORTS = ("ssd_chunk_scan", "ssd_chunk_scan_workspace_size", "ssm_state_update",
            "ssd_chunk_scan_slots", "ssm_state_update_slots", "causal_conv1d_fwd",
-           "causal_conv1d_update", "ssm_status_string", "ssm_version")
+           "causal_conv1d_update", "ssm_state_update_multi", "ssm_state_commit",
+           "causal_conv1d_update_multi", "ssm_status_string", "ssm_version")
 ACTIVATIONS = {None: 0, "none": 0, "silu": 1}
 
 
@@ -50,6 +51,14 @@ def _load():
                                       vp, vp]
     lib.causal_conv1d_update.restype = i
     lib.causal_conv1d_update.argtypes = [i, i, i, i, vp, vp, vp, i, vp, i, vp, i, vp, vp, vp]
+    lib.ssm_state_update_multi.restype = i
+    lib.ssm_state_update_multi.argtypes = [i, i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp,
+                                           vp, vp, vp, i, vp, vp, vp]
+    lib.ssm_state_commit.restype = i
+    lib.ssm_state_commit.argtypes = [i, i, i, i, i, vp, vp, vp, i, vp, vp, vp]
+    lib.causal_conv1d_update_multi.restype = i
+    lib.causal_conv1d_update_multi.argtypes = [i, i, i, i, i, vp, vp, vp, i, vp, i, vp, vp, i,
+                                               vp, vp, vp]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_status_string.argtypes = [i]
     lib.ssm_version.restype = i
@@ -335,4 +344,88 @@ def causal_conv1d_update(x, weight, bias, conv_state, activation="silu", slot_id
                                   _ptr(slot_idx), _dtype_code(y.dtype), _ptr(y), _ptr(status),
                                   _stream(stream))
     _check(st, "causal_conv1d_update")
+    return y
+
+
+def ssm_state_update_multi(state, x, dt, A, B, C, D=None, slot_idx=None, accept_len=None,
+                           inter_states=None, y=None, y_dtype=None, want_y=True,
+                           want_inter=False, status=None, stream=None):
+    """Speculative decode: ntok draft tokens per batch row from the row's state.
+
+    state : [rows, H, P, N] fp32 (rows = batch, or a pool with slot_idx);
+    x : [batch, ntok, H, P]; dt : [batch, ntok, H]; B, C : [batch, ntok, G, N].
+    accept_len : int32 [batch] or None -- rewrite each row with its state after
+    accept_len[b] tokens (None: the state is only read).
+    Returns (y or None, inter_states or None); inter_states [batch, ntok, H, P,
+    N] fp32 holds the state after each draft token when want_inter is set.
+    """
+    _dev(state, "state", torch.float32)
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    batch, ntok, H, P = x.shape
+    N = state.shape[-1]
+    G = B.shape[-2]
+    for t, n, d in ((dt, "dt", torch.float32), (A, "A", torch.float32), (B, "B", x.dtype),
+                    (C, "C", x.dtype), (D, "D", torch.float32), (slot_idx, "slot_idx", torch.int32),
+                    (accept_len, "accept_len", torch.int32), (status, "status", torch.int32)):
+        _dev(t, n, d)
+    if want_inter and inter_states is None:
+        inter_states = torch.empty((batch, ntok, H, P, N), dtype=torch.float32, device=x.device)
+    _dev(inter_states, "inter_states", torch.float32)
+    if want_y and y is None:
+        y = torch.empty((batch, ntok, H, P), dtype=y_dtype or x.dtype, device=x.device)
+    if y is not None:
+        _dev(y, "y")
+    y_code = _dtype_code(y.dtype) if y is not None else in_code
+    max_slots = state.shape[0] if slot_idx is not None else 0
+    st = lib.ssm_state_update_multi(batch, ntok, H, P, N, G, in_code, _ptr(state), max_slots,
+                                    _ptr(slot_idx), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                                    _ptr(D), _ptr(accept_len), _ptr(inter_states), y_code,
+                                    _ptr(y), _ptr(status), _stream(stream))
+    _check(st, "ssm_state_update_multi")
+    return y, inter_states
+
+
+def ssm_state_commit(inter_states, accept_len, state, slot_idx=None, status=None, stream=None):
+    """state row of b <- inter_states[b, accept_len[b] - 1] (unchanged where 0)."""
+    _dev(inter_states, "inter_states", torch.float32)
+    _dev(accept_len, "accept_len", torch.int32)
+    _dev(state, "state", torch.float32)
+    _dev(slot_idx, "slot_idx", torch.int32)
+    _dev(status, "status", torch.int32)
+    batch, ntok, H, P, N = inter_states.shape
+    max_slots = state.shape[0] if slot_idx is not None else 0
+    st = lib.ssm_state_commit(batch, ntok, H, P, N, _ptr(inter_states), _ptr(accept_len),
+                              _ptr(state), max_slots, _ptr(slot_idx), _ptr(status),
+                              _stream(stream))
+    _check(st, "ssm_state_commit")
+
+
+def causal_conv1d_update_multi(x, weight, bias, conv_state, activation="silu", slot_idx=None,
+                               accept_len=None, y=None, y_dtype=None, want_y=True,
+                               status=None, stream=None):
+    """ntok draft tokens per batch row through the causal conv1d.  x : [batch,
+    ntok, dim]; conv_state [rows, dim, width-1] is rewritten with the window
+    after accept_len[b] tokens (None: only read).  Returns y or None."""
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    batch, ntok, dim = x.shape
+    _dev(weight, "weight", torch.float32)
+    width = weight.shape[-1]
+    _dev(bias, "bias", torch.float32)
+    _dev(conv_state, "conv_state", x.dtype)
+    _dev(slot_idx, "slot_idx", torch.int32)
+    _dev(accept_len, "accept_len", torch.int32)
+    _dev(status, "status", torch.int32)
+    if want_y and y is None:
+        y = torch.empty((batch, ntok, dim), dtype=y_dtype or x.dtype, device=x.device)
+    if y is not None:
+        _dev(y, "y")
+    y_code = _dtype_code(y.dtype) if y is not None else in_code
+    max_slots = conv_state.shape[0] if (conv_state is not None and slot_idx is not None) else 0
+    st = lib.causal_conv1d_update_multi(batch, ntok, dim, width, in_code, _ptr(x), _ptr(weight),
+                                        _ptr(bias), _activation(activation), _ptr(conv_state),
+                                        max_slots, _ptr(slot_idx), _ptr(accept_len), y_code,
+                                        _ptr(y), _ptr(status), _stream(stream))
+    _check(st, "causal_conv1d_update_multi")
     return y

@@ -267,6 +267,75 @@ SSM_API int causal_conv1d_update(int batch, int dim, int width, int in_dtype, co
                                  void *conv_state, int max_slots, const int32_t *slot_idx,
                                  int y_dtype, void *y, int *status_dev, cudaStream_t stream);
 
+/*
+ * Speculative (multi-token) decode.  A draft proposes ntok candidate tokens
+ * per batch row; the model verifies them in one call, each candidate
+ * producing an intermediate state, and the number accepted decides which
+ * intermediate state (recurrent and conv) becomes the row's state (the
+ * "MTP / speculative decoding" item of the deep-research note; multi-token
+ * prediction with a draft model in "How NVIDIA's new Nemotron model works",
+ * section "训练流程与推理加速").  Two flows are supported:
+ *   1. verify with inter_states, then ssm_state_commit scatters
+ *      inter_states[b][accept_len[b]-1] into the row (state read once,
+ *      ntok states written);
+ *   2. verify without inter_states, then call ssm_state_update_multi again
+ *      on the same draft inputs with accept_len and y = NULL, which rewrites
+ *      the row in place (state read twice, written once: the cheaper flow on
+ *      HBM for ntok >= 2).
+ */
+
+/*
+ * ssm_state_update_multi -- ntok tokens per batch row, in order, from the
+ * row's fp32 state (state[b], or state[slot_idx[b]] of a pool).
+ *   x  [batch][ntok][nheads][head_dim]     dt [batch][ntok][nheads] fp32
+ *   B, C [batch][ntok][ngroups][d_state]   A, D as for ssm_state_update
+ *   y  [batch][ntok][nheads][head_dim] or NULL
+ *   inter_states  fp32 [batch][ntok][nheads][head_dim][d_state] or NULL: the
+ *                 state after each draft token
+ *   accept_len    device int32 [batch] or NULL.  When given, the row is
+ *                 rewritten with the state after accept_len[b] tokens
+ *                 (0 leaves it unchanged); a value outside [0, ntok] skips
+ *                 the row and sets SSM_ERR_DEVICE_INPUT.  When NULL the
+ *                 state is only read.
+ *   slot_idx / max_slots  as for ssm_state_update_slots (negative = padding);
+ *                 NULL / 0 when the state has one row per batch row.
+ * At least one of y, inter_states, accept_len must be given.  No output may
+ * overlap an input or another output.
+ */
+SSM_API int ssm_state_update_multi(int batch, int ntok, int nheads, int head_dim, int d_state,
+                                   int ngroups, int in_dtype, float *state, int max_slots,
+                                   const int32_t *slot_idx, const void *x, const float *dt,
+                                   const float *A, const void *B, const void *C,
+                                   const float *D, const int32_t *accept_len,
+                                   float *inter_states, int y_dtype, void *y,
+                                   int *status_dev, cudaStream_t stream);
+
+/*
+ * ssm_state_commit -- state row of b <- inter_states[b][accept_len[b] - 1]
+ * (unchanged where accept_len[b] == 0; outside [0, ntok]: skipped and
+ * SSM_ERR_DEVICE_INPUT).  Layouts as for ssm_state_update_multi.
+ */
+SSM_API int ssm_state_commit(int batch, int ntok, int nheads, int head_dim, int d_state,
+                             const float *inter_states, const int32_t *accept_len,
+                             float *state, int max_slots, const int32_t *slot_idx,
+                             int *status_dev, cudaStream_t stream);
+
+/*
+ * causal_conv1d_update_multi -- ntok tokens per batch row through the
+ * causal conv1d from the row's conv state.  x, y [batch][ntok][dim] (y may
+ * be NULL when accept_len is given).  accept_len as for
+ * ssm_state_update_multi: the conv state row is rewritten with its window
+ * after accept_len[b] tokens, or left alone when accept_len is NULL.  The
+ * intermediate conv states are not materialised: the commit call recomputes
+ * the window from the draft inputs, which costs (width-1) values per channel.
+ */
+SSM_API int causal_conv1d_update_multi(int batch, int ntok, int dim, int width, int in_dtype,
+                                       const void *x, const float *weight, const float *bias,
+                                       int activation, void *conv_state, int max_slots,
+                                       const int32_t *slot_idx, const int32_t *accept_len,
+                                       int y_dtype, void *y, int *status_dev,
+                                       cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -248,3 +248,73 @@ def test_conv_update_rejects(clib, kw, code):
 
 def test_conv_update_batch_zero_is_noop(clib):
     assert conv_update(clib, batch=0, x=None, y=None, state=None) == OK
+
+
+@pytest.fixture(scope="module")
+def mlib(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.ssm_state_update_multi.restype = i
+    lib.ssm_state_update_multi.argtypes = [i, i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp,
+                                           vp, vp, vp, i, vp, vp, vp]
+    lib.ssm_state_commit.restype = i
+    lib.ssm_state_commit.argtypes = [i, i, i, i, i, vp, vp, vp, i, vp, vp, vp]
+    lib.causal_conv1d_update_multi.restype = i
+    lib.causal_conv1d_update_multi.argtypes = [i, i, i, i, i, vp, vp, vp, i, vp, i, vp, vp, i,
+                                               vp, vp, vp]
+    return lib
+
+
+def multi(lib, batch=2, ntok=3, H=4, P=64, N=128, G=2, state=0x1000000, max_slots=0, slots=None,
+          x=0x100000, acc=None, inter=None, y=0x200000):
+    return lib.ssm_state_update_multi(batch, ntok, H, P, N, G, BF16, state, max_slots, slots, x,
+                                      0x300000, 0x310000, 0x320000, 0x330000, None, acc, inter,
+                                      BF16, y, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ntok=-1), INVALID),
+    (dict(state=None), INVALID),
+    (dict(y=None), INVALID),                        # no output asked for
+    (dict(slots=0x400000), INVALID),                # slot map without a pool size
+    (dict(acc=0x400004), MISALIGNED),
+    (dict(inter=0x1000000 + 4096), INVALID),        # intermediates inside the state
+    (dict(N=48), UNSUPPORTED),
+])
+def test_multi_rejects(mlib, kw, code):
+    assert multi(mlib, **kw) == code
+
+
+def test_multi_noops(mlib):
+    assert multi(mlib, ntok=0, state=None, x=None, y=None) == OK
+    assert multi(mlib, batch=0, state=None, x=None, y=None) == OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(inter=None), INVALID),
+    (dict(acc=None), INVALID),
+    (dict(state=0x500000 + 64), INVALID),           # state inside the intermediates
+    (dict(d_state=100), UNSUPPORTED),
+])
+def test_commit_rejects(mlib, kw, code):
+    args = dict(batch=2, ntok=3, H=4, P=64, d_state=128, inter=0x500000, acc=0x400000,
+                state=0x9000000)
+    args.update(kw)
+    assert mlib.ssm_state_commit(args["batch"], args["ntok"], args["H"], args["P"],
+                                 args["d_state"], args["inter"], args["acc"], args["state"], 0,
+                                 None, None, None) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(y=None), INVALID),                        # neither y nor a commit
+    (dict(width=9), UNSUPPORTED),
+    (dict(state=None), INVALID),
+    (dict(y=0x100000 + 32), INVALID),               # y overlaps x
+])
+def test_conv_multi_rejects(mlib, kw, code):
+    args = dict(batch=2, ntok=3, dim=256, width=4, x=0x100000, state=0x300000, acc=None,
+                y=0x400000)
+    args.update(kw)
+    assert mlib.causal_conv1d_update_multi(args["batch"], args["ntok"], args["dim"],
+                                           args["width"], BF16, args["x"], 0x200000, None, 1,
+                                           args["state"], 0, None, args["acc"], BF16, args["y"],
+                                           None, None) == code
