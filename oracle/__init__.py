@@ -22,7 +22,8 @@ semiseparable (SSD) matrix form, closed forms for dt = 0, A = 0, d_state = 1
 and time-invariant inputs, split-and-carry, and linearity),
 tests/test_oracle_conv.py (numpy's correlate, the logistic function) and
 tests/test_oracle_mtp.py (the matrix form over each draft prefix, correlate
-over [conv state, draft inputs]).
+over [conv state, draft inputs]) and tests/test_oracle_fused.py (torch's
+softplus, silu and rms_norm; closed forms).
 """
 from __future__ import annotations
 
@@ -306,3 +307,45 @@ def causal_conv1d_update_multi(x, weight, bias, state, activation="silu", accept
             if acc[b] > 0:
                 new[b] = states[acc[b] - 1][b]
     return y, new
+
+
+def dt_transform(dt, dt_bias=None, softplus=False, dt_min=None, dt_max=None):
+    """The step size the recurrence uses, from the projection's raw dt
+    (the dt_bias input of the TensorRT MambaPlugin in the deep-research
+    note, "TensorRT Plugin 做 selective state update"; softplus then the
+    time-step clamp of the Mamba-2 mixer): per (token, head h)
+
+        v = dt + dt_bias[h];  v = log(1 + e^v) if softplus;  clamp to [dt_min, dt_max]
+
+    dt : [..., H] (last axis = heads).  fp64, numpy only.
+    """
+    v = _f64(dt).copy()
+    if dt_bias is not None:
+        v = v + _f64(dt_bias)
+    if softplus:
+        v = np.logaddexp(0.0, v)
+    if dt_min is not None:
+        v = np.maximum(v, float(dt_min))
+    if dt_max is not None:
+        v = np.minimum(v, float(dt_max))
+    return v
+
+
+def gated_rmsnorm(y, z, weight, group_size, eps=1e-5):
+    """Gated group RMSNorm after the scan, gate first (norm_before_gate =
+    False; the _gated_group_rmsnorm step of the MAX nemotron_h article,
+    section 5.4 item 4): per row and per group of group_size channels,
+
+        g = y * silu(z),   out = g / sqrt(mean_group(g^2) + eps) * weight
+
+    y, z : [rows, dim]; weight : [dim].  fp64, numpy only.
+    """
+    yf, zf, wf = _f64(y), _f64(z), _f64(weight)
+    rows, dim = yf.shape
+    if dim % group_size:
+        raise ValueError("dim must be a multiple of group_size")
+    g = yf * zf / (1.0 + np.exp(-zf))
+    gg = g.reshape(rows, dim // group_size, group_size)
+    ms = np.mean(gg * gg, axis=-1, keepdims=True)
+    out = (gg / np.sqrt(ms + eps)).reshape(rows, dim) * wf
+    return out
