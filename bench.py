@@ -405,6 +405,92 @@ def time_mtp(dev, stream, seed, iters=20):
     return out
 
 
+NORM = dict(prefill=dict(rows=16384, dim=128 * 64, group=1024),
+            decode=dict(rows=64, dim=256 * 64, group=2048))
+
+
+def time_fused(dev, stream, seed, iters=20):
+    """Device time of the steps on either side of the scan: the gated group
+    RMSNorm at the prefill and decode shapes (bf16 y, z, out; y, z read and
+    out written once: 6 bytes per element), and the 4x4096 prefill fed the
+    raw dt with dt_bias + softplus + clamp applied inside the kernel."""
+    import torch
+    from hybrid_mamba_ssm_b200 import inputs as synth
+    from hybrid_mamba_ssm_b200 import ssm
+
+    def bf16(t):
+        return torch.from_numpy(np.ascontiguousarray(t.bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    def timed(fn, graph=False):
+        """ms per call: per-launch events, or (for calls of a few microseconds,
+        where the host's launch rate would set the time) the replay of a CUDA
+        graph of `iters` calls."""
+        for _ in range(3):
+            fn(stream)
+        torch.cuda.synchronize(dev)
+        if graph:
+            gs = torch.cuda.Stream(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(gs):
+                with torch.cuda.graph(g, stream=gs):
+                    for _ in range(iters):
+                        fn(gs)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            return e0.elapsed_time(e1) / iters
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(iters)]
+        for e0, e1 in ev:
+            e0.record(stream)
+            fn(stream)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
+
+    out = {}
+    for name, c in NORM.items():
+        y, z, w = synth.make_gate(seed + len(out), c["rows"], c["dim"])
+        yd, zd, wd = bf16(y), bf16(z), torch.from_numpy(w).to(dev)
+        od = torch.empty_like(yd)
+        ms = timed(lambda st: ssm.ssm_gated_rmsnorm(yd, zd, wd, c["group"], out=od, stream=st),
+                   graph=(name == "decode"))
+        nbytes = c["rows"] * c["dim"] * 6 + c["dim"] * 4
+        out["gated_rmsnorm_" + name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                                        "bytes_per_launch": nbytes, "launches": iters,
+                                        "timing": "CUDA graph replay" if name == "decode"
+                                        else "per-launch events",
+                                        "shape": f"{c['rows']} x {c['dim']}, groups of {c['group']}"}
+    p = PREFILL
+    inp = synth.make_scan_inputs(seed + 7, [p["seqlen"]] * p["nseq"], p["H"], p["P"], p["N"],
+                                 p["G"], dtype="bf16")
+    raw, bias = synth.make_raw_dt(seed + 8, (p["nseq"] * p["seqlen"], p["H"]), p["H"])
+    L = p["seqlen"]
+    x = bf16(inp.x).view(p["nseq"], L, p["H"], p["P"])
+    B = bf16(inp.B).view(p["nseq"], L, p["G"], p["N"])
+    C = bf16(inp.C).view(p["nseq"], L, p["G"], p["N"])
+    dt = torch.from_numpy(raw).to(dev).view(p["nseq"], L, p["H"])
+    A, D = torch.from_numpy(inp.A).to(dev), torch.from_numpy(inp.D).to(dev)
+    pool = torch.zeros((p["nseq"], p["H"], p["P"], p["N"]), dtype=torch.float32, device=dev)
+    fresh = torch.zeros(p["nseq"], dtype=torch.int32, device=dev)
+    y = torch.empty_like(x)
+    bias_d = torch.from_numpy(bias).to(dev)
+    ms = timed(lambda st: ssm.ssd_chunk_scan_slots(x, dt, A, B, C, D, pool, None,
+                                                   has_initial_state=fresh, y=y, stream=st,
+                                                   dt_bias=bias_d, dt_softplus=True,
+                                                   dt_limit=(1e-3, 0.1)))
+    flops, nbytes, T = prefill_work()
+    out["prefill_raw_dt"] = {"ms": ms, "tokens_per_s": T / (ms * 1e-3),
+                             "tflops": flops / (ms * 1e-3) / 1e12, "launches": iters,
+                             "dt": "raw dt; bias, softplus and clamp inside the scan"}
+    return out
+
+
 def run_reference(args, world, rank, pg):
     if rank != 0:
         return 0
@@ -590,11 +676,13 @@ def run_ours(args, world, rank, local, pg):
 
     conv = time_conv(dev, stream, seed + 17)
     conv.update(time_mtp(dev, stream, seed + 29))
+    conv.update(time_fused(dev, stream, seed + 41))
 
     # ---- numbers ----
     peaks, peak_kind = load_peaks()
     for part in conv.values():
-        part["hbm_frac"] = part["gbs"] / peaks["hbm_gbs"]
+        if "gbs" in part:
+            part["hbm_frac"] = part["gbs"] / peaks["hbm_gbs"]
     tok_step = p["nseq"] * p["seqlen"] + d["batch"]
     value = world * tok_step * K / (ms * 1e-3)
     e2e_value = world * tok_step * e2e_steps / (e2e_ms * 1e-3)

@@ -36,6 +36,22 @@ bool pow2_in(int v, int lo, int hi)
     return v >= lo && v <= hi && (v & (v - 1)) == 0;
 }
 
+// Device-side form of the optional dt transform.  Returns SSM_OK, or the
+// status for a malformed one (misaligned bias, dt_min > dt_max, NaN bounds).
+int read_dt_params(const ssm_dt_params *p, ssm::DtParams &out)
+{
+    out = ssm::DtParams{};
+    if (!p) return SSM_OK;
+    if (p->dt_bias && !aligned16(p->dt_bias)) return SSM_ERR_MISALIGNED;
+    if (p->clamp && !(p->dt_min <= p->dt_max)) return SSM_ERR_INVALID_ARG;
+    out.bias = p->dt_bias;
+    out.softplus = p->softplus != 0;
+    out.clamp = p->clamp != 0;
+    out.lo = p->dt_min;
+    out.hi = p->dt_max;
+    return SSM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -115,7 +131,7 @@ int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
     if (initial_state && final_state && initial_state != final_state && overlap(rh0, rhT))
         return SSM_ERR_INVALID_ARG;
 
-    ssm::ScanArgs a;
+    ssm::ScanArgs a{};
     a.nseq = nseq; a.seqlen = seqlen; a.cu_seqlens = cu_seqlens;
     a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
     a.ngroups = ngroups; a.chunk_size = chunk_size;
@@ -134,6 +150,7 @@ int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
                          int chunk_size, int in_dtype,
                          const void *x, const float *dt, const float *A,
                          const void *B, const void *C, const float *D,
+                         const ssm_dt_params *dt_params,
                          float *state_pool, int max_slots, const int32_t *slot_idx,
                          const int32_t *has_initial_state,
                          int y_dtype, void *y, int *status_dev, cudaStream_t stream)
@@ -144,7 +161,10 @@ int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
     if (!pow2_in(head_dim, 16, 128) || !pow2_in(d_state, 16, 128)) return SSM_ERR_UNSUPPORTED;
     if (chunk_size != 64 && chunk_size != 128) return SSM_ERR_UNSUPPORTED;
     if (nseq == 0) return SSM_OK;
-    if (max_slots <= 0 || !state_pool || !slot_idx || !A) return SSM_ERR_INVALID_ARG;
+    if (max_slots <= 0 || !state_pool || !A) return SSM_ERR_INVALID_ARG;
+    if (!slot_idx && max_slots < nseq) return SSM_ERR_INVALID_ARG;   // row s per sequence
+    ssm::DtParams dtp;
+    if (const int st = read_dt_params(dt_params, dtp)) return st;
     const long long T = cu_seqlens ? (long long)seqlen : (long long)nseq * seqlen;
     if (T > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
     if (T > 0 && (!x || !dt || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
@@ -161,14 +181,15 @@ int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
                          range_of(B, (size_t)T * ngroups * d_state * es),
                          range_of(C, (size_t)T * ngroups * d_state * es),
                          range_of(D, D ? (size_t)nheads * sizeof(float) : 0),
-                         range_of(slot_idx, (size_t)nseq * sizeof(int32_t)),
+                         range_of(slot_idx, slot_idx ? (size_t)nseq * sizeof(int32_t) : 0),
                          range_of(has_initial_state, has_initial_state ? (size_t)nseq * sizeof(int32_t) : 0),
+                         range_of(dtp.bias, dtp.bias ? (size_t)nheads * sizeof(float) : 0),
                          range_of(cu_seqlens, cu_seqlens ? (size_t)(nseq + 1) * sizeof(int32_t) : 0)};
     for (const Range &r : ins)
         if (overlap(ry, r) || overlap(rpool, r)) return SSM_ERR_INVALID_ARG;
     if (overlap(ry, rpool)) return SSM_ERR_INVALID_ARG;
 
-    ssm::ScanArgs a;
+    ssm::ScanArgs a{};
     a.nseq = nseq; a.seqlen = seqlen; a.cu_seqlens = cu_seqlens;
     a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
     a.ngroups = ngroups; a.chunk_size = chunk_size;
@@ -177,6 +198,7 @@ int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
     a.initial_state = state_pool; a.y = y; a.final_state = state_pool;
     a.status_dev = status_dev;
     a.slot_idx = slot_idx; a.has_initial = has_initial_state; a.max_slots = max_slots;
+    a.dtp = dtp;
     // empty sequences still run: a slot without an initial state is reset to zero
     const cudaError_t e = ssm::scan_tc_supports(a) ? ssm::launch_scan_tc(a, stream)
                                                    : ssm::launch_scan_simt(a, stream);
@@ -214,7 +236,7 @@ int ssm_state_update(int batch, int nheads, int head_dim, int d_state,
         if (overlap(ry, r) || overlap(rs, r)) return SSM_ERR_INVALID_ARG;
     if (overlap(ry, rs)) return SSM_ERR_INVALID_ARG;
 
-    ssm::StateUpdateArgs a;
+    ssm::StateUpdateArgs a{};
     a.batch = batch; a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
     a.ngroups = ngroups; a.in_dtype = in_dtype; a.y_dtype = y_dtype;
     a.state = state; a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.y = y;
@@ -227,6 +249,7 @@ int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
                            const int32_t *slot_idx,
                            const void *x, const float *dt, const float *A,
                            const void *B, const void *C, const float *D,
+                           const ssm_dt_params *dt_params,
                            int y_dtype, void *y, int *status_dev, cudaStream_t stream)
 {
     if (batch < 0 || nheads <= 0 || ngroups <= 0 || nheads % ngroups || head_dim <= 0)
@@ -235,8 +258,11 @@ int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
     if (head_dim > 256 || !pow2_in(d_state, 16, 256)) return SSM_ERR_UNSUPPORTED;
     if ((long long)batch * nheads > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
     if (batch == 0) return SSM_OK;
-    if (max_slots <= 0 || !state_pool || !slot_idx || !x || !dt || !A || !B || !C || !y)
+    if (max_slots <= 0 || !state_pool || !x || !dt || !A || !B || !C || !y)
         return SSM_ERR_INVALID_ARG;
+    if (!slot_idx && max_slots < batch) return SSM_ERR_INVALID_ARG;   // row b per batch row
+    ssm::DtParams dtp;
+    if (const int st = read_dt_params(dt_params, dtp)) return st;
     const void *ptrs[] = {state_pool, slot_idx, x, dt, A, B, C, D, y, status_dev};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
@@ -249,16 +275,18 @@ int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
                          range_of(B, (size_t)batch * ngroups * d_state * es),
                          range_of(C, (size_t)batch * ngroups * d_state * es),
                          range_of(D, D ? (size_t)nheads * sizeof(float) : 0),
-                         range_of(slot_idx, (size_t)batch * sizeof(int32_t))};
+                         range_of(slot_idx, slot_idx ? (size_t)batch * sizeof(int32_t) : 0),
+                         range_of(dtp.bias, dtp.bias ? (size_t)nheads * sizeof(float) : 0)};
     for (const Range &r : ins)
         if (overlap(ry, r) || overlap(rs, r)) return SSM_ERR_INVALID_ARG;
     if (overlap(ry, rs)) return SSM_ERR_INVALID_ARG;
 
-    ssm::StateUpdateArgs a;
+    ssm::StateUpdateArgs a{};
     a.batch = batch; a.nheads = nheads; a.head_dim = head_dim; a.d_state = d_state;
     a.ngroups = ngroups; a.in_dtype = in_dtype; a.y_dtype = y_dtype;
     a.state = state_pool; a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.y = y;
     a.slot_idx = slot_idx; a.max_slots = max_slots; a.status_dev = status_dev;
+    a.dtp = dtp;
     return ssm::launch_state_update(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -392,6 +420,7 @@ int ssm_state_update_multi(int batch, int ntok, int nheads, int head_dim, int d_
                            int ngroups, int in_dtype, float *state, int max_slots,
                            const int32_t *slot_idx, const void *x, const float *dt,
                            const float *A, const void *B, const void *C, const float *D,
+                           const ssm_dt_params *dt_params,
                            const int32_t *accept_len, float *inter_states, int y_dtype, void *y,
                            int *status_dev, cudaStream_t stream)
 {
@@ -405,6 +434,8 @@ int ssm_state_update_multi(int batch, int ntok, int nheads, int head_dim, int d_
     if (!state || !x || !dt || !A || !B || !C) return SSM_ERR_INVALID_ARG;
     if (!y && !inter_states && !accept_len) return SSM_ERR_INVALID_ARG;
     if (slot_idx && max_slots <= 0) return SSM_ERR_INVALID_ARG;
+    ssm::DtParams dtp;
+    if (const int st = read_dt_params(dt_params, dtp)) return st;
     const void *ptrs[] = {state, slot_idx, x, dt, A, B, C, D, accept_len, inter_states, y,
                           status_dev};
     for (const void *p : ptrs)
@@ -423,17 +454,19 @@ int ssm_state_update_multi(int batch, int ntok, int nheads, int head_dim, int d_
                          range_of(C, bt * ngroups * d_state * es),
                          range_of(D, D ? (size_t)nheads * sizeof(float) : 0),
                          range_of(slot_idx, slot_idx ? (size_t)batch * sizeof(int32_t) : 0),
-                         range_of(accept_len, accept_len ? (size_t)batch * sizeof(int32_t) : 0)};
+                         range_of(accept_len, accept_len ? (size_t)batch * sizeof(int32_t) : 0),
+                         range_of(dtp.bias, dtp.bias ? (size_t)nheads * sizeof(float) : 0)};
     for (const Range &r : ins)
         if (overlap(ry, r) || overlap(rs, r) || overlap(ri, r)) return SSM_ERR_INVALID_ARG;
     if (overlap(ry, rs) || overlap(ri, rs) || overlap(ri, ry)) return SSM_ERR_INVALID_ARG;
 
-    ssm::MultiUpdateArgs a;
+    ssm::MultiUpdateArgs a{};
     a.batch = batch; a.ntok = ntok; a.nheads = nheads; a.head_dim = head_dim;
     a.d_state = d_state; a.ngroups = ngroups; a.in_dtype = in_dtype; a.y_dtype = y_dtype;
     a.state = state; a.slot_idx = slot_idx; a.max_slots = max_slots;
     a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D;
     a.accept_len = accept_len; a.inter = inter_states; a.y = y; a.status_dev = status_dev;
+    a.dtp = dtp;
     return ssm::launch_state_update_multi(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
@@ -460,11 +493,43 @@ int ssm_state_commit(int batch, int ntok, int nheads, int head_dim, int d_state,
     for (const Range &r : ins)
         if (overlap(rs, r)) return SSM_ERR_INVALID_ARG;
 
-    ssm::CommitArgs a;
+    ssm::CommitArgs a{};
     a.batch = batch; a.ntok = ntok; a.nheads = nheads; a.head_dim = head_dim;
     a.d_state = d_state; a.inter = inter_states; a.accept_len = accept_len; a.state = state;
     a.slot_idx = slot_idx; a.max_slots = max_slots; a.status_dev = status_dev;
     return ssm::launch_state_commit(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_gated_rmsnorm(int rows, int dim, int group_size, int y_dtype, const void *y,
+                      int z_dtype, const void *z, const float *weight, float eps,
+                      int out_dtype, void *out, cudaStream_t stream)
+{
+    if (rows < 0 || dim <= 0 || group_size <= 0) return SSM_ERR_INVALID_ARG;
+    if (!valid_dtype(y_dtype) || !valid_dtype(z_dtype) || !valid_dtype(out_dtype))
+        return SSM_ERR_INVALID_ARG;
+    if (dim % group_size || !(eps >= 0.f)) return SSM_ERR_INVALID_ARG;
+    if (group_size % 256 || group_size > 8192) return SSM_ERR_UNSUPPORTED;   // whole warps
+    if ((long long)rows * (dim / group_size) > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    if (rows == 0) return SSM_OK;
+    if (!y || !z || !weight || !out) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {y, z, weight, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return SSM_ERR_MISALIGNED;
+    const size_t n = (size_t)rows * dim;
+    const Range ro = range_of(out, n * dtype_size(out_dtype));
+    const Range ryr = range_of(y, n * dtype_size(y_dtype));
+    // out may be y itself (same dtype: each element is read before it is written)
+    const bool in_place = out == y && out_dtype == y_dtype;
+    if (!in_place && overlap(ro, ryr)) return SSM_ERR_INVALID_ARG;
+    if (overlap(ro, range_of(z, n * dtype_size(z_dtype))) ||
+        overlap(ro, range_of(weight, (size_t)dim * sizeof(float))))
+        return SSM_ERR_INVALID_ARG;
+
+    ssm::GatedNormArgs a{};
+    a.rows = rows; a.dim = dim; a.group_size = group_size;
+    a.y_dtype = y_dtype; a.z_dtype = z_dtype; a.out_dtype = out_dtype;
+    a.y = y; a.z = z; a.weight = weight; a.eps = eps; a.out = out;
+    return ssm::launch_gated_rmsnorm(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 }  // extern "C"

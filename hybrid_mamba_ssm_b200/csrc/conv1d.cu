@@ -27,12 +27,6 @@ constexpr int kMaxWidth = 8;
 
 // SiLU as v * (1 / (1 + e^-v)) with the hardware approximate reciprocal
 // (rcp of +inf is 0, so large negative v gives -0 as the limit does).
-__device__ __forceinline__ float rcp_approx(float v) {
-    float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
-    return r;
-}
-
 __device__ __forceinline__ float conv_act(float v, int act) {
     return act ? v * rcp_approx(1.f + __expf(-v)) : v;
 }
@@ -216,12 +210,6 @@ __device__ __forceinline__ void store_row2(__nv_bfloat16 *p, const float2 (&v)[P
     }
     if constexpr (P2 == 4) *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
     else *reinterpret_cast<uint2 *>(p) = make_uint2(w[0], w[1]);
-}
-
-__device__ __forceinline__ float ex2_approx(float v) {
-    float r;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
-    return r;
 }
 
 // SiLU of two lanes: v / (1 + 2^(-v log2 e)), the exponential and the

@@ -108,7 +108,7 @@ scan_simt_kernel(ScanArgs a)
         const int Lc = (int)min((long)Q, t1 - c0);
         __syncthreads();
         for (int i = tid; i < Q; i += kSimtThreads)
-            dts[i] = (i < Lc) ? a.dt[(size_t)(c0 + i) * H + h] : 0.f;
+            dts[i] = (i < Lc) ? dt_apply(a.dtp, a.dt[(size_t)(c0 + i) * H + h], h) : 0.f;
         for (int i = tid; i < Q * N; i += kSimtThreads) {
             const int j = i / N, n = i - j * N;
             Bs[j * N1 + n] = (j < Lc) ? load_f32(Bg + ((size_t)(c0 + j) * G + g) * N + n) : 0.f;

@@ -270,7 +270,7 @@ __device__ __forceinline__ ChunkDecay chunk_decay(const ScanArgs &a, int H, int 
                                                   int ch, float *sPART, float *sCSB, float *vd_out)
 {
     ChunkDecay d;
-    d.dtv = (i < Lc) ? a.dt[(size_t)(c0 + i) * H + hh] : 0.f;
+    d.dtv = (i < Lc) ? dt_apply(a.dtp, a.dt[(size_t)(c0 + i) * H + hh], hh) : 0.f;
     float v = d.dtv * Ah;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace ssm {
 
 struct StateUpdateArgs {
@@ -21,6 +23,7 @@ struct StateUpdateArgs {
     const int32_t *slot_idx;      // device [batch]; < 0 skips the row
     int max_slots;
     int *status_dev;
+    DtParams dtp;                 // transform of dt (identity when all off)
 };
 
 // Speculative (multi-token) decode: ntok draft tokens per batch row, in
@@ -35,6 +38,7 @@ struct MultiUpdateArgs {
     const float *dt, *A;          // dt [batch][ntok][H]
     const void *B, *C;            // [batch][ntok][G][N]
     const float *D;
+    DtParams dtp;
     const int32_t *accept_len;    // device [batch] or nullptr (state not written)
     float *inter;                 // [batch][ntok][H][P][N] or nullptr
     void *y;                      // [batch][ntok][H][P] or nullptr
@@ -71,6 +75,7 @@ struct ScanArgs {
     const int32_t *slot_idx;
     const int32_t *has_initial;
     int max_slots;
+    DtParams dtp;
 };
 
 // Causal depthwise conv1d (prefill over packed sequences, or one decode token
@@ -101,6 +106,18 @@ cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);
 cudaError_t launch_conv1d(const ConvArgs &a, cudaStream_t stream);
 cudaError_t launch_state_update_multi(const MultiUpdateArgs &a, cudaStream_t stream);
 cudaError_t launch_state_commit(const CommitArgs &a, cudaStream_t stream);
+
+// Gated group RMSNorm (gate first): out = g / sqrt(mean_group(g^2) + eps) * w,
+// g = y * silu(z), over groups of group_size channels of each row.
+struct GatedNormArgs {
+    int rows, dim, group_size;
+    int y_dtype, z_dtype, out_dtype;
+    const void *y, *z;
+    const float *weight;
+    float eps;
+    void *out;
+};
+cudaError_t launch_gated_rmsnorm(const GatedNormArgs &a, cudaStream_t stream);
 
 // General chunked scan on the CUDA cores: any supported shape and dtype.
 cudaError_t launch_scan_simt(const ScanArgs &a, cudaStream_t stream);

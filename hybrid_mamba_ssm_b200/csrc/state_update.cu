@@ -30,7 +30,8 @@ state_update_kernel(int nheads, int head_dim, int heads_per_group, int ngroups,
                     const float *__restrict__ dt, const float *__restrict__ A,
                     const TIn *__restrict__ B, const TIn *__restrict__ C,
                     const float *__restrict__ D, TOut *__restrict__ y,
-                    const int32_t *__restrict__ slot_idx, int max_slots, int *status)
+                    const int32_t *__restrict__ slot_idx, int max_slots, int *status,
+                    DtParams dtp)
 {
     constexpr int LPR = (N / 4 < 32) ? N / 4 : 32;   // lanes per state row
     constexpr int VEC = N / (4 * LPR);               // float4s per lane
@@ -56,7 +57,7 @@ state_update_kernel(int nheads, int head_dim, int heads_per_group, int ngroups,
     const int li = lane % LPR;
     const int ri = lane / LPR;
 
-    const float dtv = __ldg(dt + bh);
+    const float dtv = dt_apply(dtp, __ldg(dt + bh), h);
     const float decay = expf(dtv * __ldg(A + h));
     const float Dh = D ? __ldg(D + h) : 0.f;
 
@@ -125,7 +126,7 @@ static cudaError_t launch_state_update_t(const StateUpdateArgs &a, cudaStream_t 
         a.nheads, a.head_dim, a.nheads / a.ngroups, a.ngroups, a.state,
         static_cast<const TIn *>(a.x), a.dt, a.A, static_cast<const TIn *>(a.B),
         static_cast<const TIn *>(a.C), a.D, static_cast<TOut *>(a.y), a.slot_idx, a.max_slots,
-        a.status_dev);
+        a.status_dev, a.dtp);
     return cudaGetLastError();
 }
 

@@ -100,7 +100,7 @@ state_update_multi_kernel(MultiUpdateArgs a)
                 sX[t][p] = load_f32(x + (((size_t)b * a.ntok + t0 + t) * H + h) * P + p);
             }
             if (threadIdx.x < nt) {
-                const float d = __ldg(a.dt + ((size_t)b * a.ntok + t0 + threadIdx.x) * H + h);
+                const float d = dt_apply(a.dtp, __ldg(a.dt + ((size_t)b * a.ntok + t0 + threadIdx.x) * H + h), h);
                 sDt[threadIdx.x] = d;
                 sDecay[threadIdx.x] = expf(d * Ah);
             }

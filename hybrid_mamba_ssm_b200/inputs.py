@@ -140,6 +140,25 @@ def make_decode_step(seed: int, batch: int, nheads: int, head_dim: int,
     return DecodeInputs(x=x, dt=dt, B=B, C=C)
 
 
+def make_raw_dt(seed: int, shape, nheads: int):
+    """Raw projection dt ~ N(0, 1) (fp32, shape [..., nheads]) and a per-head
+    dt_bias ~ U(-3.5, -2.5): softplus(dt + dt_bias) then spans the usual
+    clamp range [1e-3, 0.1] and beyond it on both sides."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    raw = rng.standard_normal(tuple(shape), dtype=np.float32)
+    bias = rng.uniform(-3.5, -2.5, nheads).astype(np.float32)
+    return raw, bias
+
+
+def make_gate(seed: int, rows: int, dim: int, dtype: str = "bf16"):
+    """Scan output y and gate z ~ N(0, 1), and an RMSNorm weight ~ U(0.5, 1.5)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    y = _store(rng.standard_normal((rows, dim), dtype=np.float32), dtype)
+    z = _store(rng.standard_normal((rows, dim), dtype=np.float32), dtype)
+    w = rng.uniform(0.5, 1.5, dim).astype(np.float32)
+    return y, z, w
+
+
 def make_head_params(seed: int, nheads: int):
     """Per-head (A, D) for a decode workload."""
     rng = np.random.Generator(np.random.PCG64(seed))

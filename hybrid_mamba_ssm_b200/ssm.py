@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED",
 EXPORTS = ("ssd_chunk_scan", "ssd_chunk_scan_workspace_size", "ssm_state_update",
            "ssd_chunk_scan_slots", "ssm_state_update_slots", "causal_conv1d_fwd",
            "causal_conv1d_update", "ssm_state_update_multi", "ssm_state_commit",
-           "causal_conv1d_update_multi", "ssm_status_string", "ssm_version")
+           "causal_conv1d_update_multi", "ssm_gated_rmsnorm", "ssm_status_string",
+           "ssm_version")
 ACTIVATIONS = {None: 0, "none": 0, "silu": 1}
 
 
@@ -41,11 +42,11 @@ def _load():
     lib.ssm_state_update.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, i,
                                      vp, vp]
     lib.ssd_chunk_scan_slots.restype = i
-    lib.ssd_chunk_scan_slots.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp,
+    lib.ssd_chunk_scan_slots.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp,
                                          vp, i, vp, vp, i, vp, vp, vp]
     lib.ssm_state_update_slots.restype = i
     lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp, vp,
-                                           i, vp, vp, vp]
+                                           vp, i, vp, vp, vp]
     lib.causal_conv1d_fwd.restype = i
     lib.causal_conv1d_fwd.argtypes = [i, i, vp, i, i, i, vp, vp, vp, i, vp, i, vp, vp, i, vp,
                                       vp, vp]
@@ -53,12 +54,14 @@ def _load():
     lib.causal_conv1d_update.argtypes = [i, i, i, i, vp, vp, vp, i, vp, i, vp, i, vp, vp, vp]
     lib.ssm_state_update_multi.restype = i
     lib.ssm_state_update_multi.argtypes = [i, i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp,
-                                           vp, vp, vp, i, vp, vp, vp]
+                                           vp, vp, vp, vp, i, vp, vp, vp]
     lib.ssm_state_commit.restype = i
     lib.ssm_state_commit.argtypes = [i, i, i, i, i, vp, vp, vp, i, vp, vp, vp]
     lib.causal_conv1d_update_multi.restype = i
     lib.causal_conv1d_update_multi.argtypes = [i, i, i, i, i, vp, vp, vp, i, vp, i, vp, vp, i,
                                                vp, vp, vp]
+    lib.ssm_gated_rmsnorm.restype = i
+    lib.ssm_gated_rmsnorm.argtypes = [i, i, i, i, vp, i, vp, vp, ctypes.c_float, i, vp, vp]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_status_string.argtypes = [i]
     lib.ssm_version.restype = i
@@ -66,6 +69,23 @@ def _load():
 
 
 lib = _load()
+
+
+class DtParams(ctypes.Structure):
+    """ssm_dt_params: dt <- clamp(softplus(dt + dt_bias[h])) inside the kernels."""
+    _fields_ = [("dt_bias", ctypes.c_void_p), ("softplus", ctypes.c_int), ("clamp", ctypes.c_int),
+                ("dt_min", ctypes.c_float), ("dt_max", ctypes.c_float)]
+
+
+def _dt_params(dt_bias, dt_softplus, dt_limit):
+    """A DtParams reference for the keyword arguments, or None when dt is final."""
+    if dt_bias is None and not dt_softplus and dt_limit is None:
+        return None
+    _dev(dt_bias, "dt_bias", torch.float32)
+    lo, hi = dt_limit if dt_limit is not None else (0.0, 0.0)
+    p = DtParams(None if dt_bias is None else dt_bias.data_ptr(), int(bool(dt_softplus)),
+                 int(dt_limit is not None), float(lo), float(hi))
+    return ctypes.byref(p)
 
 
 class SSMError(RuntimeError):
@@ -195,13 +215,17 @@ def ssm_state_update(state, x, dt, A, B, C, D=None, y=None, y_dtype=None, stream
 
 def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_state=None,
                          cu_seqlens=None, chunk_size: int = 128, y=None, y_dtype=None,
-                         status=None, stream=None):
+                         status=None, stream=None, dt_bias=None, dt_softplus=False,
+                         dt_limit=None):
     """Chunked SSD prefill whose states live in a pool, updated in place.
 
     state_pool : [max_slots, H, P, N] fp32; sequence s starts from
         state_pool[slot_idx[s]] (or zero where has_initial_state[s] == 0) and
         its final state is written back to the same row.
-    slot_idx, has_initial_state : int32 CUDA tensors [nseq].
+    slot_idx, has_initial_state : int32 CUDA tensors [nseq] (slot_idx None:
+        sequence s uses row s).
+    dt_bias [H] fp32, dt_softplus, dt_limit (lo, hi): transform the raw dt
+        inside the kernel (dt <- clamp(softplus(dt + dt_bias))).
     Other arguments as for ssd_chunk_scan.  Returns y.
     """
     _dev(x, "x")
@@ -229,9 +253,10 @@ def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_st
     if y is None:
         y = torch.empty(x.shape, dtype=y_dtype, device=x.device)
     _dev(y, "y", y_dtype)
+    dtp = _dt_params(dt_bias, dt_softplus, dt_limit)
     st = lib.ssd_chunk_scan_slots(nseq, seqlen, _ptr(cu_seqlens), H, P, N, G, int(chunk_size),
                                   in_code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                  _ptr(state_pool), state_pool.shape[0], _ptr(slot_idx),
+                                  dtp, _ptr(state_pool), state_pool.shape[0], _ptr(slot_idx),
                                   _ptr(has_initial_state), _dtype_code(y.dtype), _ptr(y),
                                   _ptr(status), _stream(stream))
     _check(st, "ssd_chunk_scan_slots")
@@ -239,7 +264,8 @@ def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_st
 
 
 def ssm_state_update_slots(state_pool, slot_idx, x, dt, A, B, C, D=None, y=None, y_dtype=None,
-                           status=None, stream=None):
+                           status=None, stream=None, dt_bias=None, dt_softplus=False,
+                           dt_limit=None):
     """One-token decode update of pool rows: batch row b updates
     state_pool[slot_idx[b]] in place (slot_idx[b] < 0: padding row, skipped).
     Returns y [batch, H, P] (padding rows left as they were)."""
@@ -261,9 +287,10 @@ def ssm_state_update_slots(state_pool, slot_idx, x, dt, A, B, C, D=None, y=None,
     if y is None:
         y = torch.zeros((batch, H, P), dtype=y_dtype, device=x.device)
     _dev(y, "y", y_dtype)
+    dtp = _dt_params(dt_bias, dt_softplus, dt_limit)
     st = lib.ssm_state_update_slots(batch, H, P, N, G, in_code, _ptr(state_pool),
                                     state_pool.shape[0], _ptr(slot_idx), _ptr(x), _ptr(dt),
-                                    _ptr(A), _ptr(B), _ptr(C), _ptr(D), _dtype_code(y.dtype),
+                                    _ptr(A), _ptr(B), _ptr(C), _ptr(D), dtp, _dtype_code(y.dtype),
                                     _ptr(y), _ptr(status), _stream(stream))
     _check(st, "ssm_state_update_slots")
     return y
@@ -349,7 +376,8 @@ def causal_conv1d_update(x, weight, bias, conv_state, activation="silu", slot_id
 
 def ssm_state_update_multi(state, x, dt, A, B, C, D=None, slot_idx=None, accept_len=None,
                            inter_states=None, y=None, y_dtype=None, want_y=True,
-                           want_inter=False, status=None, stream=None):
+                           want_inter=False, status=None, stream=None, dt_bias=None,
+                           dt_softplus=False, dt_limit=None):
     """Speculative decode: ntok draft tokens per batch row from the row's state.
 
     state : [rows, H, P, N] fp32 (rows = batch, or a pool with slot_idx);
@@ -380,7 +408,8 @@ def ssm_state_update_multi(state, x, dt, A, B, C, D=None, slot_idx=None, accept_
     max_slots = state.shape[0] if slot_idx is not None else 0
     st = lib.ssm_state_update_multi(batch, ntok, H, P, N, G, in_code, _ptr(state), max_slots,
                                     _ptr(slot_idx), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
-                                    _ptr(D), _ptr(accept_len), _ptr(inter_states), y_code,
+                                    _ptr(D), _dt_params(dt_bias, dt_softplus, dt_limit),
+                                    _ptr(accept_len), _ptr(inter_states), y_code,
                                     _ptr(y), _ptr(status), _stream(stream))
     _check(st, "ssm_state_update_multi")
     return y, inter_states
@@ -429,3 +458,23 @@ def causal_conv1d_update_multi(x, weight, bias, conv_state, activation="silu", s
                                         _ptr(y), _ptr(status), _stream(stream))
     _check(st, "causal_conv1d_update_multi")
     return y
+
+
+def ssm_gated_rmsnorm(y, z, weight, group_size: int, eps: float = 1e-5, out=None,
+                      out_dtype=None, stream=None):
+    """out = (y * silu(z)) / rms over groups of group_size channels * weight.
+    y, z : [rows, dim] (or any shape whose last axis is dim); weight [dim] fp32.
+    out may be y itself.  Returns out."""
+    _dev(y, "y")
+    _dev(z, "z")
+    _dev(weight, "weight", torch.float32)
+    dim = y.shape[-1]
+    rows = y.numel() // dim if dim else 0
+    if out is None:
+        out = torch.empty(y.shape, dtype=out_dtype or y.dtype, device=y.device)
+    _dev(out, "out")
+    st = lib.ssm_gated_rmsnorm(rows, dim, int(group_size), _dtype_code(y.dtype), _ptr(y),
+                               _dtype_code(z.dtype), _ptr(z), _ptr(weight), float(eps),
+                               _dtype_code(out.dtype), _ptr(out), _stream(stream))
+    _check(st, "ssm_gated_rmsnorm")
+    return out

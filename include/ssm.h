@@ -67,6 +67,24 @@ typedef enum {
     SSM_BF16 = 1
 } ssm_dtype;
 
+/*
+ * Optional transform of dt inside the kernels that read it, so that the raw
+ * dt of the input projection can be passed (the dt_bias input of the
+ * TensorRT MambaPlugin, deep-research note section "TensorRT Plugin 做
+ * selective state update"; softplus and the time-step clamp of the Mamba-2
+ * mixer).  Per (token, head h):
+ *     v = dt + dt_bias[h]          (dt_bias: device fp32 [nheads], or NULL)
+ *     v = log(1 + e^v)             (if softplus; v itself above 20)
+ *     v = min(max(v, dt_min), dt_max)   (if clamp; dt_min <= dt_max)
+ * A NULL ssm_dt_params pointer means dt is already final.
+ */
+typedef struct {
+    const float *dt_bias;
+    int softplus;
+    int clamp;
+    float dt_min, dt_max;
+} ssm_dt_params;
+
 /* Human-readable name of a status code (static string, never NULL). */
 SSM_API const char *ssm_status_string(int status);
 
@@ -173,9 +191,11 @@ SSM_API int ssm_state_update(int batch, int nheads, int head_dim, int d_state,
  *                      be distinct; an index outside [0, max_slots) skips that
  *                      sequence (no output written) and sets
  *                      SSM_ERR_DEVICE_INPUT in *status_dev.
+ *                      NULL: sequence s uses row s (max_slots >= nseq).
  *   has_initial_state  device int32 [nseq] or NULL (all true): 0 starts the
  *                      sequence from a zero state (a freshly claimed slot)
  *                      instead of the slot's contents.
+ *   dt_params          optional dt transform (see ssm_dt_params), or NULL.
  * Every other argument is as for ssd_chunk_scan.  A zero-length sequence
  * leaves its slot unchanged, or zeroes it when it has no initial state.  The
  * pool must not overlap any input or y.
@@ -185,6 +205,7 @@ SSM_API int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens
                                  int chunk_size, int in_dtype,
                                  const void *x, const float *dt, const float *A,
                                  const void *B, const void *C, const float *D,
+                                 const ssm_dt_params *dt_params,
                                  float *state_pool, int max_slots, const int32_t *slot_idx,
                                  const int32_t *has_initial_state,
                                  int y_dtype, void *y, int *status_dev, cudaStream_t stream);
@@ -194,14 +215,16 @@ SSM_API int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens
  * state_pool[slot_idx[b]] in place.  A negative slot index marks a padding row
  * (no state update, y not written); an index >= max_slots skips the row and
  * sets SSM_ERR_DEVICE_INPUT in *status_dev (status_dev may be NULL).  Slot
- * indices of non-padding rows must be distinct.  Other arguments as for
- * ssm_state_update.
+ * indices of non-padding rows must be distinct; slot_idx NULL means row b
+ * (max_slots >= batch).  dt_params: optional dt transform, or NULL.  Other
+ * arguments as for ssm_state_update.
  */
 SSM_API int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
                                    int ngroups, int in_dtype, float *state_pool, int max_slots,
                                    const int32_t *slot_idx,
                                    const void *x, const float *dt, const float *A,
                                    const void *B, const void *C, const float *D,
+                                   const ssm_dt_params *dt_params,
                                    int y_dtype, void *y, int *status_dev, cudaStream_t stream);
 
 /*
@@ -299,6 +322,7 @@ SSM_API int causal_conv1d_update(int batch, int dim, int width, int in_dtype, co
  *                 state is only read.
  *   slot_idx / max_slots  as for ssm_state_update_slots (negative = padding);
  *                 NULL / 0 when the state has one row per batch row.
+ *   dt_params     optional dt transform (see ssm_dt_params), or NULL.
  * At least one of y, inter_states, accept_len must be given.  No output may
  * overlap an input or another output.
  */
@@ -306,7 +330,8 @@ SSM_API int ssm_state_update_multi(int batch, int ntok, int nheads, int head_dim
                                    int ngroups, int in_dtype, float *state, int max_slots,
                                    const int32_t *slot_idx, const void *x, const float *dt,
                                    const float *A, const void *B, const void *C,
-                                   const float *D, const int32_t *accept_len,
+                                   const float *D, const ssm_dt_params *dt_params,
+                                   const int32_t *accept_len,
                                    float *inter_states, int y_dtype, void *y,
                                    int *status_dev, cudaStream_t stream);
 
@@ -335,6 +360,25 @@ SSM_API int causal_conv1d_update_multi(int batch, int ntok, int dim, int width, 
                                        const int32_t *slot_idx, const int32_t *accept_len,
                                        int y_dtype, void *y, int *status_dev,
                                        cudaStream_t stream);
+
+/*
+ * ssm_gated_rmsnorm -- the gated group RMSNorm after the scan, gate first
+ * (norm_before_gate = False: the _gated_group_rmsnorm kernel of the MAX
+ * nemotron_h article, section 5.4 item 4).  For each row and each group of
+ * group_size consecutive channels:
+ *     g = y * silu(z),   out = g / sqrt(mean over the group of g^2 + eps) * weight
+ * computed in fp32.
+ *   y    [rows][dim], y_dtype (the scan output viewed as [T][nheads*head_dim])
+ *   z    [rows][dim], z_dtype (the gate from the input projection)
+ *   weight  device fp32 [dim];  eps >= 0
+ *   out  [rows][dim], out_dtype; may be y itself (same dtype), must not
+ *        overlap z or weight otherwise
+ * dim must be a multiple of group_size; group_size a multiple of 256, at most
+ * 8192 (SSM_ERR_UNSUPPORTED otherwise).  One launch on `stream`.
+ */
+SSM_API int ssm_gated_rmsnorm(int rows, int dim, int group_size, int y_dtype, const void *y,
+                              int z_dtype, const void *z, const float *weight, float eps,
+                              int out_dtype, void *out, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -137,26 +137,33 @@ def test_update_batch_zero_is_noop(lib):
 def slib(lib):
     vp, i = ctypes.c_void_p, ctypes.c_int
     lib.ssd_chunk_scan_slots.restype = i
-    lib.ssd_chunk_scan_slots.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp,
+    lib.ssd_chunk_scan_slots.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp,
                                          vp, i, vp, vp, i, vp, vp, vp]
     lib.ssm_state_update_slots.restype = i
     lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp, vp,
-                                           i, vp, vp, vp]
+                                           vp, i, vp, vp, vp]
     return lib
 
 
 def scan_slots(lib, nseq=2, seqlen=128, H=4, P=64, N=128, G=1, pool=0x200000, max_slots=8,
-               slots=0x300000, has=None, x=A16, y=0x60000):
+               slots=0x300000, has=None, x=A16, y=0x60000, dtp=None):
     return lib.ssd_chunk_scan_slots(nseq, seqlen, None, H, P, N, G, 128, BF16, x, A16b, A16c,
-                                    0x40000, 0x50000, None, pool, max_slots, slots, has, BF16,
-                                    y, None, None)
+                                    0x40000, 0x50000, None, dtp, pool, max_slots, slots, has,
+                                    BF16, y, None, None)
+
+
+class DtParams(ctypes.Structure):
+    _fields_ = [("dt_bias", ctypes.c_void_p), ("softplus", ctypes.c_int), ("clamp", ctypes.c_int),
+                ("dt_min", ctypes.c_float), ("dt_max", ctypes.c_float)]
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(max_slots=0), INVALID),
     (dict(pool=None), INVALID),
-    (dict(slots=None), INVALID),
+    (dict(slots=None, max_slots=1), INVALID),   # no slot map: one row per sequence needed
     (dict(slots=0x300004), MISALIGNED),
+    (dict(dtp=ctypes.byref(DtParams(0x700004, 1, 0, 0.0, 0.0))), MISALIGNED),
+    (dict(dtp=ctypes.byref(DtParams(None, 1, 1, 0.5, 0.1))), INVALID),      # dt_min > dt_max
     (dict(y=0x200000 + 4096), INVALID),     # y inside the pool
     (dict(P=96), UNSUPPORTED),
 ])
@@ -169,14 +176,15 @@ def test_scan_slots_nseq_zero_is_noop(slib):
 
 
 def update_slots(lib, batch=2, H=4, P=64, N=128, G=2, pool=0x200000, max_slots=8,
-                 slots=0x300000, x=A16, y=0x60000):
+                 slots=0x300000, x=A16, y=0x60000, dtp=None):
     return lib.ssm_state_update_slots(batch, H, P, N, G, BF16, pool, max_slots, slots, x, A16b,
-                                      A16c, 0x40000, 0x50000, None, F32, y, None, None)
+                                      A16c, 0x40000, 0x50000, None, dtp, F32, y, None, None)
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(max_slots=-1), INVALID),
-    (dict(slots=None), INVALID),
+    (dict(slots=None, max_slots=1), INVALID),
+    (dict(dtp=ctypes.byref(DtParams(None, 0, 1, float("nan"), 1.0))), INVALID),
     (dict(x=None), INVALID),
     (dict(pool=0x200008), MISALIGNED),
     (dict(x=0x200000 + 512), INVALID),      # x inside the pool
@@ -255,7 +263,7 @@ def mlib(lib):
     vp, i = ctypes.c_void_p, ctypes.c_int
     lib.ssm_state_update_multi.restype = i
     lib.ssm_state_update_multi.argtypes = [i, i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp,
-                                           vp, vp, vp, i, vp, vp, vp]
+                                           vp, vp, vp, vp, i, vp, vp, vp]
     lib.ssm_state_commit.restype = i
     lib.ssm_state_commit.argtypes = [i, i, i, i, i, vp, vp, vp, i, vp, vp, vp]
     lib.causal_conv1d_update_multi.restype = i
@@ -267,8 +275,8 @@ def mlib(lib):
 def multi(lib, batch=2, ntok=3, H=4, P=64, N=128, G=2, state=0x1000000, max_slots=0, slots=None,
           x=0x100000, acc=None, inter=None, y=0x200000):
     return lib.ssm_state_update_multi(batch, ntok, H, P, N, G, BF16, state, max_slots, slots, x,
-                                      0x300000, 0x310000, 0x320000, 0x330000, None, acc, inter,
-                                      BF16, y, None, None)
+                                      0x300000, 0x310000, 0x320000, 0x330000, None, None, acc,
+                                      inter, BF16, y, None, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -318,3 +326,24 @@ def test_conv_multi_rejects(mlib, kw, code):
                                            args["width"], BF16, args["x"], 0x200000, None, 1,
                                            args["state"], 0, None, args["acc"], BF16, args["y"],
                                            None, None) == code
+
+
+def test_gated_rmsnorm_rejects(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.ssm_gated_rmsnorm.restype = i
+    lib.ssm_gated_rmsnorm.argtypes = [i, i, i, i, vp, i, vp, vp, ctypes.c_float, i, vp, vp]
+
+    def call(rows=4, dim=2048, gs=1024, y=0x100000, z=0x200000, w=0x300000, eps=1e-5,
+             out=0x400000, od=BF16):
+        return lib.ssm_gated_rmsnorm(rows, dim, gs, BF16, y, BF16, z, w, eps, od, out, None)
+
+    assert call(gs=1000) == INVALID              # dim not a multiple of the group
+    assert call(dim=2000, gs=1000) == UNSUPPORTED  # group not whole warps of 8-channel threads
+    assert call(gs=16384, dim=16384) == UNSUPPORTED
+    assert call(eps=-1.0) == INVALID
+    assert call(z=None) == INVALID
+    assert call(out=0x400008) == MISALIGNED
+    assert call(out=0x100010) == INVALID          # out partly overlaps y
+    assert call(out=0x200000 + 64) == INVALID    # out overlaps z
+    assert call(out=0x100000 + 2, od=BF16) == MISALIGNED
+    assert call(rows=0, y=None, z=None, w=None, out=None) == OK
