@@ -75,6 +75,14 @@ def _load():
             lib.oracle_causal_conv1d.argtypes = [
                 ctypes.c_int, _i64p, ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, ctypes.c_int,
                 _dp, _dp]
+            u32p = ctypes.POINTER(ctypes.c_uint32)
+            lib.oracle_philox4x32.restype = None
+            lib.oracle_philox4x32.argtypes = [u32p, u32p, ctypes.c_int, u32p]
+            lib.oracle_sr_fp16.restype = ctypes.c_double
+            lib.oracle_sr_fp16.argtypes = [ctypes.c_float, ctypes.c_uint32]
+            lib.oracle_round_state_f16.restype = None
+            lib.oracle_round_state_f16.argtypes = [ctypes.c_long, _dp, _i64p, ctypes.c_uint64,
+                                                   ctypes.c_uint64, ctypes.c_int, _dp]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -349,3 +357,60 @@ def gated_rmsnorm(y, z, weight, group_size, eps=1e-5):
     ms = np.mean(gg * gg, axis=-1, keepdims=True)
     out = (gg / np.sqrt(ms + eps)).reshape(rows, dim) * wf
     return out
+
+
+def philox4x32(counter, key, rounds=10):
+    """Philox-4x32 of one 4-word counter under a 2-word key -> 4 words."""
+    u32 = ctypes.c_uint32
+    c = (u32 * 4)(*[int(v) & 0xFFFFFFFF for v in counter])
+    k = (u32 * 2)(*[int(v) & 0xFFFFFFFF for v in key])
+    out = (u32 * 4)()
+    _load().oracle_philox4x32(c, k, int(rounds), out)
+    return [int(v) for v in out]
+
+
+def sr_fp16(v, r):
+    """Stochastic rounding of the fp32 value v to fp16 with random word r."""
+    return _load().oracle_sr_fp16(float(np.float32(v)), int(r) & 0xFFFFFFFF)
+
+
+def round_state_f16(values, elem_index, seed, offset, rounds=10):
+    """fp16 values (as fp64) a pool stores for state values written at pool
+    elements elem_index, under stochastic rounding with (seed, offset)."""
+    v = _f64(values).ravel()
+    e = np.ascontiguousarray(np.asarray(elem_index, dtype=np.int64).ravel())
+    out = np.empty_like(v)
+    _load().oracle_round_state_f16(v.size, _ptr(v), e.ctypes.data_as(_i64p), int(seed),
+                                   int(offset), int(rounds), _ptr(out))
+    return out.reshape(np.shape(values))
+
+
+def round_state_f16_nearest(values):
+    """fp16 values (as fp64) of state values rounded to fp32 then to the
+    nearest fp16 (ties to even)."""
+    return _f64(values).astype(np.float32).astype(np.float16).astype(np.float64)
+
+
+def state_update_slots_f16(pool16, slot_idx, x, dt, A, B, C, D=None, rounding=None):
+    """One decode step on an fp16 pool: rows are read as fp16, updated in fp64
+    (state_update), and written back rounded to fp16 -- stochastically with
+    rounding = (seed, offset[, rounds]), else to nearest.  Padding rows
+    (slot < 0) are skipped.  Returns (y, new_pool), fp64."""
+    pool = np.asarray(pool16, dtype=np.float16).astype(np.float64)
+    slots = np.asarray(slot_idx, dtype=np.int64)
+    live = slots >= 0
+    batch = slots.shape[0]
+    H, P, N = pool.shape[1:]
+    y = np.full((batch, H, P), np.nan)
+    out = pool.copy()
+    if live.any():
+        yl, st = state_update(pool[slots[live]], _f64(x)[live], _f64(dt)[live], A,
+                              _f64(B)[live], _f64(C)[live], D)
+        y[live] = yl
+        if rounding is None:
+            out[slots[live]] = round_state_f16_nearest(st)
+        else:
+            row = H * P * N
+            idx = slots[live][:, None] * row + np.arange(row)[None, :]
+            out[slots[live]] = round_state_f16(st.reshape(-1, row), idx, *rounding).reshape(st.shape)
+    return y, out

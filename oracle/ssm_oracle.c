@@ -224,3 +224,81 @@ int oracle_causal_conv1d(int nseq, const int64_t *cu_seqlens, int dim, int K,
     }
     return ORACLE_OK;
 }
+
+/*
+ * Philox-4x32 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+ * as 1, 2, 3", SC'11), written from the paper's description: `rounds` rounds
+ * of the 4x32 S-box -- the two 32x32 -> 64-bit products of counter words 0
+ * and 2 with the multipliers 0xD2511F53 and 0xCD9E8D57, whose high halves are
+ * xored with counter words 1 and 3 and the two key words -- with the key
+ * bumped by the Weyl constants 0x9E3779B9 and 0xBB67AE85 after each round.
+ */
+void oracle_philox4x32(const uint32_t ctr[4], const uint32_t key[2], int rounds, uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < rounds; ++r) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n1 = (uint32_t)p1;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        const uint32_t n3 = (uint32_t)p0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/*
+ * Stochastic rounding of an fp32 value to fp16, from its definition: with
+ * lo the fp16 neighbour toward zero and s the fp16 spacing there (2^(k-10) in
+ * the binade [2^k, 2^(k+1)) of the normal range, 2^-24 below 2^-14), the
+ * fraction f = (|v| - lo) / s is in [0, 1); the result moves to lo + s iff
+ * u < f with u = (r >> 8) / 2^24.  |v| >= 65504 gives +-65504.
+ */
+double oracle_sr_fp16(float vf, uint32_t r)
+{
+    const double v = vf;
+    if (v != v) return v;
+    const double a = fabs(v);
+    if (a >= 65504.0) return copysign(65504.0, v);
+    double s;
+    if (a >= ldexp(1.0, -14)) {
+        int e;
+        frexp(a, &e);                 /* a in [2^(e-1), 2^e) */
+        s = ldexp(1.0, e - 1 - 10);
+    } else {
+        s = ldexp(1.0, -24);
+    }
+    const double lo = floor(a / s) * s;
+    const double f = (a - lo) / s;
+    const double u = (double)(r >> 8) / 16777216.0;
+    double m = lo + (u < f ? s : 0.0);
+    if (m > 65504.0) m = 65504.0;
+    return copysign(m, v);
+}
+
+/*
+ * Round n state values to fp16 as they are written to a pool: value i is
+ * pool element e0 + i; its random word is word (e % 4) of Philox(counter =
+ * (e / 4 low, e / 4 high, offset low, offset high), key = (seed low, seed
+ * high)).  The decision is taken on the value rounded to fp32 (the precision
+ * the state is computed in).
+ */
+void oracle_round_state_f16(long n, const double *v, const int64_t *elem, uint64_t seed,
+                            uint64_t offset, int rounds, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (long i = 0; i < n; ++i) {
+        const uint64_t e = (uint64_t)elem[i];
+        const uint64_t q = e >> 2;
+        const uint32_t ctr[4] = {(uint32_t)q, (uint32_t)(q >> 32), (uint32_t)offset,
+                                 (uint32_t)(offset >> 32)};
+        const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+        uint32_t w[4];
+        oracle_philox4x32(ctr, key, rounds, w);
+        out[i] = oracle_sr_fp16((float)v[i], w[e & 3]);
+    }
+}

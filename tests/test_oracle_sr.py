@@ -1,0 +1,83 @@
+"""Pins of the oracle's Philox-4x32 generator and fp16 stochastic rounding:
+Philox-4x32-10 against cuRAND's host Philox generator (a library routine,
+run on the CPU); stochastic rounding against numpy's fp16 neighbours and its
+defining property, an exact mean over the random word."""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+CURAND = "/usr/local/cuda/lib64/libcurand.so"
+
+
+def _curand_words(seed, n, offset=0):
+    lib = ctypes.CDLL(CURAND)
+    gen = ctypes.c_void_p()
+    assert lib.curandCreateGeneratorHost(ctypes.byref(gen), 161) == 0   # PHILOX4_32_10
+    assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+    assert lib.curandSetGeneratorOffset(gen, ctypes.c_ulonglong(offset)) == 0
+    buf = (ctypes.c_uint32 * n)()
+    assert lib.curandGenerate(gen, buf, ctypes.c_size_t(n)) == 0
+    lib.curandDestroyGenerator(gen)
+    return list(buf)
+
+
+@pytest.mark.skipif(not os.path.exists(CURAND), reason="cuRAND host library not present")
+@pytest.mark.parametrize("seed", [0, 12345, 0xDEADBEEFCAFEF00D])
+def test_philox_matches_curand_host_generator(seed):
+    # The host generator lays its output out as 65536 interleaved streams:
+    # 4-word block b is Philox(counter = (b // 65536, 0, b % 65536, 0), key = seed).
+    words = _curand_words(seed, 4 * (65536 + 8))
+    key = (seed & 0xFFFFFFFF, seed >> 32)
+    for b in list(range(16)) + list(range(65536, 65536 + 8)):
+        got = oracle.philox4x32((b // 65536, 0, b % 65536, 0), key, 10)
+        assert got == words[4 * b:4 * b + 4], b
+
+
+def _fp16_bracket(v):
+    """The fp16 values toward and away from zero around the fp32 value v."""
+    f = np.float16(v)
+    if float(f) == float(np.float32(v)):
+        return float(f), float(f)
+    away = np.float16(np.inf) if v > 0 else np.float16(-np.inf)
+    a = np.nextafter(f, np.float16(0.0) if abs(float(f)) > abs(float(np.float32(v))) else away)
+    lo, hi = sorted([float(f), float(a)], key=abs)
+    return lo, hi
+
+
+def test_sr_returns_a_neighbour_and_keeps_exact_values():
+    rng = np.random.default_rng(5)
+    vals = np.concatenate([rng.standard_normal(200).astype(np.float32),
+                           (rng.standard_normal(50) * 1e-6).astype(np.float32),
+                           np.float16(rng.standard_normal(50)).astype(np.float32)])
+    rs = rng.integers(0, 2**32, len(vals))
+    for v, r in zip(vals, rs):
+        got = oracle.sr_fp16(v, r)
+        lo, hi = _fp16_bracket(v)
+        assert got in (lo, hi), (v, got, lo, hi)
+        if lo == hi:
+            assert got == lo
+    assert oracle.sr_fp16(70000.0, 0) == 65504.0
+    assert oracle.sr_fp16(-1e9, 123) == -65504.0
+
+
+@pytest.mark.parametrize("v", [1.0 + 3 * 2.0**-20, -0.3337, 1234.567, 3.1e-6, -5.9e-8])
+def test_sr_mean_over_the_random_word_is_exact(v):
+    v = float(np.float32(v))
+    # u = (r >> 8) / 2^24 takes every value k / 2^24 once over r = k << 8
+    if abs(v) >= 2.0**-14:
+        ks = np.arange(0, 1 << 13) << 11        # normal range: 13 bits decide
+        scale = 1 << 13
+    else:
+        ks = np.arange(0, 1 << 24)[::64]        # a spacing below fp32 resolution; sample
+        scale = None
+    vals = np.array([oracle.sr_fp16(v, int(k) << 8) for k in ks]) if scale else None
+    if scale:
+        assert vals.mean() == pytest.approx(v, rel=0, abs=0)
+    else:
+        vals = oracle.round_state_f16(np.full(len(ks), v), np.zeros(len(ks), np.int64), 0, 0)
+        lo, hi = _fp16_bracket(v)
+        assert set(np.unique(vals)) <= {lo, hi}
