@@ -491,6 +491,55 @@ def time_fused(dev, stream, seed, iters=20):
     return out
 
 
+def time_f16_decode(dev, stream, seed, iters=20):
+    """Device time of the Ultra decode step on an fp16 state pool, written back
+    with stochastic rounding (Philox-4x32 with 5 and with 10 rounds) and with
+    round-to-nearest.  Bytes: the fp16 state read and written, plus the
+    step's inputs and bf16 y."""
+    import torch
+    from hybrid_mamba_ssm_b200 import inputs as synth
+    from hybrid_mamba_ssm_b200 import ssm
+
+    d = DECODE
+    b, H, P, N, G = d["batch"], d["H"], d["P"], d["N"], d["G"]
+    A, D = synth.make_head_params(seed, H)
+    A, D = torch.from_numpy(A).to(dev), torch.from_numpy(D).to(dev)
+    pool = torch.from_numpy(synth.make_state(seed + 1, (b, H, P, N))).to(dev).half()
+    st = synth.make_decode_step(seed + 2, b, H, P, N, G)
+    bf = lambda t: torch.from_numpy(np.ascontiguousarray(t.bits).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    x, B, C = bf(st.x), bf(st.B), bf(st.C)
+    dt = torch.from_numpy(st.dt).to(dev)
+    y = torch.empty((b, H, P), dtype=torch.bfloat16, device=dev)
+    _, full_bytes, _ = decode_work()
+    nbytes = full_bytes - b * H * P * N * 4          # fp16 instead of fp32 state
+    out = {}
+    for name, rnd in (("decode_f16_sr_philox5", (7, 0, 5)), ("decode_f16_sr_philox10", (7, 0, 10)),
+                      ("decode_f16_nearest", None)):
+        calls = [0]
+
+        def call():
+            calls[0] += 1
+            r = None if rnd is None else (rnd[0], calls[0], rnd[2])   # fresh offset per step
+            ssm.ssm_state_update_slots(pool, None, x, dt, A, B, C, D, y=y, stream=stream,
+                                       rounding=r)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(iters)]
+        for e0, e1 in ev:
+            e0.record(stream)
+            call()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
+        out[name] = {"ms": ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "bytes_per_launch": nbytes,
+                     "launches": iters, "state": "fp16 [64,256,64,128]"}
+    return out
+
+
 def run_reference(args, world, rank, pg):
     if rank != 0:
         return 0
@@ -677,6 +726,7 @@ def run_ours(args, world, rank, local, pg):
     conv = time_conv(dev, stream, seed + 17)
     conv.update(time_mtp(dev, stream, seed + 29))
     conv.update(time_fused(dev, stream, seed + 41))
+    conv.update(time_f16_decode(dev, stream, seed + 53))
 
     # ---- numbers ----
     peaks, peak_kind = load_peaks()

@@ -52,6 +52,26 @@ int read_dt_params(const ssm_dt_params *p, ssm::DtParams &out)
     return SSM_OK;
 }
 
+// Storage of a state pool: fp32, or fp16 with round-to-nearest (rounding
+// NULL) or stochastic rounding.
+int read_state_format(int state_dtype, const ssm_rounding *r, ssm::RoundParams &out)
+{
+    out = ssm::RoundParams{};
+    if (state_dtype == SSM_F32) return SSM_OK;
+    if (state_dtype != SSM_F16) return SSM_ERR_INVALID_ARG;
+    out.f16 = 1;
+    if (r) {
+        if (r->philox_rounds < 1 || r->philox_rounds > 16) return SSM_ERR_INVALID_ARG;
+        out.stochastic = 1;
+        out.key0 = (uint32_t)r->seed;
+        out.key1 = (uint32_t)(r->seed >> 32);
+        out.off0 = (uint32_t)r->offset;
+        out.off1 = (uint32_t)(r->offset >> 32);
+        out.rounds = r->philox_rounds;
+    }
+    return SSM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -151,7 +171,8 @@ int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
                          const void *x, const float *dt, const float *A,
                          const void *B, const void *C, const float *D,
                          const ssm_dt_params *dt_params,
-                         float *state_pool, int max_slots, const int32_t *slot_idx,
+                         void *state_pool, int state_dtype, const ssm_rounding *rounding,
+                         int max_slots, const int32_t *slot_idx,
                          const int32_t *has_initial_state,
                          int y_dtype, void *y, int *status_dev, cudaStream_t stream)
 {
@@ -165,6 +186,9 @@ int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
     if (!slot_idx && max_slots < nseq) return SSM_ERR_INVALID_ARG;   // row s per sequence
     ssm::DtParams dtp;
     if (const int st = read_dt_params(dt_params, dtp)) return st;
+    ssm::RoundParams rp;
+    if (const int st = read_state_format(state_dtype, rounding, rp)) return st;
+    const size_t sz_state = rp.f16 ? 2 : 4;
     const long long T = cu_seqlens ? (long long)seqlen : (long long)nseq * seqlen;
     if (T > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
     if (T > 0 && (!x || !dt || !B || !C || !y)) return SSM_ERR_INVALID_ARG;
@@ -173,7 +197,7 @@ int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
     const size_t es = dtype_size(in_dtype);
-    const Range rpool = range_of(state_pool, (size_t)max_slots * nheads * head_dim * d_state * sizeof(float));
+    const Range rpool = range_of(state_pool, (size_t)max_slots * nheads * head_dim * d_state * sz_state);
     const Range ry = range_of(y, (size_t)T * nheads * head_dim * dtype_size(y_dtype));
     const Range ins[] = {range_of(x, (size_t)T * nheads * head_dim * es),
                          range_of(dt, (size_t)T * nheads * sizeof(float)),
@@ -199,6 +223,7 @@ int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens,
     a.status_dev = status_dev;
     a.slot_idx = slot_idx; a.has_initial = has_initial_state; a.max_slots = max_slots;
     a.dtp = dtp;
+    a.rp = rp;
     // empty sequences still run: a slot without an initial state is reset to zero
     const cudaError_t e = ssm::scan_tc_supports(a) ? ssm::launch_scan_tc(a, stream)
                                                    : ssm::launch_scan_simt(a, stream);
@@ -245,7 +270,8 @@ int ssm_state_update(int batch, int nheads, int head_dim, int d_state,
 }
 
 int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
-                           int ngroups, int in_dtype, float *state_pool, int max_slots,
+                           int ngroups, int in_dtype, void *state_pool, int state_dtype,
+                           const ssm_rounding *rounding, int max_slots,
                            const int32_t *slot_idx,
                            const void *x, const float *dt, const float *A,
                            const void *B, const void *C, const float *D,
@@ -263,11 +289,13 @@ int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
     if (!slot_idx && max_slots < batch) return SSM_ERR_INVALID_ARG;   // row b per batch row
     ssm::DtParams dtp;
     if (const int st = read_dt_params(dt_params, dtp)) return st;
+    ssm::RoundParams rp;
+    if (const int st = read_state_format(state_dtype, rounding, rp)) return st;
     const void *ptrs[] = {state_pool, slot_idx, x, dt, A, B, C, D, y, status_dev};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return SSM_ERR_MISALIGNED;
     const size_t es = dtype_size(in_dtype);
-    const Range rs = range_of(state_pool, (size_t)max_slots * nheads * head_dim * d_state * sizeof(float));
+    const Range rs = range_of(state_pool, (size_t)max_slots * nheads * head_dim * d_state * (rp.f16 ? 2 : 4));
     const Range ry = range_of(y, (size_t)batch * nheads * head_dim * dtype_size(y_dtype));
     const Range ins[] = {range_of(x, (size_t)batch * nheads * head_dim * es),
                          range_of(dt, (size_t)batch * nheads * sizeof(float)),
@@ -287,6 +315,7 @@ int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
     a.state = state_pool; a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.y = y;
     a.slot_idx = slot_idx; a.max_slots = max_slots; a.status_dev = status_dev;
     a.dtp = dtp;
+    a.rp = rp;
     return ssm::launch_state_update(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

@@ -101,7 +101,7 @@ scan_simt_kernel(ScanArgs a)
 
     for (int i = tid; i < P * N; i += kSimtThreads) {
         const int p = i / N, n = i - p * N;
-        Hs[p * N1 + n] = load_init ? a.initial_state[state_off + i] : 0.f;
+        Hs[p * N1 + n] = load_init ? state_load1(a.initial_state, state_off + i, a.rp) : 0.f;
     }
 
     for (long c0 = t0; c0 < t1; c0 += Q) {
@@ -188,7 +188,7 @@ scan_simt_kernel(ScanArgs a)
     if (a.final_state) {
         for (int i = tid; i < P * N; i += kSimtThreads) {
             const int p = i / N, n = i - p * N;
-            a.final_state[state_off + i] = Hs[p * N1 + n];
+            state_store1(a.final_state, state_off + i, Hs[p * N1 + n], a.rp);
         }
     }
 }

@@ -474,7 +474,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         float Hs[32];
 #pragma unroll
         for (int p = 0; p < 32; ++p)
-            Hs[p] = load_init ? a.initial_state[state_off + (size_t)p * kN] : 0.f;
+            Hs[p] = load_init ? state_load1(a.initial_state, state_off + (size_t)p * kN, a.rp) : 0.f;
         write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
 
         const float Ah = a.A[hh];
@@ -583,7 +583,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         }
         if (a.final_state) {
 #pragma unroll
-            for (int p = 0; p < 32; ++p) a.final_state[state_off + (size_t)p * kN] = Hs[p];
+            for (int p = 0; p < 32; ++p) state_store1(a.final_state, state_off + (size_t)p * kN, Hs[p], a.rp);
         }
     }
     tc::tc_fence_before();

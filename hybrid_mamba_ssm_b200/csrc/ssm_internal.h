@@ -13,7 +13,7 @@ namespace ssm {
 struct StateUpdateArgs {
     int batch, nheads, head_dim, d_state, ngroups;
     int in_dtype, y_dtype;        // 0 = fp32, 1 = bf16
-    float *state;
+    void *state;                  // fp32, or fp16 when rp.f16
     const void *x;
     const float *dt, *A;
     const void *B, *C;
@@ -24,6 +24,7 @@ struct StateUpdateArgs {
     int max_slots;
     int *status_dev;
     DtParams dtp;                 // transform of dt (identity when all off)
+    RoundParams rp;               // state storage (fp32, or fp16 and its rounding)
 };
 
 // Speculative (multi-token) decode: ntok draft tokens per batch row, in
@@ -65,9 +66,9 @@ struct ScanArgs {
     const float *dt, *A;
     const void *B, *C;
     const float *D;
-    const float *initial_state;   // nullptr = zero
+    const void *initial_state;    // nullptr = zero; fp32, or fp16 when rp.f16
     void *y;
-    float *final_state;           // nullptr = not written
+    void *final_state;            // nullptr = not written; same storage type
     int *status_dev;              // nullptr = not reported
     // slot-indexed state pool: sequence s reads and writes state row
     // slot_idx[s] of initial_state / final_state (the same pool); nullptr
@@ -76,6 +77,7 @@ struct ScanArgs {
     const int32_t *has_initial;
     int max_slots;
     DtParams dtp;
+    RoundParams rp;
 };
 
 // Causal depthwise conv1d (prefill over packed sequences, or one decode token

@@ -118,12 +118,128 @@ state_update_kernel(int nheads, int head_dim, int heads_per_group, int ngroups,
     }
 }
 
+// fp16 state pool: the state is read as fp16, updated in fp32 and rounded
+// back (nearest even, or stochastically with 16 Philox bits per element).
+// Each lane owns 8 adjacent d_state elements of a row (one 16-byte load and
+// store, one Philox call), so a warp covers 32 / (d_state / 8) rows per step
+// and a CTA has its whole 64 x 128 fp16 slice (16 KB) in flight at once.
+constexpr int kF16Unroll = 4;
+
+template <int N, typename TIn, typename TOut>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+state_update_f16_kernel(int nheads, int head_dim, int heads_per_group, int ngroups,
+                        __half *__restrict__ state, const TIn *__restrict__ x,
+                        const float *__restrict__ dt, const float *__restrict__ A,
+                        const TIn *__restrict__ B, const TIn *__restrict__ C,
+                        const float *__restrict__ D, TOut *__restrict__ y,
+                        const int32_t *__restrict__ slot_idx, int max_slots, int *status,
+                        DtParams dtp, RoundParams rp)
+{
+    constexpr int LPR = (N / 8 < 32) ? N / 8 : 32;   // lanes per state row
+    constexpr int RPW = 32 / LPR;                    // rows per warp step
+    constexpr int ROWS_PER_PASS = kDecodeWarps * RPW * kF16Unroll;
+    static_assert(N == 8 * LPR, "one 8-element vector per lane");
+
+    const int bh = blockIdx.x;
+    const int b = bh / nheads;
+    const int h = bh - b * nheads;
+    const int g = h / heads_per_group;
+    size_t srow = (size_t)b;
+    if (slot_idx) {
+        const int slot = __ldg(slot_idx + b);
+        if (slot < 0) return;
+        if (slot >= max_slots) {
+            if (threadIdx.x == 0) report_status(status, 6);
+            return;
+        }
+        srow = (size_t)slot;
+    }
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int li = lane % LPR;
+    const int ri = lane / LPR;
+    const float dtv = dt_apply(dtp, __ldg(dt + bh), h);
+    const float decay = expf(dtv * __ldg(A + h));
+    const float Dh = D ? __ldg(D + h) : 0.f;
+    float bv[8], cv[8];
+    {
+        const float4 b0 = load4(B + ((size_t)b * ngroups + g) * N + li * 8);
+        const float4 b1 = load4(B + ((size_t)b * ngroups + g) * N + li * 8 + 4);
+        const float4 c0 = load4(C + ((size_t)b * ngroups + g) * N + li * 8);
+        const float4 c1 = load4(C + ((size_t)b * ngroups + g) * N + li * 8 + 4);
+        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { bv[j] = bb[j]; cv[j] = cc[j]; }
+    }
+    const size_t st0 = (srow * nheads + h) * (size_t)head_dim * N;   // element index of the slice
+    __half *st = state + st0;
+    const TIn *xp = x + (size_t)bh * head_dim;
+    TOut *yp = y + (size_t)bh * head_dim;
+
+    for (int base = 0; base < head_dim; base += ROWS_PER_PASS) {
+        uint4 raw[kF16Unroll];
+#pragma unroll
+        for (int k = 0; k < kF16Unroll; ++k) {
+            const int r = base + (k * kDecodeWarps + warp) * RPW + ri;
+            raw[k] = (r < head_dim) ? __ldcs(reinterpret_cast<const uint4 *>(st + (size_t)r * N + li * 8))
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < kF16Unroll; ++k) {
+            const int r = base + (k * kDecodeWarps + warp) * RPW + ri;
+            const float xr = (r < head_dim) ? load_f32(xp + r) : 0.f;
+            const float dtx = dtv * xr;
+            const __half2 *hv = reinterpret_cast<const __half2 *>(&raw[k]);
+            float q[8];
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __half22float2(hv[j]);
+                q[2 * j] = fmaf(f.x, decay, dtx * bv[2 * j]);
+                q[2 * j + 1] = fmaf(f.y, decay, dtx * bv[2 * j + 1]);
+                acc = fmaf(q[2 * j], cv[2 * j], acc);
+                acc = fmaf(q[2 * j + 1], cv[2 * j + 1], acc);
+            }
+            if (r < head_dim) {
+                const size_t off = (size_t)r * N + li * 8;
+                uint32_t w[4] = {0u, 0u, 0u, 0u};
+                if (rp.stochastic) {
+                    const uint4 rnd = state_random8(rp, st0 + off);
+                    w[0] = rnd.x; w[1] = rnd.y; w[2] = rnd.z; w[3] = rnd.w;
+                }
+                uint32_t packed[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const __half2 hh = __halves2half2(state_to_half(rp, q[2 * j], w[j] & 0xFFFFu),
+                                                      state_to_half(rp, q[2 * j + 1], w[j] >> 16));
+                    packed[j] = *reinterpret_cast<const uint32_t *>(&hh);
+                }
+                __stcs(reinterpret_cast<uint4 *>(st + off),
+                       make_uint4(packed[0], packed[1], packed[2], packed[3]));
+            }
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1)
+                acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (li == 0 && r < head_dim) store_out(yp + r, fmaf(Dh, xr, acc));
+        }
+    }
+}
+
 template <int N, typename TIn, typename TOut>
 static cudaError_t launch_state_update_t(const StateUpdateArgs &a, cudaStream_t stream)
 {
     dim3 grid((unsigned)((size_t)a.batch * a.nheads));
+    if (a.rp.f16) {
+        state_update_f16_kernel<N, TIn, TOut><<<grid, kDecodeWarps * 32, 0, stream>>>(
+            a.nheads, a.head_dim, a.nheads / a.ngroups, a.ngroups, static_cast<__half *>(a.state),
+            static_cast<const TIn *>(a.x), a.dt, a.A, static_cast<const TIn *>(a.B),
+            static_cast<const TIn *>(a.C), a.D, static_cast<TOut *>(a.y), a.slot_idx,
+            a.max_slots, a.status_dev, a.dtp, a.rp);
+        return cudaGetLastError();
+    }
     state_update_kernel<N, TIn, TOut><<<grid, kDecodeWarps * 32, 0, stream>>>(
-        a.nheads, a.head_dim, a.nheads / a.ngroups, a.ngroups, a.state,
+        a.nheads, a.head_dim, a.nheads / a.ngroups, a.ngroups, static_cast<float *>(a.state),
         static_cast<const TIn *>(a.x), a.dt, a.A, static_cast<const TIn *>(a.B),
         static_cast<const TIn *>(a.C), a.D, static_cast<TOut *>(a.y), a.slot_idx, a.max_slots,
         a.status_dev, a.dtp);

@@ -15,7 +15,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libssm.so")
 
-SSM_F32, SSM_BF16 = 0, 1
+SSM_F32, SSM_BF16, SSM_F16 = 0, 1, 2
 STATUS_NAMES = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED",
                 3: "SSM_ERR_MISALIGNED", 4: "SSM_ERR_CUDA", 5: "SSM_ERR_TIMEOUT",
                 6: "SSM_ERR_DEVICE_INPUT"}
@@ -43,10 +43,10 @@ def _load():
                                      vp, vp]
     lib.ssd_chunk_scan_slots.restype = i
     lib.ssd_chunk_scan_slots.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp,
-                                         vp, i, vp, vp, i, vp, vp, vp]
+                                         vp, i, vp, i, vp, vp, i, vp, vp, vp]
     lib.ssm_state_update_slots.restype = i
-    lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp, vp,
-                                           vp, i, vp, vp, vp]
+    lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, i, vp, vp, vp, vp, vp,
+                                           vp, vp, vp, i, vp, vp, vp]
     lib.causal_conv1d_fwd.restype = i
     lib.causal_conv1d_fwd.argtypes = [i, i, vp, i, i, i, vp, vp, vp, i, vp, i, vp, vp, i, vp,
                                       vp, vp]
@@ -86,6 +86,26 @@ def _dt_params(dt_bias, dt_softplus, dt_limit):
     p = DtParams(None if dt_bias is None else dt_bias.data_ptr(), int(bool(dt_softplus)),
                  int(dt_limit is not None), float(lo), float(hi))
     return ctypes.byref(p)
+
+
+class Rounding(ctypes.Structure):
+    """ssm_rounding: stochastic rounding of an fp16 state pool (Philox-4x32)."""
+    _fields_ = [("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64),
+                ("philox_rounds", ctypes.c_int)]
+
+
+def _state_format(pool, rounding):
+    """(state dtype code, ssm_rounding reference or None) of a state pool.
+    rounding: None (nearest even) or (seed, offset[, philox_rounds=10])."""
+    if pool.dtype == torch.float32:
+        return SSM_F32, None
+    if pool.dtype != torch.float16:
+        raise TypeError(f"state pool must be float32 or float16, got {pool.dtype}")
+    if rounding is None:
+        return SSM_F16, None
+    seed, offset = int(rounding[0]), int(rounding[1])
+    rounds = int(rounding[2]) if len(rounding) > 2 else 10
+    return SSM_F16, ctypes.byref(Rounding(seed, offset, rounds))
 
 
 class SSMError(RuntimeError):
@@ -216,7 +236,7 @@ def ssm_state_update(state, x, dt, A, B, C, D=None, y=None, y_dtype=None, stream
 def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_state=None,
                          cu_seqlens=None, chunk_size: int = 128, y=None, y_dtype=None,
                          status=None, stream=None, dt_bias=None, dt_softplus=False,
-                         dt_limit=None):
+                         dt_limit=None, rounding=None):
     """Chunked SSD prefill whose states live in a pool, updated in place.
 
     state_pool : [max_slots, H, P, N] fp32; sequence s starts from
@@ -226,6 +246,8 @@ def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_st
         sequence s uses row s).
     dt_bias [H] fp32, dt_softplus, dt_limit (lo, hi): transform the raw dt
         inside the kernel (dt <- clamp(softplus(dt + dt_bias))).
+    state_pool may be float16; rounding = (seed, offset[, philox_rounds])
+        then rounds the written states stochastically (None: nearest even).
     Other arguments as for ssd_chunk_scan.  Returns y.
     """
     _dev(x, "x")
@@ -244,7 +266,8 @@ def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_st
     _dev(B, "B", x.dtype)
     _dev(C, "C", x.dtype)
     _dev(D, "D", torch.float32)
-    _dev(state_pool, "state_pool", torch.float32)
+    _dev(state_pool, "state_pool")
+    sd, rnd = _state_format(state_pool, rounding)
     _dev(slot_idx, "slot_idx", torch.int32)
     _dev(has_initial_state, "has_initial_state", torch.int32)
     _dev(status, "status", torch.int32)
@@ -256,7 +279,7 @@ def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_st
     dtp = _dt_params(dt_bias, dt_softplus, dt_limit)
     st = lib.ssd_chunk_scan_slots(nseq, seqlen, _ptr(cu_seqlens), H, P, N, G, int(chunk_size),
                                   in_code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                                  dtp, _ptr(state_pool), state_pool.shape[0], _ptr(slot_idx),
+                                  dtp, _ptr(state_pool), sd, rnd, state_pool.shape[0], _ptr(slot_idx),
                                   _ptr(has_initial_state), _dtype_code(y.dtype), _ptr(y),
                                   _ptr(status), _stream(stream))
     _check(st, "ssd_chunk_scan_slots")
@@ -265,11 +288,14 @@ def ssd_chunk_scan_slots(x, dt, A, B, C, D, state_pool, slot_idx, has_initial_st
 
 def ssm_state_update_slots(state_pool, slot_idx, x, dt, A, B, C, D=None, y=None, y_dtype=None,
                            status=None, stream=None, dt_bias=None, dt_softplus=False,
-                           dt_limit=None):
+                           dt_limit=None, rounding=None):
     """One-token decode update of pool rows: batch row b updates
-    state_pool[slot_idx[b]] in place (slot_idx[b] < 0: padding row, skipped).
+    state_pool[slot_idx[b]] in place (slot_idx[b] < 0: padding row, skipped;
+    slot_idx None: row b).  state_pool may be float16, with rounding =
+    (seed, offset[, philox_rounds]) for stochastic rounding (None: nearest).
     Returns y [batch, H, P] (padding rows left as they were)."""
-    _dev(state_pool, "state_pool", torch.float32)
+    _dev(state_pool, "state_pool")
+    sd, rnd = _state_format(state_pool, rounding)
     _dev(slot_idx, "slot_idx", torch.int32)
     _dev(x, "x")
     in_code = _dtype_code(x.dtype)
@@ -288,7 +314,7 @@ def ssm_state_update_slots(state_pool, slot_idx, x, dt, A, B, C, D=None, y=None,
         y = torch.zeros((batch, H, P), dtype=y_dtype, device=x.device)
     _dev(y, "y", y_dtype)
     dtp = _dt_params(dt_bias, dt_softplus, dt_limit)
-    st = lib.ssm_state_update_slots(batch, H, P, N, G, in_code, _ptr(state_pool),
+    st = lib.ssm_state_update_slots(batch, H, P, N, G, in_code, _ptr(state_pool), sd, rnd,
                                     state_pool.shape[0], _ptr(slot_idx), _ptr(x), _ptr(dt),
                                     _ptr(A), _ptr(B), _ptr(C), _ptr(D), dtp, _dtype_code(y.dtype),
                                     _ptr(y), _ptr(status), _stream(stream))

@@ -64,7 +64,8 @@ typedef enum {
 
 typedef enum {
     SSM_F32 = 0,
-    SSM_BF16 = 1
+    SSM_BF16 = 1,
+    SSM_F16 = 2    /* state pools only (the *_slots entry points) */
 } ssm_dtype;
 
 /*
@@ -84,6 +85,26 @@ typedef struct {
     int clamp;
     float dt_min, dt_max;
 } ssm_dt_params;
+
+/*
+ * Stochastic rounding of an fp16 state pool (the float16 SSM cache with
+ * stochastic rounding and Philox rounds of the deployment flags listed in the
+ * modeling_nemotron_h.py walk-through, section "部署时如何调这些缓存").  The
+ * state is computed in fp32 and rounded to fp16 when it is written: a value
+ * moves to its fp16 neighbour away from zero iff u < frac, frac being its
+ * distance from the neighbour toward zero in units of the fp16 spacing there
+ * and u = (r >> 8) / 2^24 for a random word r; magnitudes beyond 65504
+ * saturate.  r for state element e (its index in the pool) is word e % 4 of
+ * Philox-4x32 with philox_rounds rounds (10 = the published Philox-4x32-10),
+ * key = seed, counter = (e / 4 as 64 bits, offset as 64 bits).  Callers pass
+ * a fresh offset per call (e.g. the decode step).  A NULL ssm_rounding
+ * pointer means round to nearest even.
+ */
+typedef struct {
+    uint64_t seed;
+    uint64_t offset;
+    int philox_rounds;   /* 1 .. 16 */
+} ssm_rounding;
 
 /* Human-readable name of a status code (static string, never NULL). */
 SSM_API const char *ssm_status_string(int status);
@@ -184,8 +205,10 @@ SSM_API int ssm_state_update(int batch, int nheads, int head_dim, int d_state,
 /*
  * ssd_chunk_scan_slots -- ssd_chunk_scan whose initial and final states are
  * rows of a state pool.
- *   state_pool         device fp32 [max_slots][nheads][head_dim][d_state], read
- *                      and written in place (only the rows named in slot_idx)
+ *   state_pool         device [max_slots][nheads][head_dim][d_state], read and
+ *                      written in place (only the rows named in slot_idx)
+ *   state_dtype        SSM_F32, or SSM_F16 (computed in fp32, rounded on write
+ *                      with `rounding`: see ssm_rounding; NULL = nearest even)
  *   max_slots          number of rows of the pool (> 0)
  *   slot_idx           device int32 [nseq]: pool row of sequence s.  Rows must
  *                      be distinct; an index outside [0, max_slots) skips that
@@ -206,7 +229,9 @@ SSM_API int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens
                                  const void *x, const float *dt, const float *A,
                                  const void *B, const void *C, const float *D,
                                  const ssm_dt_params *dt_params,
-                                 float *state_pool, int max_slots, const int32_t *slot_idx,
+                                 void *state_pool, int state_dtype,
+                                 const ssm_rounding *rounding, int max_slots,
+                                 const int32_t *slot_idx,
                                  const int32_t *has_initial_state,
                                  int y_dtype, void *y, int *status_dev, cudaStream_t stream);
 
@@ -216,11 +241,14 @@ SSM_API int ssd_chunk_scan_slots(int nseq, int seqlen, const int32_t *cu_seqlens
  * (no state update, y not written); an index >= max_slots skips the row and
  * sets SSM_ERR_DEVICE_INPUT in *status_dev (status_dev may be NULL).  Slot
  * indices of non-padding rows must be distinct; slot_idx NULL means row b
- * (max_slots >= batch).  dt_params: optional dt transform, or NULL.  Other
- * arguments as for ssm_state_update.
+ * (max_slots >= batch).  dt_params: optional dt transform, or NULL.
+ * state_dtype / rounding: as for ssd_chunk_scan_slots (fp16 pools are read as
+ * fp16, updated in fp32 and rounded back).  Other arguments as for
+ * ssm_state_update.
  */
 SSM_API int ssm_state_update_slots(int batch, int nheads, int head_dim, int d_state,
-                                   int ngroups, int in_dtype, float *state_pool, int max_slots,
+                                   int ngroups, int in_dtype, void *state_pool, int state_dtype,
+                                   const ssm_rounding *rounding, int max_slots,
                                    const int32_t *slot_idx,
                                    const void *x, const float *dt, const float *A,
                                    const void *B, const void *C, const float *D,

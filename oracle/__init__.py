@@ -369,9 +369,9 @@ def philox4x32(counter, key, rounds=10):
     return [int(v) for v in out]
 
 
-def sr_fp16(v, r):
-    """Stochastic rounding of the fp32 value v to fp16 with random word r."""
-    return _load().oracle_sr_fp16(float(np.float32(v)), int(r) & 0xFFFFFFFF)
+def sr_fp16(v, r16):
+    """Stochastic rounding of the fp32 value v to fp16 with 16 random bits r16."""
+    return _load().oracle_sr_fp16(float(np.float32(v)), int(r16) & 0xFFFF)
 
 
 def round_state_f16(values, elem_index, seed, offset, rounds=10):

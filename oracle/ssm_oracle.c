@@ -256,9 +256,10 @@ void oracle_philox4x32(const uint32_t ctr[4], const uint32_t key[2], int rounds,
  * lo the fp16 neighbour toward zero and s the fp16 spacing there (2^(k-10) in
  * the binade [2^k, 2^(k+1)) of the normal range, 2^-24 below 2^-14), the
  * fraction f = (|v| - lo) / s is in [0, 1); the result moves to lo + s iff
- * u < f with u = (r >> 8) / 2^24.  |v| >= 65504 gives +-65504.
+ * u < f with u = r16 / 2^16 for the element's 16 random bits r16.
+ * |v| >= 65504 gives +-65504.
  */
-double oracle_sr_fp16(float vf, uint32_t r)
+double oracle_sr_fp16(float vf, uint32_t r16)
 {
     const double v = vf;
     if (v != v) return v;
@@ -274,7 +275,7 @@ double oracle_sr_fp16(float vf, uint32_t r)
     }
     const double lo = floor(a / s) * s;
     const double f = (a - lo) / s;
-    const double u = (double)(r >> 8) / 16777216.0;
+    const double u = (double)(r16 & 0xFFFFu) / 65536.0;
     double m = lo + (u < f ? s : 0.0);
     if (m > 65504.0) m = 65504.0;
     return copysign(m, v);
@@ -282,10 +283,10 @@ double oracle_sr_fp16(float vf, uint32_t r)
 
 /*
  * Round n state values to fp16 as they are written to a pool: value i is
- * pool element e0 + i; its random word is word (e % 4) of Philox(counter =
- * (e / 4 low, e / 4 high, offset low, offset high), key = (seed low, seed
- * high)).  The decision is taken on the value rounded to fp32 (the precision
- * the state is computed in).
+ * pool element e = elem[i]; its 16 random bits are half (e % 2, low half
+ * first) of word (e % 8) / 2 of Philox(counter = (e / 8 low, e / 8 high,
+ * offset low, offset high), key = (seed low, seed high)).  The decision is
+ * taken on the value rounded to fp32 (the precision the state is computed in).
  */
 void oracle_round_state_f16(long n, const double *v, const int64_t *elem, uint64_t seed,
                             uint64_t offset, int rounds, double *out)
@@ -293,12 +294,13 @@ void oracle_round_state_f16(long n, const double *v, const int64_t *elem, uint64
 #pragma omp parallel for schedule(static)
     for (long i = 0; i < n; ++i) {
         const uint64_t e = (uint64_t)elem[i];
-        const uint64_t q = e >> 2;
+        const uint64_t q = e >> 3;
         const uint32_t ctr[4] = {(uint32_t)q, (uint32_t)(q >> 32), (uint32_t)offset,
                                  (uint32_t)(offset >> 32)};
         const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
         uint32_t w[4];
         oracle_philox4x32(ctr, key, rounds, w);
-        out[i] = oracle_sr_fp16((float)v[i], w[e & 3]);
+        const uint32_t word = w[(e & 7) >> 1];
+        out[i] = oracle_sr_fp16((float)v[i], (e & 1) ? (word >> 16) : (word & 0xFFFFu));
     }
 }

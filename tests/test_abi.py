@@ -138,18 +138,23 @@ def slib(lib):
     vp, i = ctypes.c_void_p, ctypes.c_int
     lib.ssd_chunk_scan_slots.restype = i
     lib.ssd_chunk_scan_slots.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp,
-                                         vp, i, vp, vp, i, vp, vp, vp]
+                                         vp, i, vp, i, vp, vp, i, vp, vp, vp]
     lib.ssm_state_update_slots.restype = i
-    lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, vp, vp, vp, vp, vp, vp,
-                                           vp, i, vp, vp, vp]
+    lib.ssm_state_update_slots.argtypes = [i, i, i, i, i, i, vp, i, vp, i, vp, vp, vp, vp, vp,
+                                           vp, vp, vp, i, vp, vp, vp]
     return lib
 
 
 def scan_slots(lib, nseq=2, seqlen=128, H=4, P=64, N=128, G=1, pool=0x200000, max_slots=8,
-               slots=0x300000, has=None, x=A16, y=0x60000, dtp=None):
+               slots=0x300000, has=None, x=A16, y=0x60000, dtp=None, sd=F32, rnd=None):
     return lib.ssd_chunk_scan_slots(nseq, seqlen, None, H, P, N, G, 128, BF16, x, A16b, A16c,
-                                    0x40000, 0x50000, None, dtp, pool, max_slots, slots, has,
-                                    BF16, y, None, None)
+                                    0x40000, 0x50000, None, dtp, pool, sd, rnd, max_slots, slots,
+                                    has, BF16, y, None, None)
+
+
+class Rounding(ctypes.Structure):
+    _fields_ = [("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64),
+                ("philox_rounds", ctypes.c_int)]
 
 
 class DtParams(ctypes.Structure):
@@ -164,6 +169,8 @@ class DtParams(ctypes.Structure):
     (dict(slots=0x300004), MISALIGNED),
     (dict(dtp=ctypes.byref(DtParams(0x700004, 1, 0, 0.0, 0.0))), MISALIGNED),
     (dict(dtp=ctypes.byref(DtParams(None, 1, 1, 0.5, 0.1))), INVALID),      # dt_min > dt_max
+    (dict(sd=BF16), INVALID),                                                 # bf16 pools: no
+    (dict(sd=2, rnd=ctypes.byref(Rounding(1, 2, 0))), INVALID),               # 0 Philox rounds
     (dict(y=0x200000 + 4096), INVALID),     # y inside the pool
     (dict(P=96), UNSUPPORTED),
 ])
@@ -176,15 +183,18 @@ def test_scan_slots_nseq_zero_is_noop(slib):
 
 
 def update_slots(lib, batch=2, H=4, P=64, N=128, G=2, pool=0x200000, max_slots=8,
-                 slots=0x300000, x=A16, y=0x60000, dtp=None):
-    return lib.ssm_state_update_slots(batch, H, P, N, G, BF16, pool, max_slots, slots, x, A16b,
-                                      A16c, 0x40000, 0x50000, None, dtp, F32, y, None, None)
+                 slots=0x300000, x=A16, y=0x60000, dtp=None, sd=F32, rnd=None):
+    return lib.ssm_state_update_slots(batch, H, P, N, G, BF16, pool, sd, rnd, max_slots, slots,
+                                      x, A16b, A16c, 0x40000, 0x50000, None, dtp, F32, y, None,
+                                      None)
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(max_slots=-1), INVALID),
     (dict(slots=None, max_slots=1), INVALID),
     (dict(dtp=ctypes.byref(DtParams(None, 0, 1, float("nan"), 1.0))), INVALID),
+    (dict(sd=2, rnd=ctypes.byref(Rounding(1, 2, 17))), INVALID),              # > 16 rounds
+    (dict(sd=2, x=0x200000 + 256), INVALID),                                  # x inside fp16 pool
     (dict(x=None), INVALID),
     (dict(pool=0x200008), MISALIGNED),
     (dict(x=0x200000 + 512), INVALID),      # x inside the pool
