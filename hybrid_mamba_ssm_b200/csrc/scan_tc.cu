@@ -262,15 +262,21 @@ struct ChunkDecay {
     bool safe;       // the row block's own decay fits the factorised path
 };
 
-// Cumulative decay of head hh over the chunk starting at c0 with Lc tokens
-// (warpgroup-wide), and this warpgroup's share of the column factors vd,
-// written to vd_out (only the warpgroup with ch == 0 writes).
-__device__ __forceinline__ ChunkDecay chunk_decay(const ScanArgs &a, int H, int hh, float Ah,
-                                                  long c0, int Lc, int i, int wq, int lane, int wg,
+// Raw dt of row i of the chunk starting at c0 (0 past the sequence end t1),
+// loaded ahead of use: the compute loop keeps two chunks of it in flight.
+__device__ __forceinline__ float load_dt(const ScanArgs &a, int H, int hh, long c0, long t1, int i) {
+    return (c0 + i < t1) ? __ldg(a.dt + (size_t)(c0 + i) * H + hh) : 0.f;
+}
+
+// Cumulative decay of head hh over a chunk of Lc tokens whose raw dt for row
+// i is dt_raw (warpgroup-wide), and this warpgroup's share of the column
+// factors vd, written to vd_out (only the warpgroup with ch == 0 writes).
+__device__ __forceinline__ ChunkDecay chunk_decay(const ScanArgs &a, int hh, float Ah, float dt_raw,
+                                                  int Lc, int i, int wq, int lane, int wg,
                                                   int ch, float *sPART, float *sCSB, float *vd_out)
 {
     ChunkDecay d;
-    d.dtv = (i < Lc) ? dt_apply(a.dtp, a.dt[(size_t)(c0 + i) * H + hh], hh) : 0.f;
+    d.dtv = (i < Lc) ? dt_apply(a.dtp, dt_raw, hh) : 0.f;
     float v = d.dtv * Ah;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -483,8 +489,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         float *vd_tab = reinterpret_cast<float *>(smem + OFF_VD);   // [2 buffers][2 heads][128]
         ChunkDecay cur{};
         if (t1 > t0)
-            cur = chunk_decay(a, H, hh, Ah, t0, (int)min((long)kQ, t1 - t0), i, wq, lane, wg, ch,
-                              sPART, sCSB, vd_tab + hd * 128);
+            cur = chunk_decay(a, hh, Ah, load_dt(a, H, hh, t0, t1, i), (int)min((long)kQ, t1 - t0),
+                              i, wq, lane, wg, ch, sPART, sCSB, vd_tab + hd * 128);
+        float dt_n1 = load_dt(a, H, hh, t0 + kQ, t1, i);   // raw dt of the next chunk
         tc::named_sync(BAR_COMPUTE, kCompute);
         uint32_t phase = 0, vb = 0;
         for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u, vb ^= 1u) {
@@ -492,6 +499,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             const long c1 = c0 + kQ;
             const bool has_next = c1 < t1;
             const bool live = i < Lc;
+
+            // dt two chunks ahead, so its load has a whole chunk to land
+            const float dt_n2 = load_dt(a, H, hh, c0 + 2 * kQ, t1, i);
 
             // ---- operands to fp16 (rows past the chunk end zeroed) ----
             tc::mbar_wait_bounded(bar_x, phase, ok);
@@ -522,7 +532,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             // ---- next chunk's decay while the MMAs run ----
             ChunkDecay nxt{};
             if (has_next)
-                nxt = chunk_decay(a, H, hh, Ah, c1, (int)min((long)kQ, t1 - c1), i, wq, lane, wg, ch,
+                nxt = chunk_decay(a, hh, Ah, dt_n1, (int)min((long)kQ, t1 - c1), i, wq, lane, wg, ch,
                                   sPART, sCSB, vd_tab + (vb ^ 1u) * 256 + hd * 128);
             tc::named_sync(BAR_COMPUTE, kCompute);
 
@@ -580,6 +590,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             tc::tc_fence_before();
             tc::named_arrive(BAR_YSTAGED, kCompute + 32);
             cur = nxt;
+            dt_n1 = dt_n2;
         }
         if (a.final_state) {
 #pragma unroll
