@@ -723,10 +723,12 @@ def run_ours(args, world, rank, local, pg):
     barrier(pg, dev)
     e2e_ms = max_over_ranks(pg, s2.elapsed_time(e2), dev)
 
-    conv = time_conv(dev, stream, seed + 17)
-    conv.update(time_mtp(dev, stream, seed + 29))
-    conv.update(time_fused(dev, stream, seed + 41))
-    conv.update(time_f16_decode(dev, stream, seed + 53))
+    conv = {}
+    if not args.no_parts:   # the steps around the scan, timed beside the step
+        conv = time_conv(dev, stream, seed + 17)
+        conv.update(time_mtp(dev, stream, seed + 29))
+        conv.update(time_fused(dev, stream, seed + 41))
+        conv.update(time_f16_decode(dev, stream, seed + 53))
 
     # ---- numbers ----
     peaks, peak_kind = load_peaks()
@@ -801,6 +803,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-parts", action="store_true",
+                    help="skip the timings of the kernels around the scan (conv1d, "
+                         "speculative decode, fused steps, fp16 pools)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # timing rule: at least 3 warm-up steps
     world, rank, local, pg = dist_setup(args)
