@@ -210,8 +210,16 @@ __device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, c
             const float vd[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
             float m[8];
             if (jc < wq) {
+                // (G ua) vd on fp32x2 lanes
+                const float2 ua2 = make_float2(ua, ua);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) m[e] = __uint_as_float(r[q2 * 8 + e]) * ua * vd[e];
+                for (int e = 0; e < 4; ++e) {
+                    const float2 g2 = make_float2(__uint_as_float(r[q2 * 8 + 2 * e]),
+                                                  __uint_as_float(r[q2 * 8 + 2 * e + 1]));
+                    const float2 m2 = __fmul2_rn(__fmul2_rn(g2, ua2), make_float2(vd[2 * e], vd[2 * e + 1]));
+                    m[2 * e] = m2.x;
+                    m[2 * e + 1] = m2.y;
+                }
             } else if (block_safe) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -578,8 +586,14 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 tc::tmem_ld16(tmem + tlane + TM_YO + hd * 64 + ch * 32 + q * 16, ro);
                 tc::tmem_ld_wait();
                 float out[16];
+                const float2 e2 = make_float2(cur.e, cur.e);
 #pragma unroll
-                for (int c = 0; c < 16; ++c) out[c] = fmaf(cur.e, __uint_as_float(ro[c]), __uint_as_float(ry[c]));
+                for (int c = 0; c < 8; ++c) {
+                    const float2 o2 = __ffma2_rn(e2, make_float2(__uint_as_float(ro[2 * c]), __uint_as_float(ro[2 * c + 1])),
+                                                 make_float2(__uint_as_float(ry[2 * c]), __uint_as_float(ry[2 * c + 1])));
+                    out[2 * c] = o2.x;
+                    out[2 * c + 1] = o2.y;
+                }
                 if (kStoreByTma && Lc == kQ) {
                     stage16_bf16(sbase + OFF_MB + hd * HALF, i, 4 * ch + 2 * q, out);
                 } else if (live) {
