@@ -97,9 +97,9 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
 }
 
 __device__ __forceinline__ uint32_t bf2_to_h2(uint32_t v, float scale) {
-    const float lo = __uint_as_float(v << 16) * scale;
-    const float hi = __uint_as_float(v & 0xffff0000u) * scale;
-    __half2 h = __floats2half2_rn(lo, hi);
+    const float2 p = __fmul2_rn(make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u)),
+                                make_float2(scale, scale));
+    __half2 h = __floats2half2_rn(p.x, p.y);
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
@@ -552,9 +552,14 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 uint32_t r[16];
                 tc::tmem_ld16(tmem + tlane + TM_S + hd * 64 + ch * 32 + q * 16, r);
                 tc::tmem_ld_wait();
+                const float2 al2 = make_float2(cur.a_last, cur.a_last);
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    Hs[q * 16 + e] = fmaf(cur.a_last, Hs[q * 16 + e], __uint_as_float(r[e]));
+                for (int e = 0; e < 8; ++e) {
+                    const float2 h2 = __ffma2_rn(al2, make_float2(Hs[q * 16 + 2 * e], Hs[q * 16 + 2 * e + 1]),
+                                                 make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])));
+                    Hs[q * 16 + 2 * e] = h2.x;
+                    Hs[q * 16 + 2 * e + 1] = h2.y;
+                }
             }
             tc::tc_fence_before();
             tc::named_sync(BAR_COMPUTE, kCompute);   // every S column read: M may overwrite them
