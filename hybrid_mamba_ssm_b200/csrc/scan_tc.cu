@@ -221,11 +221,16 @@ __device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, c
                     m[2 * e + 1] = m2.y;
                 }
             } else if (block_safe) {
+                const float2 ua2 = make_float2(ua, ua);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int jl = q * 8 + e;
-                    const float mv = (jl <= lane) ? __uint_as_float(r[q2 * 8 + e]) * ua * vd[e] : 0.f;
-                    m[e] = (jl == lane) ? mv + Dh : mv;
+                for (int e = 0; e < 4; ++e) {
+                    const float2 g2 = make_float2(__uint_as_float(r[q2 * 8 + 2 * e]),
+                                                  __uint_as_float(r[q2 * 8 + 2 * e + 1]));
+                    const float2 m2 = __fmul2_rn(__fmul2_rn(g2, ua2), make_float2(vd[2 * e], vd[2 * e + 1]));
+                    const int j0 = q * 8 + 2 * e;
+                    const float a0 = (j0 <= lane) ? m2.x : 0.f, a1 = (j0 + 1 <= lane) ? m2.y : 0.f;
+                    m[2 * e] = (j0 == lane) ? a0 + Dh : a0;
+                    m[2 * e + 1] = (j0 + 1 == lane) ? a1 + Dh : a1;
                 }
             } else {
 #pragma unroll
