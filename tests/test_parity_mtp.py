@@ -142,3 +142,33 @@ def test_conv_multi_verify_and_commit(dim):
                                    accept_len=torch.from_numpy(acc).cuda(), want_y=False)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(to_np(state), new_ref)
+
+
+@pytest.mark.parametrize("ntok", [1, 2, 5, 8, 9])
+@pytest.mark.parametrize("dtype,P", [("bf16", 64), ("f32", 48)])
+def test_verify_only_against_oracle(ntok, dtype, P):
+    """y-only verify (the pass that reads the state without stepping it), with
+    slots, a padding row and the dt transform; 9 tokens take the stepping
+    kernel, fewer the state-space-duality form."""
+    from hybrid_mamba_ssm_b200 import ssm
+    H, N, G, max_slots = 8, 128, 2, 5
+    slots = np.array([3, -1, 0], dtype=np.int32)
+    batch = slots.shape[0]
+    A, D = synth.make_head_params(281 + ntok, H)
+    pool0 = synth.make_state(282, (max_slots, H, P, N))
+    (x, _, B, C), (xd, _, Bd, Cd) = _draft(283 + ntok, batch, ntok, H, P, N, G, dtype)
+    raw, bias = synth.make_raw_dt(284, (batch, ntok, H), H)
+    pool = dev_f32(pool0)
+    y = torch.full((batch, ntok, H, P), 7.0, device="cuda")
+    ssm.ssm_state_update_multi(pool, xd, dev_f32(raw), dev_f32(A), Bd, Cd, dev_f32(D),
+                               slot_idx=torch.from_numpy(slots).cuda(), y=y,
+                               dt_bias=dev_f32(bias), dt_softplus=True, dt_limit=(1e-3, 0.1))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(pool), pool0.astype(np.float64))   # only read
+    dt = oracle.dt_transform(raw, bias, softplus=True, dt_min=1e-3, dt_max=0.1)
+    live = slots >= 0
+    y_ref, _, _ = oracle.state_update_multi(pool0[slots[live]], x[live], dt[live], A, B[live],
+                                            C[live], D)
+    yn = to_np(y)
+    assert rel_err(yn[live], y_ref) < TOL
+    assert (yn[~live] == 7.0).all()
