@@ -63,6 +63,9 @@ state_update_multi_kernel(MultiUpdateArgs a)
             return;
         }
     }
+    // without y or intermediate states only the committed tokens matter
+    const int nsteps = (!a.y && !a.inter) ? commit : a.ntok;
+    if (nsteps == 0) return;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int li = lane % LPR;
@@ -86,8 +89,8 @@ state_update_multi_kernel(MultiUpdateArgs a)
                                         st + (size_t)r * N + (v * LPR + li) * 4))
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        for (int t0 = 0; t0 < a.ntok; t0 += kTokBlock) {
-            const int nt = min(kTokBlock, a.ntok - t0);
+        for (int t0 = 0; t0 < nsteps; t0 += kTokBlock) {
+            const int nt = min(kTokBlock, nsteps - t0);
             // stage the block's per-token inputs (issued while the state loads fly)
             for (int i = threadIdx.x; i < nt * N; i += blockDim.x) {
                 const int t = i / N, n = i - t * N;
