@@ -89,3 +89,27 @@ def test_bad_cu_seqlens_reported_on_device():
     ssm.ssd_chunk_scan(*args, cu_seqlens=bad, status=status)
     torch.cuda.synchronize()
     assert status.item() == 6
+
+
+def test_scan_many_short_sequences_tensor_core():
+    """Packed sequences of 1..9 tokens and a few longer ones on the
+    tensor-core path: chunks restart at every sequence start, most chunks are
+    ragged, and several sequences share a 128-token TMA tile."""
+    rng = np.random.default_rng(15)
+    lens = [int(v) for v in rng.integers(1, 10, 40)] + [130, 0, 257, 1]
+    inp = synth.make_scan_inputs(15, lens, 8, 64, 128, 2, dtype="bf16", init_state=True)
+    ey, eh, ehs = check(inp, y_dtype=torch.float32, varlen=True)
+    assert ey < TOL and eh < TOL and ehs < 10 * TOL, (ey, eh, ehs)
+
+
+@pytest.mark.parametrize("dt", [0.1, 0.2])
+def test_scan_large_dt_decays_to_zero(dt):
+    """Large dt with A at its most negative: long decays push exp(cs) toward
+    0 inside a chunk.  At dt 0.1 a 32-token block decays by e^-51 (factorised
+    path); at 0.2 by e^-102, beyond the factorised path's bound, so the mask
+    takes one exp per element.  Neither may overflow or produce NaN."""
+    inp = synth.make_scan_inputs(16, [512], 4, 64, 128, 1, dtype="bf16", init_state=True)
+    inp.dt[:] = dt
+    inp.A[:] = -16.0
+    ey, eh, _ = check(inp, y_dtype=torch.float32)
+    assert ey < TOL and eh < TOL, (ey, eh)
