@@ -79,3 +79,18 @@ def test_sr_mean_over_the_random_word_is_exact(v):
         lo, hi = _fp16_bracket(v)
         assert set(np.unique(vals)) <= {lo, hi}
         assert abs(vals.mean() - v) <= 2.0**-24 * 2.0**-16 * 1.0001
+
+
+def test_round_state_draw_layout():
+    """Element e of a pool draws half e % 2 (low half first) of word
+    (e % 8) / 2 of Philox(counter = (e / 8, offset)): values exactly halfway
+    between fp16 neighbours (1 + 2^-11) round up iff that half is below 2^15."""
+    v = np.full(24, 1.0 + 2.0**-11)
+    got = oracle.round_state_f16(v, np.arange(24), 7, 3)
+    ref = []
+    for e in range(24):
+        w = oracle.philox4x32((e // 8, 0, 3, 0), (7, 0), 10)[(e % 8) // 2]
+        r16 = (w >> 16) if e % 2 else (w & 0xFFFF)
+        ref.append(1.0 + 2.0**-10 if r16 < 32768 else 1.0)
+    assert list(got) == ref
+    assert 0 < sum(g > 1.0 for g in got) < 24
