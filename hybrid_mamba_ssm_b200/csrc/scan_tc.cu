@@ -30,12 +30,13 @@
 // Pipeline per chunk (single-buffered tiles, with prefetch where a buffer
 // frees early):
 //   cumsum / decay tables -> wait TMA(x), TMA(B, C) -> convert bf16 -> fp16
-//   (C rows by warpgroup 0, B rows by warpgroup 1, x and w o x per head)
+//   (C into TMEM and B in place, a quarter of d_state per warpgroup; x and
+//   w o x per head)
 //   -> issue TMA(x of next chunk) into the raw x buffers
 //   -> MMA S^T (2 heads), G  [commit] , Yoff (2 heads) [commit]
-//   -> decay mask M per head (overlaps the Yoff MMAs)
-//   -> issue TMA(B, C of next chunk); MMA Y (2 heads) [commit]
-//   -> state update from S^T (overlaps the Y MMAs) -> epilogue y.
+//   -> issue TMA(B, C of next chunk) once S^T and G are done
+//   -> state update from S^T, decay mask M per head (overlap the Yoff MMAs)
+//   -> MMA Y (2 heads) [commit] -> epilogue y.
 //
 // Precision: bf16 inputs are converted to fp16 (exact for |v| < 65504) so the
 // derived operands M, w o x and H (rounded to fp16, 11 significant bits) keep
@@ -66,7 +67,7 @@ constexpr int kThreads = 544;   // 16 compute warps + 1 issuing warp
 // elements (128 B), 8-row groups of 1024 B, 16-byte chunk c of row r stored at
 // c ^ (r % 8).  128-wide tiles are two 64-column halves 16 KB apart.
 constexpr uint32_t HALF = 16384;
-constexpr uint32_t OFF_C = 0;            // C [128 i][128 n]  (bf16 -> fp16 in place)
+constexpr uint32_t OFF_C = 0;            // C [128 i][128 n]  bf16 (TMA target; fp16 copy in TMEM)
 constexpr uint32_t OFF_B = 32768;        // B [128 j][128 n]  (bf16 -> fp16 in place)
 constexpr uint32_t OFF_XR = 65536;       // raw x, 2 heads x [128 j][64 p] bf16 (TMA target)
 constexpr uint32_t OFF_XH = 98304;       // x as fp16, 2 heads
@@ -82,7 +83,10 @@ constexpr uint32_t OFF_TM = OFF_BAR + 40;
 constexpr uint32_t SMEM_BYTES = OFF_TM + 16;
 
 // TMEM columns (fp32 accumulators, lane = row).
-constexpr uint32_t TM_G = 0, TM_S = 128, TM_YO = 256, TM_Y = 384;
+// G and Y share columns: the y MMAs write Y only after the mask has read G,
+// and the next chunk's G is issued only after the epilogue has read Y.  C
+// (fp16, two values per column) is the TMEM A operand of C.B^T and C.H^T.
+constexpr uint32_t TM_G = 0, TM_Y = 0, TM_S = 128, TM_YO = 256, TM_C = 384;
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_G = tc::idesc_f16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
@@ -411,7 +415,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         // descriptors (start-address field advanced by offset >> 4 per K step)
         const uint64_t dBmn = tc::sdesc_sw128(sbase + OFF_B, HALF, 1024);   // B^T, MN-major
         const uint64_t dW = tc::sdesc_sw128(sbase + OFF_WM, HALF, 1024);    // [wX_a | wX_b]
-        const uint64_t dCk = tc::sdesc_sw128(sbase + OFF_C, 16, 1024);      // C, K-major
         const uint64_t dBk = tc::sdesc_sw128(sbase + OFF_B, 16, 1024);      // B, K-major
         const uint64_t dH = tc::sdesc_sw128(sbase + OFF_H, HALF, 1024);     // [H_a^T | H_b^T]
         const uint64_t dXa = tc::sdesc_sw128(sbase + OFF_XH, HALF, 1024);
@@ -445,20 +448,17 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
-                    tc::mma_f16_ss(tmem + TM_G, dCk + ko, dBk + ko, IDESC_G, kk > 0);
+                    tc::mma_f16_ts(tmem + TM_G, tmem + TM_C + kk * 8, dBk + ko, IDESC_G, kk > 0);
                 }
                 tc::mma_commit(bar_sg);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
-                    tc::mma_f16_ss(tmem + TM_YO, dCk + ko, dH + kk * 128, IDESC_YO2, kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ts(tmem + TM_YO, tmem + TM_C + kk * 8, dH + kk * 128, IDESC_YO2, kk > 0);
                 tc::mma_commit(bar_yo);
-            }
-            __syncwarp();
-            tc::named_sync(BAR_MASK, kCompute + 32);
-            if (leader) {
-                tc::mbar_wait_bounded(bar_yo, phase, ok);   // C and B tiles free
+                // The compute warps read C from shared memory before the operand
+                // barrier; B is read by the S and G MMAs only: both tiles are free
+                // once those complete.
+                tc::mbar_wait_bounded(bar_sg, phase, ok);
                 if (has_next) {
                     tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
                     tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)c1);
@@ -466,6 +466,10 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                     tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)c1);
                     tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)c1);
                 }
+            }
+            __syncwarp();
+            tc::named_sync(BAR_MASK, kCompute + 32);
+            if (leader) {
                 tc::tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
@@ -520,10 +524,24 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             tc::mbar_wait_bounded(bar_x, phase, ok);
             tc::mbar_wait_bounded(bar_cb, phase, ok);
             {
-                const uint32_t tile = sbase + (hd == 0 ? OFF_C : OFF_B) + ch * HALF;
+                // warpgroup wg takes d_state columns n in [32 wg, 32 wg + 32) of row i:
+                // C as fp16 pairs into TMEM (lane i, columns 16 wg ..), B in place
+                const uint32_t ctile = sbase + OFF_C + (wg >> 1) * HALF;
+                const uint32_t btile = sbase + OFF_B + (wg >> 1) * HALF;
+                uint32_t pc[16];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t addr = tile + sw128(i, k);
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = live ? cvt_chunk(lds128(ctile + sw128(i, 4 * (wg & 1) + q)))
+                                         : make_uint4(0, 0, 0, 0);
+                    pc[4 * q] = v.x;
+                    pc[4 * q + 1] = v.y;
+                    pc[4 * q + 2] = v.z;
+                    pc[4 * q + 3] = v.w;
+                }
+                tc::tmem_st16(tmem + tlane + TM_C + 16 * wg, pc);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t addr = btile + sw128(i, 4 * (wg & 1) + q);
                     sts128(addr, live ? cvt_chunk(lds128(addr)) : make_uint4(0, 0, 0, 0));
                 }
 #pragma unroll
@@ -539,7 +557,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                     }
                 }
             }
+            tc::tmem_st_wait();
             tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
             tc::named_arrive(BAR_OPERANDS, kCompute + 32);
 
             // ---- next chunk's decay while the MMAs run ----
