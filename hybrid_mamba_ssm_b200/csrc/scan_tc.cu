@@ -184,6 +184,34 @@ __device__ __forceinline__ void write_state_half(uint32_t sH, uint32_t n, int ch
     }
 }
 
+// Diagonal block jc of row i when the block's own decay is beyond the
+// factorised path's bound: one exp per element.  It only runs for extreme
+// decays, so it is kept out of line, out of the instruction stream of the
+// chunk loop.
+__device__ __noinline__ void mask_block_exact(uint32_t g_taddr, uint32_t m_taddr, int jc, int lane,
+                                              float cs, float dtv, float Dh)
+{
+    uint32_t pk[16];
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {   // 16 columns at a time
+        uint32_t r[16];
+        tc::tmem_ld16(g_taddr + jc * 32 + qq * 16, r);
+        tc::tmem_ld_wait();
+        float m[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int jl = qq * 16 + e;   // column within the block = lane of its row
+            const float csj = __shfl_sync(0xffffffffu, cs, jl);
+            const float dtj = __shfl_sync(0xffffffffu, dtv, jl);
+            const float mv = (jl <= lane) ? __uint_as_float(r[e]) * expf(cs - csj) * dtj : 0.f;
+            m[e] = (jl == lane) ? mv + Dh : mv;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pk[qq * 8 + e] = f2_to_h2(m[2 * e], m[2 * e + 1]);
+    }
+    tc::tmem_st16(m_taddr + jc * 16, pk);
+}
+
 // One 32-column block jc of row i of the decay mask M, as fp16 pairs into
 // TMEM (lane i, columns m_taddr + 16 jc ..  + 16: the A operand of the y MMA):
 //   off-diagonal (jc < wq):  G[i][j] * exp(cs_i - cs_{r_jc}) * vd[j]
@@ -199,6 +227,10 @@ __device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, c
 #pragma unroll
         for (int q = 0; q < 16; ++q) pk[q] = 0u;
         tc::tmem_st16(m_taddr + jc * 16, pk);
+        return;
+    }
+    if (jc == wq && !block_safe) {
+        mask_block_exact(g_taddr, m_taddr, jc, lane, cs, dtv, Dh);
         return;
     }
     const float4 *vd4 = reinterpret_cast<const float4 *>(sVD + jc * 32);
@@ -224,7 +256,7 @@ __device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, c
                     m[2 * e] = m2.x;
                     m[2 * e + 1] = m2.y;
                 }
-            } else if (block_safe) {
+            } else {   // diagonal block, factorised
                 const float2 ua2 = make_float2(ua, ua);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -235,15 +267,6 @@ __device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, c
                     const float a0 = (j0 <= lane) ? m2.x : 0.f, a1 = (j0 + 1 <= lane) ? m2.y : 0.f;
                     m[2 * e] = (j0 == lane) ? a0 + Dh : a0;
                     m[2 * e + 1] = (j0 + 1 == lane) ? a1 + Dh : a1;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int jl = q * 8 + e;
-                    const float csj = __shfl_sync(0xffffffffu, cs, jl);
-                    const float dtj = __shfl_sync(0xffffffffu, dtv, jl);
-                    const float mv = (jl <= lane) ? __uint_as_float(r[q2 * 8 + e]) * expf(cs - csj) * dtj : 0.f;
-                    m[e] = (jl == lane) ? mv + Dh : mv;
                 }
             }
 #pragma unroll
