@@ -590,7 +590,6 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             if (has_next)
                 nxt = chunk_decay(a, hh, Ah, dt_n1, (int)min((long)kQ, t1 - c1), i, wq, lane, wg, ch,
                                   sPART, sCSB, vd_tab + (vb ^ 1u) * 256 + hd * 128);
-            tc::named_sync(BAR_COMPUTE, kCompute);
 
             // ---- carried state: H <- exp(cs_L) H + S (d_state row i, p half ch) ----
             tc::mbar_wait_bounded(bar_sg, phase, ok);
