@@ -19,21 +19,22 @@
 // The diagonal j = i belongs to M because the output reads the updated state.
 //
 // Work decomposition: one CTA per (sequence, pair of heads of one group),
-// sweeping the sequence's chunks in order.  512 threads = four warpgroups;
-// warpgroup wg works on head 2k + (wg & 1) and on half (wg >> 1) of the
-// columns: thread i of it owns TMEM lane i (row i of G, M, Y, Yoff; d_state
-// index i of S^T and of the carried state, 32 of whose 64 head_dim entries it
-// keeps in fp32 registers for the whole sequence).  Thread 0 issues TMA and
-// the MMAs; the products shared by both heads (C.B^T, and B^T or C against the
-// two heads' operands side by side) are single N = 128 MMAs.
+// sweeping the sequence's chunks in order.  544 threads: four compute
+// warpgroups and one issuing warp.  Compute warpgroup wg works on head
+// 2k + (wg & 1) and on half (wg >> 1) of the columns: thread i of it owns TMEM
+// lane i (row i of G, M, Y, Yoff; d_state index i of S^T and of the carried
+// state, 32 of whose 64 head_dim entries it keeps in fp32 registers for the
+// whole sequence).  Lane 0 of the issuing warp issues TMA and the MMAs; the
+// products shared by both heads (C.B^T, and B^T or C against the two heads'
+// operands side by side) are single N = 128 MMAs.
 //
 // Pipeline per chunk (single-buffered tiles, with prefetch where a buffer
 // frees early):
-//   cumsum / decay tables -> wait TMA(x), TMA(B, C) -> convert bf16 -> fp16
-//   (C into TMEM and B in place, a quarter of d_state per warpgroup; x and
-//   w o x per head)
+//   wait TMA(x), TMA(B, C) -> convert bf16 -> fp16 (C into TMEM and B in
+//   place, a quarter of d_state per warpgroup; x and w o x per head)
 //   -> issue TMA(x of next chunk) into the raw x buffers
 //   -> MMA S^T (2 heads), G  [commit] , Yoff (2 heads) [commit]
+//   -> the next chunk's cumulative decay (while the MMAs run)
 //   -> issue TMA(B, C of next chunk) once S^T and G are done
 //   -> state update from S^T, decay mask M per head (overlap the Yoff MMAs)
 //   -> MMA Y (2 heads) [commit] -> epilogue y.
