@@ -58,7 +58,7 @@ typedef enum {
     SSM_ERR_UNSUPPORTED = 2,   /* valid request this build does not handle */
     SSM_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
     SSM_ERR_CUDA = 4,          /* the CUDA runtime reported a launch error */
-    SSM_ERR_TIMEOUT = 5,       /* reserved: a bounded device wait expired */
+    SSM_ERR_TIMEOUT = 5,       /* written to status_dev: a bounded device wait expired */
     SSM_ERR_DEVICE_INPUT = 6   /* written to status_dev: bad cu_seqlens or slot index */
 } ssm_status;
 
