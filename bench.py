@@ -10,10 +10,14 @@ One step = one pass of the whole hot path over one batch of synthetic input:
     on a 512 MiB fp32 state, bf16 x/B/C, bf16 y; per-step inputs cycle through
     a ring of 8 seeded input sets.
 ``value`` is tokens/s over both (16384 prefill + 64 decode tokens per step and
-per GPU); the per-kernel numbers the metric names (prefill tokens/s and % of
-tensor peak, decode GB/s and % of HBM peak) are under ``parts``, with the
-causal conv1d that feeds the scan timed beside the step (``conv1d_prefill``:
-4 x 4096 tokens x 10240 channels; ``conv1d_decode``: 64 rows x 18432 channels).
+per GPU); the numbers the metric names (prefill ms, TFLOP/s and % of tensor
+peak, decode GB/s and % of HBM peak) are top-level keys of the headline line.
+Timed beside the step: the long prefill at the Ultra layer shape (1 x 32768
+tokens, 256 heads, nonzero initial state) and the mixed workload (8 packed
+sequences of 512..16384 tokens, then 128 decode steps), both summarised in the
+headline; the causal conv1d that feeds the scan, speculative decode, the
+fused steps and fp16 state pools, detailed on a separate JSON line printed
+just before the headline (``bench_parts``).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun each rank runs its own batch (weak scaling, no data-path
@@ -55,18 +59,27 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def prefill_work(p=PREFILL, y_bytes=2):
+# Long prefill at the Ultra layer shape (nonzero initial state, bf16 y) and
+# the mixed prefill-then-decode workload (8 packed sequences of seeded
+# lengths, then 128 decode steps each): timed beside the step.
+ULTRA32K = dict(nseq=1, seqlen=32768, H=256, P=64, N=128, G=8, Q=128, h0=True)
+MIXED = dict(nseq=8, lo=512, hi=16384, H=128, P=64, N=128, G=8, Q=128, decode_steps=128)
+
+
+def prefill_work(p=PREFILL, y_bytes=2, T=None):
     """Algorithmic flops and bytes of one prefill launch.
 
     flops per token = H(2QP + 4NP) + G*2QN (full Q x Q masked tile, the four
     per-head contractions C.B^T-masked.X, X^T.B, C.H^T and the group's C.B^T);
-    bytes = x + B + C + dt + y per token, plus the fp32 final state.
+    bytes = x + B + C + dt + y per token, plus the fp32 final state (and the
+    initial state when the workload has one).
     """
-    T = p["nseq"] * p["seqlen"]
+    T = p["nseq"] * p["seqlen"] if T is None else T
     H, P, N, G, Q = p["H"], p["P"], p["N"], p["G"], p["Q"]
     flops = T * (H * (2 * Q * P + 4 * N * P) + G * 2 * Q * N)
     per_tok = H * P * 2 + 2 * G * N * 2 + H * 4 + H * P * y_bytes
-    bytes_ = T * per_tok + p["nseq"] * H * P * N * 4 + 2 * H * 4
+    states = 2 if p.get("h0") else 1
+    bytes_ = T * per_tok + states * p["nseq"] * H * P * N * 4 + 2 * H * 4
     return flops, bytes_, T
 
 
@@ -540,6 +553,124 @@ def time_f16_decode(dev, stream, seed, iters=20):
     return out
 
 
+def prefill_numbers(flops, nbytes, tokens, ms, peaks):
+    """Throughput and roofline fractions of one prefill launch."""
+    t_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tf = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": ms, "tokens_per_s": tokens / (ms * 1e-3), "tflops": tf,
+            "tensor_frac_burst": tf / peaks["bf16_tflops"], "tensor_frac_sustained": tf / t_sus,
+            "gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"], "flops_per_launch": flops,
+            "bytes_per_launch": nbytes}
+
+
+def time_ultra32k(dev, stream, peaks, iters=10):
+    """Long prefill, 1 x 32768 tokens at the Ultra layer shape (256 heads,
+    nonzero fp32 initial state, bf16 y, fp32 final state): per-launch CUDA
+    events; 2.3 GB of inputs and outputs per launch, larger than L2."""
+    import torch
+    from hybrid_mamba_ssm_b200 import inputs as synth
+    from hybrid_mamba_ssm_b200 import ssm
+    u = ULTRA32K
+    inp = synth.make_scan_inputs(1000 + 3, [u["seqlen"]], u["H"], u["P"], u["N"], u["G"],
+                                 dtype="bf16", init_state=True)
+    b16 = lambda t: torch.from_numpy(np.ascontiguousarray(t.bits).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+    L = u["seqlen"]
+    x = b16(inp.x).view(1, L, u["H"], u["P"])
+    B = b16(inp.B).view(1, L, u["G"], u["N"])
+    C = b16(inp.C).view(1, L, u["G"], u["N"])
+    dt = f32(inp.dt).view(1, L, u["H"])
+    A, D, h0 = f32(inp.A), f32(inp.D), f32(inp.h0)
+    del inp
+    y = torch.empty_like(x)
+    hT = torch.empty_like(h0)
+    call = lambda: ssm.ssd_chunk_scan(x, dt, A, B, C, D, h0, chunk_size=u["Q"], y=y,
+                                      final_state=hT, stream=stream)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
+    f, b, T = prefill_work(u)
+    out = prefill_numbers(f, b, T, ms, peaks)
+    out["launches"] = iters
+    del x, B, C, dt, y
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_mixed(dev, stream, peaks, iters=5):
+    """Mixed workload: 8 packed sequences (seeded lengths in 512..16384,
+    128 heads, per-sequence fp32 initial states) prefilled with one varlen
+    ssd_chunk_scan, then 128 ssm_state_update steps on the 8 final states.
+    Prefill tokens/s from per-launch events; decode steps/s over the 128
+    consecutive steps (fresh inputs each step)."""
+    import torch
+    from hybrid_mamba_ssm_b200 import inputs as synth
+    from hybrid_mamba_ssm_b200 import ssm
+    m = MIXED
+    seed = 1000 + 4
+    lens = synth.mixed_seqlens(seed, m["nseq"], m["lo"], m["hi"])
+    inp = synth.make_scan_inputs(seed, lens, m["H"], m["P"], m["N"], m["G"], dtype="bf16",
+                                 init_state=True)
+    b16 = lambda t: torch.from_numpy(np.ascontiguousarray(t.bits).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+    x, B, C, dt = b16(inp.x), b16(inp.B), b16(inp.C), f32(inp.dt)
+    A, D, h0 = f32(inp.A), f32(inp.D), f32(inp.h0)
+    cu = torch.from_numpy(inp.cu_seqlens.astype(np.int32)).to(dev)
+    y = torch.empty_like(x)
+    hT = torch.empty_like(h0)
+    pre = lambda: ssm.ssd_chunk_scan(x, dt, A, B, C, D, h0, cu_seqlens=cu, chunk_size=m["Q"],
+                                     y=y, final_state=hT, stream=stream)
+    steps = [synth.make_decode_step(seed + 500 + k, m["nseq"], m["H"], m["P"], m["N"], m["G"])
+             for k in range(m["decode_steps"])]
+    dsteps = [(b16(s.x), f32(s.dt), b16(s.B), b16(s.C)) for s in steps]
+    dy = torch.empty((m["nseq"], m["H"], m["P"]), dtype=torch.bfloat16, device=dev)
+    state = torch.empty_like(hT)
+
+    def decode_all():
+        for xs, dts, Bs, Cs in dsteps:
+            ssm.ssm_state_update(state, xs, dts, A, Bs, Cs, D, y=dy, stream=stream)
+
+    for _ in range(3):
+        pre()
+    state.copy_(hT)
+    decode_all()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        pre()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    pre_ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / iters
+    state.copy_(hT)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    decode_all()
+    d1.record(stream)
+    torch.cuda.synchronize(dev)
+    dec_ms = d0.elapsed_time(d1)
+    T = int(sum(lens))
+    f, b, _ = prefill_work(dict(m, nseq=m["nseq"], h0=True), T=T)
+    out = {"prefill": prefill_numbers(f, b, T, pre_ms, peaks),
+           "decode_steps_per_s": m["decode_steps"] / (dec_ms * 1e-3),
+           "decode_ms_per_step": dec_ms / m["decode_steps"], "tokens": T,
+           "seqlens": [int(v) for v in lens]}
+    out["prefill"]["launches"] = iters
+    return out
+
+
 def run_reference(args, world, rank, pg):
     if rank != 0:
         return 0
@@ -723,6 +854,12 @@ def run_ours(args, world, rank, local, pg):
     barrier(pg, dev)
     e2e_ms = max_over_ranks(pg, s2.elapsed_time(e2), dev)
 
+    peaks, peak_kind = load_peaks()
+    # the other prefill workloads, timed beside the step
+    ultra = mixed = None
+    if not args.no_parts:
+        ultra = time_ultra32k(dev, stream, peaks)
+        mixed = time_mixed(dev, stream, peaks)
     conv = {}
     if not args.no_parts:   # the steps around the scan, timed beside the step
         conv = time_conv(dev, stream, seed + 17)
@@ -731,7 +868,6 @@ def run_ours(args, world, rank, local, pg):
         conv.update(time_f16_decode(dev, stream, seed + 53))
 
     # ---- numbers ----
-    peaks, peak_kind = load_peaks()
     for part in conv.values():
         if "gbs" in part:
             part["hbm_frac"] = part["gbs"] / peaks["hbm_gbs"]
@@ -742,12 +878,7 @@ def run_ours(args, world, rank, local, pg):
     df, db, _ = decode_work()
     hbm = peaks["hbm_gbs"]
     t_sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    pre = {"tokens_per_s": ptok / (pre_ms * 1e-3), "ms": pre_ms,
-           "tflops": pf / (pre_ms * 1e-3) / 1e12,
-           "tensor_frac_sustained": pf / (pre_ms * 1e-3) / 1e12 / t_sus,
-           "tensor_frac_burst": pf / (pre_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
-           "gbs": pb / (pre_ms * 1e-3) / 1e9, "hbm_frac": pb / (pre_ms * 1e-3) / 1e9 / hbm,
-           "flops_per_launch": pf, "bytes_per_launch": pb}
+    pre = prefill_numbers(pf, pb, ptok, pre_ms, peaks)
     dec = {"gbs": db / (dec_ms * 1e-3) / 1e9, "ms": dec_ms,
            "hbm_frac": db / (dec_ms * 1e-3) / 1e9 / hbm,
            "hbm_frac_of_8TBs": db / (dec_ms * 1e-3) / 8e12,
@@ -769,17 +900,22 @@ def run_ours(args, world, rank, local, pg):
                 "traffic": measured_traffic("ssm_state_update", "state_update.cu")}
     roof["peak_source"] = peak_kind
 
+    r3 = lambda v: float(f"{v:.4g}")
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "prefill 4x4096 H128 P64 N128 G8 Q128 + decode 64x256x64x128 G8",
-                       "prefill": dict(PREFILL, in_dtype="bf16", y_dtype="bf16",
-                                       initial_state="zero"),
-                       "decode": dict(DECODE, in_dtype="bf16", y_dtype="bf16", ring=RING),
                        "l2": "inputs larger than L2 (about 1.7 GB touched per step)",
                        "parallelism": f"replicas x{world} (independent batches per GPU)"},
-            "parts": {"prefill": pre, "decode": dec, **conv},
+            # the two numbers the metric names: prefill (% tensor peak) and decode (% HBM)
+            "prefill_ms": r3(pre_ms), "prefill_tokens_per_s": r3(pre["tokens_per_s"]),
+            "prefill_tflops": r3(pre["tflops"]),
+            "prefill_tensor_frac_burst": r3(pre["tensor_frac_burst"]),
+            "prefill_tensor_frac_sustained": r3(pre["tensor_frac_sustained"]),
+            "prefill_hbm_frac": r3(pre["hbm_frac"]),
+            "decode_ms": r3(dec_ms), "decode_gbs": r3(dec["gbs"]),
+            "decode_hbm_frac": r3(dec["hbm_frac"]), "decode_frac_of_8TBs": r3(dec["hbm_frac_of_8TBs"]),
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -787,11 +923,26 @@ def run_ours(args, world, rank, local, pg):
             "gpu_launches": 2 * K,
             "clocks": clock_info}
 
+    if ultra is not None:
+        line["prefill_ultra_32k"] = {k: r3(ultra[k]) for k in ("ms", "tokens_per_s", "tflops",
+                                                               "tensor_frac_burst", "hbm_frac")}
+        line["mixed_varlen"] = {"prefill_tokens_per_s": r3(mixed["prefill"]["tokens_per_s"]),
+                                "decode_steps_per_s": r3(mixed["decode_steps_per_s"])}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         step_s, desc, cores = oracle_step_sample(3000, 1024, 8, 4)
         line["cpu_baseline"] = {"value": tok_step / step_s, "unit": "tokens/s", "cores": cores,
                                 "kind": "oracle", "sample": desc}
     if rank == 0:
+        # per-kernel detail on its own line first; the headline line, short,
+        # is the last line printed
+        detail = {"bench_parts": {"prefill": pre, "decode": dec, "prefill_ultra_32k": ultra,
+                                  "mixed_varlen": mixed, **conv},
+                  "workloads": {"prefill": dict(PREFILL, in_dtype="bf16", y_dtype="bf16",
+                                                initial_state="zero"),
+                                "decode": dict(DECODE, in_dtype="bf16", y_dtype="bf16",
+                                               ring=RING),
+                                "prefill_ultra_32k": ULTRA32K, "mixed_varlen": MIXED}}
+        print(json.dumps(detail), flush=True)
         print(json.dumps(line), flush=True)
     return 0
 

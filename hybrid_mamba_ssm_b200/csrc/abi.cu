@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include "../../include/ssm.h"
+#include "../../include/ssm_testing.h"
 #include "ssm_internal.h"
 
 namespace {
@@ -86,6 +87,8 @@ const char *ssm_status_string(int status)
     case SSM_ERR_CUDA: return "SSM_ERR_CUDA: CUDA launch error";
     case SSM_ERR_TIMEOUT: return "SSM_ERR_TIMEOUT: bounded device wait expired";
     case SSM_ERR_DEVICE_INPUT: return "SSM_ERR_DEVICE_INPUT: inconsistent cu_seqlens or slot index";
+    case SSM_ERR_RANGE: return "SSM_ERR_RANGE: a value beyond the fp16 range of the tensor-core operands";
+    case SSM_ERR_INTERNAL: return "SSM_ERR_INTERNAL: launch configuration broke a kernel layout rule";
     default: return "unknown ssm status";
     }
 }
@@ -559,6 +562,53 @@ int ssm_gated_rmsnorm(int rows, int dim, int group_size, int y_dtype, const void
     a.y_dtype = y_dtype; a.z_dtype = z_dtype; a.out_dtype = out_dtype;
     a.y = y; a.z = z; a.weight = weight; a.eps = eps; a.out = out;
     return ssm::launch_gated_rmsnorm(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+
+// ---------------------------------------------------------------- testing hooks
+int ssm_testing_scan_stalled(int nseq, int seqlen, int nheads, int ngroups,
+                             const void *x, const float *dt, const float *A,
+                             const void *B, const void *C, void *y,
+                             unsigned long long wait_ns, int *status_dev, cudaStream_t stream)
+{
+    if (nseq <= 0 || seqlen <= 0 || nheads <= 0 || ngroups <= 0 || nheads % ngroups)
+        return SSM_ERR_INVALID_ARG;
+    if (!x || !dt || !A || !B || !C || !y || !status_dev) return SSM_ERR_INVALID_ARG;
+    if (wait_ns < 1000ull || wait_ns > 10000000000ull) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, dt, A, B, C, y, status_dev};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return SSM_ERR_MISALIGNED;
+    if ((long long)nseq * seqlen > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    ssm::ScanArgs a{};
+    a.nseq = nseq; a.seqlen = seqlen; a.cu_seqlens = nullptr;
+    a.nheads = nheads; a.head_dim = 64; a.d_state = 128; a.ngroups = ngroups; a.chunk_size = 128;
+    a.in_dtype = SSM_BF16; a.y_dtype = SSM_BF16;
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = nullptr;
+    a.y = y; a.status_dev = status_dev;
+    a.wait_ns = wait_ns; a.stall_producer = 1;
+    if (!ssm::scan_tc_supports(a)) return SSM_ERR_UNSUPPORTED;
+    return ssm::launch_scan_tc(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
+}
+
+int ssm_testing_conv1d_stalled(int nseq, int seqlen, int dim, int width, const void *x,
+                               const float *weight, void *y, unsigned long long wait_ns,
+                               int *status_dev, cudaStream_t stream)
+{
+    if (nseq <= 0 || seqlen <= 0 || dim <= 0 || dim % 8 || width < 1 || width > 8)
+        return SSM_ERR_INVALID_ARG;
+    if (!x || !weight || !y || !status_dev) return SSM_ERR_INVALID_ARG;
+    if (wait_ns < 1000ull || wait_ns > 10000000000ull) return SSM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, weight, y, status_dev};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return SSM_ERR_MISALIGNED;
+    if ((long long)nseq * seqlen > 0x7fffffffLL) return SSM_ERR_UNSUPPORTED;
+    ssm::ConvArgs a{};
+    a.update = 0; a.nseq = nseq; a.seqlen = seqlen;
+    a.dim = dim; a.width = width; a.activation = 0;
+    a.in_dtype = SSM_BF16; a.y_dtype = SSM_BF16;
+    a.x = x; a.weight = weight; a.y = y; a.status_dev = status_dev;
+    a.wait_ns = wait_ns; a.stall_producer = 1;
+    return ssm::launch_conv1d(a, stream) == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 
 }  // extern "C"

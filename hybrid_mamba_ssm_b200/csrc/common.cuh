@@ -153,6 +153,16 @@ __device__ __forceinline__ void state_store1(void *base, size_t e, float v, cons
 }
 
 // Status word written by kernels (only ever set to a nonzero code).
+// Codes a kernel writes to the caller's status word (the ssm_status values of
+// include/ssm.h).
+constexpr int kStatusTimeout = 5;      // a bounded wait expired
+constexpr int kStatusDeviceInput = 6;  // inconsistent cu_seqlens or slot index
+constexpr int kStatusRange = 7;        // a tensor-core operand beyond the fp16 range
+constexpr int kStatusInternal = 8;     // a launch that breaks the kernel's own layout rule
+
+// Default limit of a bounded wait (wall time, via %globaltimer).
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+
 __device__ __forceinline__ void report_status(int *status, int code) {
     if (status) atomicCAS(status, 0, code);
 }

@@ -253,6 +253,7 @@ conv1d_fwd_pipe_kernel(ConvArgs a, int ncta)
     using Raw = typename ConvVec<TIn>::Raw;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_seq;
+    __shared__ int s_abort;   // set when a stage's wait expires
     const uint32_t ring = tc::smem_u32(smem);
     const uint32_t bar0 = ring + kPipeStages * kPipeRows * kPipeRowBytes;
     const int tid = threadIdx.x, dim = a.dim;
@@ -267,7 +268,11 @@ conv1d_fwd_pipe_kernel(ConvArgs a, int ncta)
     const TIn *x = static_cast<const TIn *>(a.x);
     TOut *y = static_cast<TOut *>(a.y);
 
+    const bool produce = a.stall_producer == 0;
+    int issued = 0;   // stages armed so far (thread 0), for the drain after an abort
     auto issue = [&](int g) {
+        if (!produce) return;
+        issued = g + 1;
         const int slot = g % kPipeStages;
         const long r0 = t_begin + (long)g * kPipeRows;
         const int n = (int)min((long)kPipeRows, t_end - r0);
@@ -279,6 +284,7 @@ conv1d_fwd_pipe_kernel(ConvArgs a, int ncta)
     };
     if (tid == 0) {
         for (int i = 0; i < kPipeStages; ++i) tc::mbar_init(bar0 + 8 * i, 1);
+        s_abort = 0;
         tc::fence_mbar_init();
         for (int g = 0; g < min(kPipeStages, groups); ++g) issue(g);
         int s = 0;
@@ -366,17 +372,20 @@ conv1d_fwd_pipe_kernel(ConvArgs a, int ncta)
             for (int p = 0; p < P2; ++p) win[W - 1][p] = cur[p];
     };
 
+    const uint64_t limit_ns = a.wait_ns ? a.wait_ns : kDefaultWaitNs;
     bool ok = true;
-    for (int g = 0; g < groups; ++g) {
+    int g = 0;
+    for (; g < groups; ++g) {
         const int slot = g % kPipeStages;
-        if (!tc::mbar_wait_bounded(bar0 + 8 * slot, (uint32_t)((g / kPipeStages) & 1), ok)) {
-            if (tid == 0) report_status(a.status_dev, 5);
-            return;   // a bulk copy that never lands: nothing in flight can be waited for
-        }
+        // A stage that does not land in time raises the CTA-wide abort flag;
+        // every thread sees it after this iteration's barrier and leaves the
+        // loop, and thread 0 then drains the copies still in flight.
+        if (!tc::mbar_wait_bounded(bar0 + 8 * slot, (uint32_t)((g / kPipeStages) & 1), ok, limit_ns))
+            *reinterpret_cast<volatile int *>(&s_abort) = 1;
         const long r0 = t_begin + (long)g * kPipeRows;
         const int n = (int)min((long)kPipeRows, t_end - r0);
         const uint8_t *base = smem + slot * kPipeRows * kPipeRowBytes + tid * 16;
-        if (active && !dead) {
+        if (ok && active && !dead) {
             if (n == kPipeRows && r0 + kPipeRows <= te) {
                 // whole stage inside the current sequence
 #pragma unroll
@@ -400,10 +409,21 @@ conv1d_fwd_pipe_kernel(ConvArgs a, int ncta)
             }
         }
         __syncthreads();                 // every thread is done with this slot
+        if (*reinterpret_cast<volatile int *>(&s_abort)) break;   // uniform after the barrier
         if (tid == 0 && g + kPipeStages < groups) {
             tc::fence_proxy_async_smem();
             issue(g + kPipeStages);
         }
+    }
+    if (g < groups && tid == 0) {
+        // Aborted at stage g: wait (bounded) for the last phase armed on each
+        // ring slot, so that no bulk copy lands after the CTA has exited.
+        for (int q = max(g, issued - kPipeStages); q < issued; ++q) {
+            bool dok = true;
+            tc::mbar_wait_bounded(bar0 + 8 * (q % kPipeStages), (uint32_t)((q / kPipeStages) & 1), dok,
+                                  limit_ns);
+        }
+        report_status(a.status_dev, kStatusTimeout);
     }
 }
 

@@ -19,29 +19,38 @@
 // The diagonal j = i belongs to M because the output reads the updated state.
 //
 // Work decomposition: one CTA per (sequence, pair of heads of one group),
-// sweeping the sequence's chunks in order.  544 threads: four compute
-// warpgroups and one issuing warp.  Compute warpgroup wg works on head
-// 2k + (wg & 1) and on half (wg >> 1) of the columns: thread i of it owns TMEM
-// lane i (row i of G, M, Y, Yoff; d_state index i of S^T and of the carried
-// state, 32 of whose 64 head_dim entries it keeps in fp32 registers for the
-// whole sequence).  Lane 0 of the issuing warp issues TMA and the MMAs; the
-// products shared by both heads (C.B^T, and B^T or C against the two heads'
-// operands side by side) are single N = 128 MMAs.
+// sweeping the sequence's chunks in order, with three warp roles that work on
+// different chunks at the same time (640 threads, 20 warps):
+//   * compute warpgroups (warps 4-19): head 2k + (wg & 1), column half wg >> 1;
+//     thread i owns TMEM lane i (row i of G, M, Y, Yoff; d_state index i of
+//     S^T and of the carried state, 32 of whose 64 head_dim entries it keeps
+//     in fp32 registers for the whole sequence).  Per chunk: the next chunk's
+//     cumulative decay (published for the converters), state update, decay
+//     mask, new H^T tile, the next chunk's C converted into TMEM (the A
+//     operand of C.B^T and C.H^T, double-buffered), output epilogue;
+//   * converter warps (warps 0-2): one chunk ahead of the compute warps, they
+//     convert the chunk's bf16 B and x tiles to fp16 in place in shared
+//     memory and form the decay-weighted x (w o x) from the published decay;
+//   * issuing warp (warp 3): lane 0 issues the TMA loads and stores and the
+//     MMAs as their operands become ready.
+// Every hand-off between roles is an mbarrier with a bounded wait (no named
+// barrier spans two roles), so a wait that never completes cannot hang the
+// kernel: it raises a CTA-wide abort flag instead.  20 warps keep 5 warps on
+// each SM sub-partition, so every thread gets 96 registers.
 //
-// Pipeline per chunk (single-buffered tiles, with prefetch where a buffer
-// frees early):
-//   wait TMA(x), TMA(B, C) -> convert bf16 -> fp16 (C into TMEM and B in
-//   place, a quarter of d_state per warpgroup; x and w o x per head)
-//   -> issue TMA(x of next chunk) into the raw x buffers
-//   -> MMA S^T (2 heads), G  [commit] , Yoff (2 heads) [commit]
-//   -> the next chunk's cumulative decay (while the MMAs run)
-//   -> issue TMA(B, C of next chunk) once S^T and G are done
-//   -> state update from S^T, decay mask M per head (overlap the Yoff MMAs)
-//   -> MMA Y (2 heads) [commit] -> epilogue y.
+// Per chunk k, the issuing thread runs
+//   S_k = B^T [wX_a|wX_b]  (once Y_{k-1} has read M_{k-1}, whose TMEM S reuses)
+//   G_k = C B^T            (once the epilogue of k-1 has read Y_{k-1})
+//   Yoff_k = C [H_a^T|H_b^T] (once H_{k-1}^T is in shared memory)
+//   Y_k = M_k X_k          (once the mask of chunk k is in TMEM)
+// while the compute warps work through chunk k and the converters prepare
+// chunk k+1.
 //
 // Precision: bf16 inputs are converted to fp16 (exact for |v| < 65504) so the
 // derived operands M, w o x and H (rounded to fp16, 11 significant bits) keep
-// the result within ~3e-4 of the fp64 recurrence; accumulation is fp32.
+// the result within ~3e-4 of the fp64 recurrence; accumulation is fp32.  An
+// operand beyond the fp16 range makes some output non-finite; the epilogue
+// detects that and the kernel reports SSM_ERR_RANGE.
 //
 // Decay factors are never ratios of exponentials.  With block ends r_K =
 // 32K+31, exp(cs_i - cs_j) = exp(cs_i - cs_{r_I}) exp(cs_{r_I} - cs_{r_J})
@@ -61,32 +70,65 @@ namespace {
 constexpr int kQ = 128;       // chunk length
 constexpr int kP = 64;        // head_dim
 constexpr int kN = 128;       // d_state
-constexpr int kThreads = 544;   // 16 compute warps + 1 issuing warp
+constexpr int kConvThreads = 96;       // converter warps 0-2 (lane-free work)
+constexpr int kIssuerBase = 96;        // warp 3
+constexpr int kComputeBase = 128;      // compute warpgroups: warps 4-19
+constexpr int kCompute = 512;
+constexpr int kThreads = kComputeBase + kCompute;      // 640
 
 // Shared memory (bytes from the 1024-aligned dynamic base).  16-bit tiles use
 // the 128B-swizzled layout TMA writes and the MMA descriptors read: rows of 64
 // elements (128 B), 8-row groups of 1024 B, 16-byte chunk c of row r stored at
 // c ^ (r % 8).  128-wide tiles are two 64-column halves 16 KB apart.
 constexpr uint32_t HALF = 16384;
-constexpr uint32_t OFF_C = 0;            // C [128 i][128 n]  bf16 (TMA target; fp16 copy in TMEM)
-constexpr uint32_t OFF_B = 32768;        // B [128 j][128 n]  (bf16 -> fp16 in place)
-constexpr uint32_t OFF_XR = 65536;       // raw x, 2 heads x [128 j][64 p] bf16 (TMA target)
-constexpr uint32_t OFF_XH = 98304;       // x as fp16, 2 heads
-constexpr uint32_t OFF_WM = 131072;      // w o x, 2 heads x [128 j][64 p]
-constexpr uint32_t OFF_MB = 163840;      // y staging, 2 heads x [128 t][64 p] bf16
-constexpr uint32_t OFF_H = 196608;       // H^T fp16, 2 heads x [128 n][64 p]
+constexpr uint32_t OFF_C = 0;            // C [128 i][128 n] bf16 (TMA target; fp16 copy in TMEM)
+constexpr uint32_t OFF_B = 32768;        // B buffer 0 [128 j][128 n] (bf16 -> fp16 in place)
+constexpr uint32_t OFF_X = 65536;        // x, 2 buffers x 2 heads x [128 j][64 p] (bf16 -> fp16 in
+                                         // place; after Y_k, the staging of y_k for its TMA store)
+constexpr uint32_t XBUF = 32768;
+constexpr uint32_t OFF_W = 131072;       // w o x, 2 heads x [128 j][64 p] fp16
+constexpr uint32_t OFF_H = 163840;       // H^T fp16, 2 heads x [128 n][64 p]
+constexpr uint32_t OFF_B1 = 196608;      // B buffer 1
 constexpr uint32_t OFF_MISC = 229376;
-constexpr uint32_t OFF_VD = OFF_MISC;              // float[2 buffers][2 heads][128]
-constexpr uint32_t OFF_CSB = OFF_VD + 2048;        // float[4][8]: block-end cs, cs_last per warpgroup
-constexpr uint32_t OFF_PART = OFF_CSB + 128;       // float[4][4] warp partial sums
-constexpr uint32_t OFF_BAR = OFF_PART + 64;        // 5 mbarriers
-constexpr uint32_t OFF_TM = OFF_BAR + 40;
+constexpr uint32_t OFF_VD = OFF_MISC;              // float[2 buffers][2 heads][128]: column factors vd
+constexpr uint32_t OFF_WF = OFF_VD + 2048;         // float[2 buffers][2 heads][4]: exp(cs_last - cs_{r_J})
+constexpr uint32_t OFF_CSBT = OFF_WF + 64;         // float[2 buffers][2 heads][8]: block-end cs, cs_last
+constexpr uint32_t OFF_CSB = OFF_CSBT + 128;       // float[4][8]: scan scratch per compute warpgroup
+constexpr uint32_t OFF_PART = OFF_CSB + 128;       // float[4][4]: compute warp partial sums
+constexpr uint32_t OFF_BAR = OFF_PART + 64;        // mbarriers (8 B each)
+constexpr uint32_t NBAR = 18;
+constexpr uint32_t OFF_TM = OFF_BAR + 8 * NBAR;    // TMEM base address (4 B)
+constexpr uint32_t OFF_ABORT = OFF_TM + 4;         // CTA-wide abort flag (int)
+constexpr uint32_t OFF_RANGE = OFF_TM + 8;         // set when an output is not finite (int)
 constexpr uint32_t SMEM_BYTES = OFF_TM + 16;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// mbarrier indices (address OFF_BAR + 8 * index).  A barrier that serves
+// alternate chunks (x buffers, converter hand-off, decay tables) comes in a
+// pair indexed by chunk parity, so that no waiter can ever be two phases
+// behind the barrier it waits on.
+enum : uint32_t {
+    BAR_X0 = 0, BAR_X1 = 1,   // x tiles of buffer 0 / 1 landed (TMA)
+    BAR_CT = 2,               // C tile landed (TMA)
+    BAR_BT0 = 3, BAR_BT1 = 4, // B tile of buffer 0 / 1 landed (TMA)
+    BAR_CRAW = 5,             // compute warps have read the C tile (16 warp arrivals)
+    BAR_CV0 = 6, BAR_CV1 = 7, // converters done with a chunk of parity 0 / 1 (3 warp arrivals)
+    BAR_DC0 = 8, BAR_DC1 = 9, // decay tables of a chunk of parity 0 / 1 published (8 warp arrivals)
+    BAR_S = 10,               // S MMAs of a chunk done (commit): w o x may be rewritten
+    BAR_SG = 11,              // S and G MMAs of a chunk done (commit)
+    BAR_YO = 12,              // Yoff MMAs done (commit)
+    BAR_Y = 13,               // Y MMAs done (commit)
+    BAR_MASK = 14,            // decay mask written (16 compute-warp arrivals)
+    BAR_STATE = 15,           // H^T tile written (16 compute-warp arrivals)
+    BAR_EPI = 16,             // epilogue done and next C in TMEM (16 compute-warp arrivals)
+    BAR_DRAIN = 17            // abort path: every issued MMA done (commit)
+};
 
 // TMEM columns (fp32 accumulators, lane = row).
 // G and Y share columns: the y MMAs write Y only after the mask has read G,
 // and the next chunk's G is issued only after the epilogue has read Y.  C
-// (fp16, two values per column) is the TMEM A operand of C.B^T and C.H^T.
+// (fp16, two values per column, double-buffered) is the TMEM A operand of
+// C.B^T and C.H^T.
 constexpr uint32_t TM_G = 0, TM_Y = 0, TM_S = 128, TM_YO = 256, TM_C = 384;
 constexpr uint32_t TM_COLS = 512;
 
@@ -96,6 +138,39 @@ constexpr uint32_t IDESC_YO2 = tc::idesc_f16_f32(128, 128, 0, 1); // C (K-major)
 constexpr uint32_t IDESC_Y = tc::idesc_f16_f32(128, 64, 0, 1);    // M (TMEM) x X (MN-major)
 
 constexpr float kSafeBlockDecay = 80.f;   // max exp argument taken by the factorised path
+
+// Named barriers (never shared between roles): 1..4 per compute warpgroup,
+// 5 all compute warps.
+constexpr uint32_t NB_COMPUTE = 5;
+
+extern __shared__ __align__(1024) uint8_t smem[];
+
+__device__ __forceinline__ volatile int &abort_flag() {
+    return *reinterpret_cast<volatile int *>(smem + OFF_ABORT);
+}
+__device__ __forceinline__ volatile int &range_flag() {
+    return *reinterpret_cast<volatile int *>(smem + OFF_RANGE);
+}
+__device__ __forceinline__ uint64_t wait_limit(unsigned long long wait_ns) {
+    return wait_ns ? wait_ns : kDefaultWaitNs;
+}
+
+// Bounded mbarrier wait: when it expires (or the abort flag is already up)
+// `ok` turns false, the CTA-wide abort flag goes up, and every later wait of
+// this thread returns at once.  The roles then run to the end of their loops
+// without waiting, the issuing thread drains what it has in flight, and the
+// kernel reports SSM_ERR_TIMEOUT.
+__device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, bool &ok,
+                                              unsigned long long wait_ns) {
+    if (ok && abort_flag()) ok = false;
+    if (ok && !tc::mbar_wait_bounded(bar, parity, ok, wait_limit(wait_ns))) abort_flag() = 1;
+}
+
+// One arrival per warp on an mbarrier, after every lane's prior writes.
+__device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(bar);
+}
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
@@ -297,28 +372,33 @@ struct ChunkDecay {
     float cs;        // inclusive cumulative dt*A at row i
     float dtv;       // dt of row i (0 past the chunk end)
     float uaA, uaB;  // exp(cs_i - cs_{r_K}) for this thread's two column blocks
-    float w;         // exp(cs_last - cs_i) dt_i   (weights of the chunk state)
     float e;         // exp(cs_i)                  (decay of the carried state to row i)
     float a_last;    // exp(cs_last)               (decay over the whole chunk)
     bool safe;       // the row block's own decay fits the factorised path
 };
 
 // Raw dt of row i of the chunk starting at c0 (0 past the sequence end t1),
-// loaded ahead of use: the compute loop keeps two chunks of it in flight.
+// loaded ahead of use: the compute and converter loops keep two chunks of it
+// in flight.
 __device__ __forceinline__ float load_dt(const ScanArgs &a, int H, int hh, long c0, long t1, int i) {
     return (c0 + i < t1) ? __ldg(a.dt + (size_t)(c0 + i) * H + hh) : 0.f;
 }
 
 // Cumulative decay of head hh over a chunk of Lc tokens whose raw dt for row
-// i is dt_raw (warpgroup-wide), and this warpgroup's share of the column
-// factors vd, written to vd_out (only the warpgroup with ch == 0 writes).
-__device__ __forceinline__ ChunkDecay chunk_decay(const ScanArgs &a, int hh, float Ah, float dt_raw,
-                                                  int Lc, int i, int wq, int lane, int wg,
-                                                  int ch, float *sPART, float *sCSB, float *vd_out)
+// i is dt_raw (warpgroup-wide); returns (cs_i, dt_i).  The warpgroup with
+// ch == 0 publishes the chunk's tables, read later by the compute warps
+// (decay_derive, the mask) and by the converters (w o x):
+//   vd[j]   = exp(cs_{r_J} - cs_j) dt_j, J = j's 32-row block (column factors)
+//   wf[J]   = exp(cs_last - cs_{r_J})      (so the chunk-state weight is
+//                                          w_j = wf[J] vd_j: two factors <= 1)
+//   csb[J]  = cs_{r_J} (J < 4), csb[4] = cs_last
+__device__ __forceinline__ float2 decay_scan(const ScanArgs &a, int hh, float Ah, float dt_raw,
+                                             int Lc, int i, int wq, int lane, int wg, int ch,
+                                             float *sPART, float *sCSB, float *vd_out,
+                                             float *wf_out, float *csb_out)
 {
-    ChunkDecay d;
-    d.dtv = (i < Lc) ? dt_apply(a.dtp, dt_raw, hh) : 0.f;
-    float v = d.dtv * Ah;
+    const float dtv = (i < Lc) ? dt_apply(a.dtp, dt_raw, hh) : 0.f;
+    float v = dtv * Ah;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const float u = __shfl_up_sync(0xffffffffu, v, o);
@@ -328,28 +408,33 @@ __device__ __forceinline__ ChunkDecay chunk_decay(const ScanArgs &a, int hh, flo
     wg_sync(wg);
     float pre = 0.f;
     for (int w = 0; w < wq; ++w) pre += sPART[w];
-    d.cs = v + pre;
-    if (lane == 31) sCSB[wq] = d.cs;
-    if (i == Lc - 1) sCSB[4] = d.cs;
+    const float cs = v + pre;
+    if (lane == 31) sCSB[wq] = cs;
+    if (i == Lc - 1) sCSB[4] = cs;
     wg_sync(wg);
-    const float cs_last = sCSB[4];
-    const float cs_own_end = sCSB[wq];
-    d.safe = (__shfl_sync(0xffffffffu, d.cs, 0) - cs_own_end) <= kSafeBlockDecay;
-    const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
-    d.uaA = (kA <= wq) ? exp_dec(d.cs - sCSB[kA]) : 0.f;
-    d.uaB = (kB <= wq) ? exp_dec(d.cs - sCSB[kB]) : 0.f;
-    if (ch == 0) vd_out[i] = exp_dec(cs_own_end - d.cs) * d.dtv;   // <= dt
-    d.w = (i < Lc) ? exp_dec(cs_last - d.cs) * d.dtv : 0.f;
-    d.e = exp_dec(d.cs);
-    d.a_last = exp_dec(cs_last);
-    return d;
+    if (ch == 0) {
+        const float cs_last = sCSB[4];
+        vd_out[i] = exp_dec(sCSB[wq] - cs) * dtv;   // <= dt
+        if (i < 4) wf_out[i] = exp_dec(cs_last - sCSB[i]);
+        if (i < 5) csb_out[i] = sCSB[i];
+    }
+    return make_float2(cs, dtv);
 }
 
-// Named barriers: 1..4 per-warpgroup; the compute warps signal the issuing
-// warp with bar.arrive on 5 (operands ready), 6 (decay mask ready) and 7 (y
-// staged); 8 is compute-warps-only.
-constexpr uint32_t BAR_OPERANDS = 5, BAR_MASK = 6, BAR_YSTAGED = 7, BAR_COMPUTE = 8;
-constexpr uint32_t kCompute = 512;
+// The per-row decay quantities of ChunkDecay from row i's (cs, dt) and the
+// chunk's published block ends csb.
+__device__ __forceinline__ ChunkDecay decay_derive(float2 csdt, const float *csb, int wq, int ch) {
+    ChunkDecay d;
+    d.cs = csdt.x;
+    d.dtv = csdt.y;
+    const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
+    d.uaA = (kA <= wq) ? exp_dec(d.cs - csb[kA]) : 0.f;
+    d.uaB = (kB <= wq) ? exp_dec(d.cs - csb[kB]) : 0.f;
+    d.safe = (__shfl_sync(0xffffffffu, d.cs, 0) - csb[wq]) <= kSafeBlockDecay;
+    d.e = exp_dec(d.cs);
+    d.a_last = exp_dec(csb[4]);
+    return d;
+}
 
 template <typename TOut>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -357,19 +442,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y,
                const ScanArgs a)
 {
-    // bf16 y of full chunks is staged in shared memory (the M tile of head 1,
-    // free between the y MMAs and the next chunk's mask) and written by TMA;
+    // bf16 y of full chunks is staged in shared memory and written by TMA;
     // fp32 y and partial chunks are stored row by row.
     constexpr bool kStoreByTma = sizeof(TOut) == 2;
-    extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = tc::smem_u32(smem);
     const int tid = threadIdx.x;
-    const bool issuer = tid >= (int)kCompute;  // warp 16: TMA and MMA issue
-    const int wg = (tid >> 7) & 3;       // compute warpgroup 0..3
-    const int hd = wg & 1;               // head slot of the pair
-    const int ch = wg >> 1;              // column half
-    const int i = tid & 127;             // row / TMEM lane / d_state index
-    const int wq = i >> 5;               // warp within the warpgroup = 32-row block
     const int lane = tid & 31;
 
     const int H = a.nheads, G = a.ngroups;
@@ -378,10 +455,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     const int s = blockIdx.x / pairs;
     const int h0 = (blockIdx.x - s * pairs) * 2;
     const int g = h0 / hpg;
-    const int hh = h0 + hd;
 
     if (sbase & 1023u) {                 // the swizzled layouts need 1024-B alignment
-        if (tid == 0) report_status(a.status_dev, 5);
+        if (tid == 0) report_status(a.status_dev, kStatusInternal);
         return;
     }
 
@@ -390,41 +466,55 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         const int c0 = a.cu_seqlens[0], cs0 = a.cu_seqlens[s], cs1 = a.cu_seqlens[s + 1];
         const int cend = a.cu_seqlens[a.nseq];
         if (c0 != 0 || cs1 < cs0 || cs0 < 0 || cend != a.seqlen || cs1 > a.seqlen) {
-            if (tid == 0) report_status(a.status_dev, 6);
+            if (tid == 0) report_status(a.status_dev, kStatusDeviceInput);
             return;
         }
         t0 = cs0; t1 = cs1;
     } else {
         t0 = (long)s * a.seqlen; t1 = t0 + a.seqlen;
     }
+    const int nch = (int)((t1 - t0 + kQ - 1) / kQ);   // chunks of this sequence
 
     size_t srow = (size_t)s;   // state row of this sequence
     bool load_init = a.initial_state != nullptr;
     if (a.slot_idx) {
         const int slot = a.slot_idx[s];
         if (slot < 0 || slot >= a.max_slots) {
-            if (tid == 0) report_status(a.status_dev, 6);
+            if (tid == 0) report_status(a.status_dev, kStatusDeviceInput);
             return;
         }
         srow = (size_t)slot;
         if (a.has_initial && a.has_initial[s] == 0) load_init = false;
     }
 
-    float *sCSB = reinterpret_cast<float *>(smem + OFF_CSB) + wg * 8;
-    float *sPART = reinterpret_cast<float *>(smem + OFF_PART) + wg * 4;
-    const uint32_t bar_x = sbase + OFF_BAR, bar_cb = bar_x + 8, bar_sg = bar_x + 16;
-    const uint32_t bar_yo = bar_x + 24, bar_y = bar_x + 32;
+    const uint32_t bar0 = sbase + OFF_BAR;
+    auto bar = [&](uint32_t idx) { return bar0 + 8u * idx; };
 
     if (tid < 32) {
         tc::tmem_alloc(sbase + OFF_TM, TM_COLS);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(bar_x, 1);
-        tc::mbar_init(bar_cb, 1);
-        tc::mbar_init(bar_sg, 1);
-        tc::mbar_init(bar_yo, 1);
-        tc::mbar_init(bar_y, 1);
+        tc::mbar_init(bar(BAR_X0), 1);
+        tc::mbar_init(bar(BAR_X1), 1);
+        tc::mbar_init(bar(BAR_CT), 1);
+        tc::mbar_init(bar(BAR_BT0), 1);
+        tc::mbar_init(bar(BAR_BT1), 1);
+        tc::mbar_init(bar(BAR_S), 1);
+        tc::mbar_init(bar(BAR_CRAW), 16);
+        tc::mbar_init(bar(BAR_CV0), 3);
+        tc::mbar_init(bar(BAR_CV1), 3);
+        tc::mbar_init(bar(BAR_DC0), 8);
+        tc::mbar_init(bar(BAR_DC1), 8);
+        tc::mbar_init(bar(BAR_SG), 1);
+        tc::mbar_init(bar(BAR_YO), 1);
+        tc::mbar_init(bar(BAR_Y), 1);
+        tc::mbar_init(bar(BAR_MASK), 16);
+        tc::mbar_init(bar(BAR_STATE), 16);
+        tc::mbar_init(bar(BAR_EPI), 16);
+        tc::mbar_init(bar(BAR_DRAIN), 1);
+        abort_flag() = 0;
+        range_flag() = 0;
         tc::fence_mbar_init();
     }
     tc::tc_fence_before();
@@ -432,185 +522,306 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     tc::tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_TM);
     bool ok = true;
+    float *vd_tab = reinterpret_cast<float *>(smem + OFF_VD);   // [2 buffers][2 heads][128]
+    float *wf_tab = reinterpret_cast<float *>(smem + OFF_WF);   // [2 buffers][2 heads][4]
 
-    if (issuer) {
-        // ================= TMA / MMA issuing warp =================
-        const bool leader = lane == 0;
-        // descriptors (start-address field advanced by offset >> 4 per K step)
-        const uint64_t dBmn = tc::sdesc_sw128(sbase + OFF_B, HALF, 1024);   // B^T, MN-major
-        const uint64_t dW = tc::sdesc_sw128(sbase + OFF_WM, HALF, 1024);    // [wX_a | wX_b]
-        const uint64_t dBk = tc::sdesc_sw128(sbase + OFF_B, 16, 1024);      // B, K-major
-        const uint64_t dH = tc::sdesc_sw128(sbase + OFF_H, HALF, 1024);     // [H_a^T | H_b^T]
-        const uint64_t dXa = tc::sdesc_sw128(sbase + OFF_XH, HALF, 1024);
-        const uint64_t dXb = dXa + (HALF >> 4);
-        if (leader && t1 > t0) {
-            tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
-            tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, h0, (int)t0);
-            tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, h0 + 1, (int)t0);
-            tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
-            tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)t0);
-            tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, g, (int)t0);
-            tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)t0);
-            tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)t0);
-        }
-        uint32_t phase = 0;
-        for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u) {
-            const long c1 = c0 + kQ;
-            const bool has_next = c1 < t1;
-            tc::named_sync(BAR_OPERANDS, kCompute + 32);
-            if (leader) {
-                tc::bulk_wait_read();   // previous y staging (in the M tiles) was read
-                if (has_next) {
-                    tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
-                    tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, h0, (int)c1);
-                    tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, h0 + 1, (int)c1);
-                }
-                tc::tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16_ss(tmem + TM_S, dBmn + kk * 128, dW + kk * 128, IDESC_S2, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
-                    tc::mma_f16_ts(tmem + TM_G, tmem + TM_C + kk * 8, dBk + ko, IDESC_G, kk > 0);
-                }
-                tc::mma_commit(bar_sg);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16_ts(tmem + TM_YO, tmem + TM_C + kk * 8, dH + kk * 128, IDESC_YO2, kk > 0);
-                tc::mma_commit(bar_yo);
-                // The compute warps read C from shared memory before the operand
-                // barrier; B is read by the S and G MMAs only: both tiles are free
-                // once those complete.
-                tc::mbar_wait_bounded(bar_sg, phase, ok);
-                if (has_next) {
-                    tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
-                    tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, g, (int)c1);
-                    tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, g, (int)c1);
-                    tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, g, (int)c1);
-                    tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, g, (int)c1);
-                }
-            }
-            __syncwarp();
-            tc::named_sync(BAR_MASK, kCompute + 32);
-            if (leader) {
-                tc::tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16_ts(tmem + TM_Y, tmem + TM_S + kk * 8, dXa + kk * 128, IDESC_Y, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_f16_ts(tmem + TM_Y + 64, tmem + TM_S + 64 + kk * 8, dXb + kk * 128, IDESC_Y, kk > 0);
-                tc::mma_commit(bar_y);
-            }
-            __syncwarp();
-            tc::named_sync(BAR_YSTAGED, kCompute + 32);
-            if (kStoreByTma && leader && c1 <= t1) {   // full chunk: both heads' y tiles by TMA
-                tc::tma_store_3d(&map_y, sbase + OFF_MB, 0, h0, (int)c0);
-                tc::tma_store_3d(&map_y, sbase + OFF_MB + HALF, 0, h0 + 1, (int)c0);
+    if (tid >= kIssuerBase && tid < kComputeBase) {
+        // ================= TMA / MMA issuing thread =================
+        if (lane == 0) {
+            const bool produce = a.stall_producer == 0;
+            // Work in flight, for the drain after an abort: phases armed on the
+            // TMA barriers, and whether any MMA was issued.
+            uint32_t armed_x[2] = {0, 0}, armed_b[2] = {0, 0}, armed_c = 0;
+            bool mma_issued = false;
+            auto tile_row = [&](int k) { return (int)(t0 + (long)k * kQ); };
+            auto load_x = [&](int k) {
+                const uint32_t b = (uint32_t)k & 1u;
+                tc::mbar_arrive_expect_tx(bar(BAR_X0 + b), 2 * HALF);
+                tc::tma_load_3d(sbase + OFF_X + b * XBUF, &map_x, bar(BAR_X0 + b), 0, h0, tile_row(k));
+                tc::tma_load_3d(sbase + OFF_X + b * XBUF + HALF, &map_x, bar(BAR_X0 + b), 0, h0 + 1, tile_row(k));
+                ++armed_x[b];
+            };
+            auto load_c = [&](int k) {
+                tc::mbar_arrive_expect_tx(bar(BAR_CT), 2 * HALF);
+                tc::tma_load_3d(sbase + OFF_C, &map_c, bar(BAR_CT), 0, g, tile_row(k));
+                tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar(BAR_CT), 64, g, tile_row(k));
+                ++armed_c;
+            };
+            auto load_b = [&](int k) {
+                const uint32_t b = (uint32_t)k & 1u;
+                const uint32_t dst = b ? sbase + OFF_B1 : sbase + OFF_B;
+                tc::mbar_arrive_expect_tx(bar(BAR_BT0 + b), 2 * HALF);
+                tc::tma_load_3d(dst, &map_b, bar(BAR_BT0 + b), 0, g, tile_row(k));
+                tc::tma_load_3d(dst + HALF, &map_b, bar(BAR_BT0 + b), 64, g, tile_row(k));
+                ++armed_b[b];
+            };
+            auto store_y = [&](int k) {   // y tiles of full chunk k, staged in its x buffer
+                const uint32_t src = sbase + OFF_X + ((uint32_t)k & 1u) * XBUF;
+                tc::tma_store_3d(&map_y, src, 0, h0, tile_row(k));
+                tc::tma_store_3d(&map_y, src + HALF, 0, h0 + 1, tile_row(k));
                 tc::bulk_commit();
+            };
+            if (produce && nch > 0) {
+                load_c(0);
+                load_x(0);
+                load_b(0);
+                if (nch > 1) {
+                    load_x(1);
+                    load_b(1);
+                }
+                wait_or_abort(bar(BAR_CRAW), 0, ok, a.wait_ns);   // compute warps read C_0
+                if (ok && nch > 1) load_c(1);
             }
-            __syncwarp();
+            for (int k = 0; k < nch && produce && ok; ++k) {
+                const uint32_t b = (uint32_t)k & 1u;
+                const uint32_t ph = (uint32_t)k & 1u;
+                // chunk k converted (B and x in fp16, w o x)
+                wait_or_abort(bar(BAR_CV0 + b), ((uint32_t)k >> 1) & 1u, ok, a.wait_ns);
+                // S_k overwrites TMEM that held M_{k-1}: Y_{k-1} must be done
+                if (k > 0) wait_or_abort(bar(BAR_Y), ph ^ 1u, ok, a.wait_ns);
+                if (!ok) break;
+                tc::tc_fence_after();
+                const uint32_t sB = b ? sbase + OFF_B1 : sbase + OFF_B;
+                {
+                    const uint64_t dBmn = tc::sdesc_sw128(sB, HALF, 1024);               // B^T, MN-major
+                    const uint64_t dW = tc::sdesc_sw128(sbase + OFF_W, HALF, 1024);    // [wX_a | wX_b]
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_f16_ss(tmem + TM_S, dBmn + kk * 128, dW + kk * 128, IDESC_S2, kk > 0);
+                }
+                tc::mma_commit(bar(BAR_S));
+                mma_issued = true;
+                // G_k overwrites Y_{k-1}, Yoff_k overwrites Yoff_{k-1}, and G_k needs C_k
+                // in TMEM: the epilogue of k-1 (which converts C_k) must be done
+                wait_or_abort(bar(BAR_EPI), ph, ok, a.wait_ns);
+                if (!ok) break;
+                if (k > 0 && kStoreByTma) store_y(k - 1);   // chunk k-1 is full (chunk k follows it)
+                tc::tc_fence_after();
+                const uint32_t tC = tmem + TM_C + 64u * b;
+                {
+                    const uint64_t dBk = tc::sdesc_sw128(sB, 16, 1024);                  // B, K-major
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
+                        tc::mma_f16_ts(tmem + TM_G, tC + kk * 8, dBk + ko, IDESC_G, kk > 0);
+                    }
+                }
+                tc::mma_commit(bar(BAR_SG));
+                // x of chunk k+1 into the buffer of chunk k-1, once Y_{k-1} has read
+                // x_{k-1} and the store of y_{k-1} (staged there) has read it
+                if (k > 0 && k + 1 < nch) {
+                    tc::bulk_wait_read();
+                    load_x(k + 1);
+                }
+                // Yoff_k reads H_{k-1}^T (the initial state's for k = 0)
+                wait_or_abort(bar(BAR_STATE), ph, ok, a.wait_ns);
+                if (!ok) break;
+                tc::tc_fence_after();
+                {
+                    const uint64_t dH = tc::sdesc_sw128(sbase + OFF_H, HALF, 1024);     // [H_a^T | H_b^T]
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_f16_ts(tmem + TM_YO, tC + kk * 8, dH + kk * 128, IDESC_YO2, kk > 0);
+                }
+                tc::mma_commit(bar(BAR_YO));
+                // B of chunk k+2 into this buffer once S_k and G_k have read B_k
+                wait_or_abort(bar(BAR_SG), ph, ok, a.wait_ns);
+                if (!ok) break;
+                if (k + 2 < nch) load_b(k + 2);
+                // Y_k needs the mask
+                wait_or_abort(bar(BAR_MASK), ph, ok, a.wait_ns);
+                if (!ok) break;
+                tc::tc_fence_after();
+                {
+                    const uint64_t dX = tc::sdesc_sw128(sbase + OFF_X + b * XBUF, HALF, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_f16_ts(tmem + TM_Y, tmem + TM_S + kk * 8, dX + kk * 128, IDESC_Y, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_f16_ts(tmem + TM_Y + 64, tmem + TM_S + 64 + kk * 8,
+                                       dX + (HALF >> 4) + kk * 128, IDESC_Y, kk > 0);
+                }
+                tc::mma_commit(bar(BAR_Y));
+                // C of chunk k+2 once the compute warps have read C_{k+1}
+                if (k + 2 < nch) {
+                    wait_or_abort(bar(BAR_CRAW), ((uint32_t)k + 1u) & 1u, ok, a.wait_ns);
+                    if (!ok) break;
+                    load_c(k + 2);
+                }
+            }
+            // y of the last chunk
+            if (ok && produce && nch > 0) {
+                wait_or_abort(bar(BAR_EPI), (uint32_t)nch & 1u, ok, a.wait_ns);
+                if (ok && kStoreByTma && t0 + (long)nch * kQ <= t1) store_y(nch - 1);
+            }
+            if (!ok) {
+                // Aborted: wait (bounded) for every MMA issued and for the last
+                // phase armed on each load barrier, so that nothing writes TMEM
+                // or shared memory after they are released.
+                const uint64_t lim = wait_limit(a.wait_ns);
+                bool dok = true;
+                if (mma_issued) {
+                    tc::mma_commit(bar(BAR_DRAIN));
+                    tc::mbar_wait_bounded(bar(BAR_DRAIN), 0, dok, lim);
+                }
+                for (int b = 0; b < 2; ++b) {
+                    bool xok = true;
+                    if (armed_x[b]) tc::mbar_wait_bounded(bar(BAR_X0 + b), (armed_x[b] - 1) & 1u, xok, lim);
+                }
+                for (int b = 0; b < 2; ++b) {
+                    bool bok = true;
+                    if (armed_b[b]) tc::mbar_wait_bounded(bar(BAR_BT0 + b), (armed_b[b] - 1) & 1u, bok, lim);
+                }
+                bool cok = true;
+                if (armed_c) tc::mbar_wait_bounded(bar(BAR_CT), (armed_c - 1) & 1u, cok, lim);
+            }
+            tc::bulk_wait_all();
         }
-        if (leader) tc::bulk_wait_all();
         __syncwarp();
-    } else {
+    } else if (tid < kConvThreads) {
+        // ================= converter warps: one chunk ahead =================
+        // 4096 jobs of one 16-byte chunk (8 values) per tile row: jobs 0..2047
+        // are x (head, row, chunk): x -> fp16 in place and w o x; jobs
+        // 2048..4095 are B (half, row, chunk) -> fp16 in place.  Thread t takes
+        // jobs t, t + 96, ...; a warp's 32 consecutive jobs cover 4 whole rows,
+        // so its 16-byte accesses hit every bank once per 128 bytes.
+        for (int k = 0; k < nch; ++k) {
+            const uint32_t b = (uint32_t)k & 1u;
+            const long c0 = t0 + (long)k * kQ;
+            const int Lc = (int)min((long)kQ, t1 - c0);
+            const uint32_t xt = sbase + OFF_X + b * XBUF;
+            wait_or_abort(bar(BAR_X0 + b), ((uint32_t)k >> 1) & 1u, ok, a.wait_ns);
+            wait_or_abort(bar(BAR_DC0 + b), ((uint32_t)k >> 1) & 1u, ok, a.wait_ns);
+            // w o x overwrites the tile S_{k-1} read
+            if (k >= 1) wait_or_abort(bar(BAR_S), ((uint32_t)k - 1u) & 1u, ok, a.wait_ns);
+            const float *vd = vd_tab + b * 256;
+            const float *wf = wf_tab + b * 8;
+#pragma unroll 4
+            for (int j = tid; j < 2048; j += kConvThreads) {
+                const int hd = j >> 10, row = (j >> 3) & 127, q = j & 7;
+                const uint32_t off = hd * HALF + sw128(row, q);
+                if (row < Lc) {
+                    const float w = wf[hd * 4 + (row >> 5)] * vd[hd * 128 + row];
+                    const uint4 v = lds128(xt + off);
+                    sts128(xt + off, cvt_chunk(v));
+                    sts128(sbase + OFF_W + off, cvt_chunk_scaled(v, w));
+                } else {
+                    sts128(xt + off, make_uint4(0, 0, 0, 0));
+                    sts128(sbase + OFF_W + off, make_uint4(0, 0, 0, 0));
+                }
+            }
+            wait_or_abort(bar(BAR_BT0 + b), ((uint32_t)k >> 1) & 1u, ok, a.wait_ns);
+            const uint32_t bt = b ? sbase + OFF_B1 : sbase + OFF_B;
+#pragma unroll 4
+            for (int j = tid; j < 2048; j += kConvThreads) {
+                const int hf = j >> 10, row = (j >> 3) & 127, q = j & 7;
+                const uint32_t addr = bt + hf * HALF + sw128(row, q);
+                sts128(addr, row < Lc ? cvt_chunk(lds128(addr)) : make_uint4(0, 0, 0, 0));
+            }
+            tc::fence_proxy_async_smem();
+            warp_arrive(bar(BAR_CV0 + b), lane);
+        }
+    } else if (tid >= kComputeBase) {
         // ================= compute warpgroups =================
+        const int ctid = tid - kComputeBase;
+        const int wg = ctid >> 7;            // compute warpgroup 0..3
+        const int hd = wg & 1;               // head slot of the pair
+        const int ch = wg >> 1;              // column half
+        const int i = ctid & 127;            // row / TMEM lane / d_state index
+        const int wq = i >> 5;               // warp within the warpgroup = 32-row block
+        const int hh = h0 + hd;
         const uint32_t tlane = (uint32_t)(wq * 32) << 16;
+        float *sCSB = reinterpret_cast<float *>(smem + OFF_CSB) + wg * 8;
+        float *sPART = reinterpret_cast<float *>(smem + OFF_PART) + wg * 4;
         const size_t state_off = (srow * H + hh) * (size_t)(kP * kN) + (size_t)(32 * ch) * kN + i;
+
+        // Row i's quarter wg of C_k (d_state n in [32 wg, 32 wg + 32)) as fp16
+        // pairs into TMEM C[k & 1] (lane i, columns 16 wg ..): the A operand
+        // of C.B^T and C.H^T.  Rows past the chunk end are zero.
+        auto convert_c = [&](int k) {
+            const long ck = t0 + (long)k * kQ;
+            const bool live_c = i < (int)min((long)kQ, t1 - ck);
+            wait_or_abort(bar(BAR_CT), (uint32_t)k & 1u, ok, a.wait_ns);
+            const uint32_t ctile = sbase + OFF_C + (wg >> 1) * HALF;
+            uint4 v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                v[q] = live_c ? lds128(ctile + sw128(i, 4 * (wg & 1) + q)) : make_uint4(0, 0, 0, 0);
+            warp_arrive(bar(BAR_CRAW), lane);   // the C tile may be reloaded
+            uint32_t pc[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 u = cvt_chunk(v[q]);
+                pc[4 * q] = u.x; pc[4 * q + 1] = u.y; pc[4 * q + 2] = u.z; pc[4 * q + 3] = u.w;
+            }
+            tc::tmem_st16(tmem + tlane + TM_C + 64u * ((uint32_t)k & 1u) + 16 * wg, pc);
+            tc::tmem_st_wait();
+        };
+
         float Hs[32];
 #pragma unroll
         for (int p = 0; p < 32; ++p)
             Hs[p] = load_init ? state_load1(a.initial_state, state_off + (size_t)p * kN, a.rp) : 0.f;
         write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+        tc::fence_proxy_async_smem();
+        warp_arrive(bar(BAR_STATE), lane);     // H_{-1}^T ready for Yoff_0
 
         const float Ah = a.A[hh];
         const float Dh = a.D ? a.D[hh] : 0.f;
         TOut *y = static_cast<TOut *>(a.y);
-        float *vd_tab = reinterpret_cast<float *>(smem + OFF_VD);   // [2 buffers][2 heads][128]
-        ChunkDecay cur{};
-        if (t1 > t0)
-            cur = chunk_decay(a, hh, Ah, load_dt(a, H, hh, t0, t1, i), (int)min((long)kQ, t1 - t0),
-                              i, wq, lane, wg, ch, sPART, sCSB, vd_tab + hd * 128);
+        float *csb_tab = reinterpret_cast<float *>(smem + OFF_CSBT);   // [2 buffers][2 heads][8]
+        float2 cs_cur = make_float2(0.f, 0.f);   // (cs_i, dt_i) of the current chunk
+        if (nch > 0) {
+            convert_c(0);
+            tc::tc_fence_before();
+            warp_arrive(bar(BAR_EPI), lane);   // C_0 in TMEM for G_0
+            cs_cur = decay_scan(a, hh, Ah, load_dt(a, H, hh, t0, t1, i), (int)min((long)kQ, t1 - t0),
+                                i, wq, lane, wg, ch, sPART, sCSB, vd_tab + hd * 128, wf_tab + hd * 4,
+                                csb_tab + hd * 8);
+            if (ch == 0) warp_arrive(bar(BAR_DC0), lane);
+        }
+        tc::named_sync(NB_COMPUTE, kCompute);   // chunk 0's tables visible to every compute warp
         float dt_n1 = load_dt(a, H, hh, t0 + kQ, t1, i);   // raw dt of the next chunk
-        tc::named_sync(BAR_COMPUTE, kCompute);
-        uint32_t phase = 0, vb = 0;
-        for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u, vb ^= 1u) {
+        for (int k = 0; k < nch; ++k) {
+            const uint32_t ph = (uint32_t)k & 1u, vb = (uint32_t)k & 1u;
+            const long c0 = t0 + (long)k * kQ;
             const int Lc = (int)min((long)kQ, t1 - c0);
             const long c1 = c0 + kQ;
             const bool has_next = c1 < t1;
             const bool live = i < Lc;
-
             // dt two chunks ahead, so its load has a whole chunk to land
             const float dt_n2 = load_dt(a, H, hh, c0 + 2 * kQ, t1, i);
 
-            // ---- operands to fp16 (rows past the chunk end zeroed) ----
-            tc::mbar_wait_bounded(bar_x, phase, ok);
-            tc::mbar_wait_bounded(bar_cb, phase, ok);
-            {
-                // warpgroup wg takes d_state columns n in [32 wg, 32 wg + 32) of row i:
-                // C as fp16 pairs into TMEM (lane i, columns 16 wg ..), B in place
-                const uint32_t ctile = sbase + OFF_C + (wg >> 1) * HALF;
-                const uint32_t btile = sbase + OFF_B + (wg >> 1) * HALF;
-                uint32_t pc[16];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 v = live ? cvt_chunk(lds128(ctile + sw128(i, 4 * (wg & 1) + q)))
-                                         : make_uint4(0, 0, 0, 0);
-                    pc[4 * q] = v.x;
-                    pc[4 * q + 1] = v.y;
-                    pc[4 * q + 2] = v.z;
-                    pc[4 * q + 3] = v.w;
-                }
-                tc::tmem_st16(tmem + tlane + TM_C + 16 * wg, pc);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t addr = btile + sw128(i, 4 * (wg & 1) + q);
-                    sts128(addr, live ? cvt_chunk(lds128(addr)) : make_uint4(0, 0, 0, 0));
-                }
-#pragma unroll
-                for (int k = 4 * ch; k < 4 * ch + 4; ++k) {
-                    const uint32_t off = hd * HALF + sw128(i, k);
-                    if (live) {
-                        const uint4 r = lds128(sbase + OFF_XR + off);
-                        sts128(sbase + OFF_XH + off, cvt_chunk(r));
-                        sts128(sbase + OFF_WM + off, cvt_chunk_scaled(r, cur.w));
-                    } else {
-                        sts128(sbase + OFF_XH + off, make_uint4(0, 0, 0, 0));
-                        sts128(sbase + OFF_WM + off, make_uint4(0, 0, 0, 0));
-                    }
-                }
+            const ChunkDecay cur = decay_derive(cs_cur, csb_tab + vb * 16 + hd * 8, wq, ch);
+            // ---- next chunk's decay, published for the converters (while S_k, G_k run) ----
+            float2 cs_nxt = make_float2(0.f, 0.f);
+            if (has_next) {
+                cs_nxt = decay_scan(a, hh, Ah, dt_n1, (int)min((long)kQ, t1 - c1), i, wq, lane, wg, ch,
+                                    sPART, sCSB, vd_tab + (vb ^ 1u) * 256 + hd * 128,
+                                    wf_tab + (vb ^ 1u) * 8 + hd * 4, csb_tab + (vb ^ 1u) * 16 + hd * 8);
+                if (ch == 0) warp_arrive(bar(BAR_DC0 + (vb ^ 1u)), lane);
             }
-            tc::tmem_st_wait();
-            tc::fence_proxy_async_smem();
-            tc::tc_fence_before();
-            tc::named_arrive(BAR_OPERANDS, kCompute + 32);
-
-            // ---- next chunk's decay while the MMAs run ----
-            ChunkDecay nxt{};
-            if (has_next)
-                nxt = chunk_decay(a, hh, Ah, dt_n1, (int)min((long)kQ, t1 - c1), i, wq, lane, wg, ch,
-                                  sPART, sCSB, vd_tab + (vb ^ 1u) * 256 + hd * 128);
 
             // ---- carried state: H <- exp(cs_L) H + S (d_state row i, p half ch) ----
-            tc::mbar_wait_bounded(bar_sg, phase, ok);
+            wait_or_abort(bar(BAR_SG), ph, ok, a.wait_ns);
             tc::tc_fence_after();
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                uint32_t r[16];
-                tc::tmem_ld16(tmem + tlane + TM_S + hd * 64 + ch * 32 + q * 16, r);
+                uint32_t rr[16];
+                tc::tmem_ld16(tmem + tlane + TM_S + hd * 64 + ch * 32 + q * 16, rr);
                 tc::tmem_ld_wait();
                 const float2 al2 = make_float2(cur.a_last, cur.a_last);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float2 h2 = __ffma2_rn(al2, make_float2(Hs[q * 16 + 2 * e], Hs[q * 16 + 2 * e + 1]),
-                                                 make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])));
+                                                 make_float2(__uint_as_float(rr[2 * e]), __uint_as_float(rr[2 * e + 1])));
                     Hs[q * 16 + 2 * e] = h2.x;
                     Hs[q * 16 + 2 * e + 1] = h2.y;
                 }
             }
             tc::tc_fence_before();
-            tc::named_sync(BAR_COMPUTE, kCompute);   // every S column read: M may overwrite them
+            tc::named_sync(NB_COMPUTE, kCompute);   // every S column read: M may overwrite them
             tc::tc_fence_after();
 
             // ---- decay mask M of head hd into TMEM (over S of this head) ----
@@ -623,14 +834,19 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 tc::tmem_st_wait();
             }
             tc::tc_fence_before();
-            tc::named_arrive(BAR_MASK, kCompute + 32);
+            warp_arrive(bar(BAR_MASK), lane);
 
-            // ---- new H^T tile for the next chunk (Yoff of this chunk read the old one) ----
-            tc::mbar_wait_bounded(bar_yo, phase, ok);
+            // ---- new H^T tile for the next chunk (Yoff_k read the old one) ----
+            wait_or_abort(bar(BAR_YO), ph, ok, a.wait_ns);
             write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+            tc::fence_proxy_async_smem();
+            warp_arrive(bar(BAR_STATE), lane);
+
+            // ---- C of the next chunk into TMEM (while the y MMAs run) ----
+            if (has_next) convert_c(k + 1);
 
             // ---- y = Y + exp(cs_i) Yoff (row i, p half ch; D x is inside Y) ----
-            tc::mbar_wait_bounded(bar_y, phase, ok);
+            wait_or_abort(bar(BAR_Y), ph, ok, a.wait_ns);
             tc::tc_fence_after();
 #pragma unroll
             for (int q = 0; q < 2; ++q) {   // 16 columns at a time
@@ -640,23 +856,26 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 tc::tmem_ld_wait();
                 float out[16];
                 const float2 e2 = make_float2(cur.e, cur.e);
+                float2 ysum = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const float2 o2 = __ffma2_rn(e2, make_float2(__uint_as_float(ro[2 * c]), __uint_as_float(ro[2 * c + 1])),
                                                  make_float2(__uint_as_float(ry[2 * c]), __uint_as_float(ry[2 * c + 1])));
                     out[2 * c] = o2.x;
                     out[2 * c + 1] = o2.y;
+                    ysum = __fadd2_rn(ysum, o2);
                 }
-                if (kStoreByTma && Lc == kQ) {
-                    stage16_bf16(sbase + OFF_MB + hd * HALF, i, 4 * ch + 2 * q, out);
+                if (!isfinite(ysum.x + ysum.y)) range_flag() = 1;
+                if (kStoreByTma && Lc == kQ) {   // into x_k's buffer: Y_k has read it
+                    stage16_bf16(sbase + OFF_X + vb * XBUF + hd * HALF, i, 4 * ch + 2 * q, out);
                 } else if (live) {
                     store16(y + ((size_t)(c0 + i) * H + hh) * kP + 32 * ch + 16 * q, out);
                 }
             }
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
-            tc::named_arrive(BAR_YSTAGED, kCompute + 32);
-            cur = nxt;
+            warp_arrive(bar(BAR_EPI), lane);
+            cs_cur = cs_nxt;
             dt_n1 = dt_n2;
         }
         if (a.final_state) {
@@ -670,7 +889,11 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, TM_COLS);
     }
-    if (!ok) report_status(a.status_dev, 5);
+    if (abort_flag()) {
+        if (tid == 0) report_status(a.status_dev, kStatusTimeout);
+    } else if (tid == 0 && range_flag()) {
+        report_status(a.status_dev, kStatusRange);
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -724,7 +947,7 @@ cudaError_t launch_tc_t(const ScanArgs &a, cudaStream_t stream)
     cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<TOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((size_t)a.nseq * (a.nheads / 2)));
+    const dim3 grid((unsigned)((size_t)a.nseq * (a.nheads / 2)));
     scan_tc_kernel<TOut><<<grid, kThreads, SMEM_BYTES, stream>>>(mx, mb, mc, my, a);
     return cudaGetLastError();
 }

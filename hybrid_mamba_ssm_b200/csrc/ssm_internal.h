@@ -78,6 +78,11 @@ struct ScanArgs {
     int max_slots;
     DtParams dtp;
     RoundParams rp;
+    // Failure-path testing only (both 0 in every entry point but the
+    // testing hooks of ssm_testing.h): limit of the bounded waits in ns
+    // (0 = the 2 s default), and a producer that issues no load or MMA.
+    unsigned long long wait_ns;
+    int stall_producer;
 };
 
 // Causal depthwise conv1d (prefill over packed sequences, or one decode token
@@ -102,6 +107,9 @@ struct ConvArgs {
     int max_slots;
     void *y;
     int *status_dev;
+    // Failure-path testing only, as for ScanArgs (the pipelined prefill kernel).
+    unsigned long long wait_ns;
+    int stall_producer;
 };
 
 cudaError_t launch_state_update(const StateUpdateArgs &a, cudaStream_t stream);

@@ -28,6 +28,11 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// Plain arrival (release semantics at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
                  ::"r"(bar), "r"(bytes) : "memory");
@@ -42,21 +47,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait for the phase with the given parity to complete, for at most
-// timeout_ns of wall time.  Returns false (and leaves `ok` false) on timeout;
-// once `ok` is false every later wait returns immediately, so a kernel whose
-// barrier never completes runs to its end instead of hanging.
+// try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes or about hint_ns have passed, instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(done) : "r"(bar), "r"(parity), "r"(hint_ns) : "memory");
+    return done != 0;
+}
+
+// Wait for the phase with the given parity to complete, for at most about
+// timeout_ns of wall time (plus one sleep slice of at most 1 ms).  Returns
+// false (and leaves `ok` false) on timeout; once `ok` is false every later
+// wait returns immediately, so a kernel whose barrier never completes runs to
+// its end instead of hanging.  Waiting threads sleep in hardware between
+// checks: they issue no instructions and no shared-memory polls.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, bool &ok,
                                                   uint64_t timeout_ns = 2000000000ull) {
     if (!ok) return false;
-    uint64_t t0 = 0;
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 255u) {
-            const uint64_t now = globaltimer_ns();
-            if (t0 == 0) t0 = now;
-            else if (now - t0 > timeout_ns) { ok = false; return false; }
-        }
+    const uint32_t slice = timeout_ns < 1000000ull ? (uint32_t)timeout_ns : 1000000u;
+    if (mbar_try_wait_sleep(bar, parity, slice)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, slice)) return true;
+        if (globaltimer_ns() - t0 > timeout_ns) { ok = false; return false; }
     }
 }
 

@@ -49,6 +49,11 @@ class Tensor16:
         return "f32" if self.bits is None else "bf16"
 
 
+def store(a32: np.ndarray, dtype: str) -> Tensor16:
+    """Store float32 values as ``dtype`` ("bf16" rounds to nearest even)."""
+    return _store(a32, dtype)
+
+
 def _store(a32: np.ndarray, dtype: str) -> Tensor16:
     if dtype == "f32":
         return Tensor16(values=np.ascontiguousarray(a32, dtype=np.float32))

@@ -18,12 +18,13 @@ LIB_PATH = os.path.join(_HERE, "libssm.so")
 SSM_F32, SSM_BF16, SSM_F16 = 0, 1, 2
 STATUS_NAMES = {0: "SSM_OK", 1: "SSM_ERR_INVALID_ARG", 2: "SSM_ERR_UNSUPPORTED",
                 3: "SSM_ERR_MISALIGNED", 4: "SSM_ERR_CUDA", 5: "SSM_ERR_TIMEOUT",
-                6: "SSM_ERR_DEVICE_INPUT"}
+                6: "SSM_ERR_DEVICE_INPUT", 7: "SSM_ERR_RANGE", 8: "SSM_ERR_INTERNAL"}
+SSM_ERR_TIMEOUT, SSM_ERR_DEVICE_INPUT, SSM_ERR_RANGE = 5, 6, 7
 EXPORTS = ("ssd_chunk_scan", "ssd_chunk_scan_workspace_size", "ssm_state_update",
            "ssd_chunk_scan_slots", "ssm_state_update_slots", "causal_conv1d_fwd",
            "causal_conv1d_update", "ssm_state_update_multi", "ssm_state_commit",
            "causal_conv1d_update_multi", "ssm_gated_rmsnorm", "ssm_status_string",
-           "ssm_version")
+           "ssm_version", "ssm_testing_scan_stalled", "ssm_testing_conv1d_stalled")
 ACTIVATIONS = {None: 0, "none": 0, "silu": 1}
 
 
@@ -65,6 +66,11 @@ def _load():
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_status_string.argtypes = [i]
     lib.ssm_version.restype = i
+    u64 = ctypes.c_ulonglong
+    lib.ssm_testing_scan_stalled.restype = i
+    lib.ssm_testing_scan_stalled.argtypes = [i, i, i, i, vp, vp, vp, vp, vp, vp, u64, vp, vp]
+    lib.ssm_testing_conv1d_stalled.restype = i
+    lib.ssm_testing_conv1d_stalled.argtypes = [i, i, i, i, vp, vp, vp, u64, vp, vp]
     return lib
 
 
@@ -504,3 +510,37 @@ def ssm_gated_rmsnorm(y, z, weight, group_size: int, eps: float = 1e-5, out=None
                                _dtype_code(out.dtype), _ptr(out), _stream(stream))
     _check(st, "ssm_gated_rmsnorm")
     return out
+
+
+# ---------------------------------------------------------------------------
+# Testing hooks (include/ssm_testing.h): the pipelined kernels with a stalled
+# producer and a short wait limit, to exercise their timeout path.
+# ---------------------------------------------------------------------------
+def testing_scan_stalled(x, dt, A, B, C, y, status, wait_ns: int = 1_000_000, stream=None):
+    """Tensor-core scan kernel whose producer issues nothing: every CTA's first
+    bounded wait expires after ``wait_ns`` and the kernel writes
+    SSM_ERR_TIMEOUT to ``status``.  x [nseq, L, H, 64] bf16, dt [nseq, L, H],
+    B, C [nseq, L, G, 128] bf16, y like x (meaningless output)."""
+    for t, n in ((x, "x"), (y, "y"), (B, "B"), (C, "C")):
+        _dev(t, n, torch.bfloat16)
+    _dev(dt, "dt", torch.float32)
+    _dev(A, "A", torch.float32)
+    _dev(status, "status", torch.int32)
+    nseq, L, H, _ = x.shape
+    G = B.shape[-2]
+    st = lib.ssm_testing_scan_stalled(nseq, L, H, G, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                                      _ptr(y), int(wait_ns), _ptr(status), _stream(stream))
+    _check(st, "ssm_testing_scan_stalled")
+
+
+def testing_conv1d_stalled(x, weight, y, status, wait_ns: int = 1_000_000, stream=None):
+    """Bulk-copy ring conv1d kernel whose producer issues nothing (see
+    testing_scan_stalled).  x, y [nseq, L, dim] bf16, weight [dim, width] fp32."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(y, "y", torch.bfloat16)
+    _dev(weight, "weight", torch.float32)
+    _dev(status, "status", torch.int32)
+    nseq, L, dim = x.shape
+    st = lib.ssm_testing_conv1d_stalled(nseq, L, dim, weight.shape[1], _ptr(x), _ptr(weight),
+                                        _ptr(y), int(wait_ns), _ptr(status), _stream(stream))
+    _check(st, "ssm_testing_conv1d_stalled")

@@ -59,7 +59,11 @@ typedef enum {
     SSM_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
     SSM_ERR_CUDA = 4,          /* the CUDA runtime reported a launch error */
     SSM_ERR_TIMEOUT = 5,       /* written to status_dev: a bounded device wait expired */
-    SSM_ERR_DEVICE_INPUT = 6   /* written to status_dev: bad cu_seqlens or slot index */
+    SSM_ERR_DEVICE_INPUT = 6,  /* written to status_dev: bad cu_seqlens or slot index */
+    SSM_ERR_RANGE = 7,         /* written to status_dev: a value beyond the fp16 range of the
+                                  tensor-core operands made y non-finite (see ssd_chunk_scan) */
+    SSM_ERR_INTERNAL = 8       /* written to status_dev: a launch broke a kernel's own layout
+                                  rule (e.g. shared-memory alignment); nothing was computed */
 } ssm_status;
 
 typedef enum {
@@ -93,12 +97,14 @@ typedef struct {
  * state is computed in fp32 and rounded to fp16 when it is written: a value
  * moves to its fp16 neighbour away from zero iff u < frac, frac being its
  * distance from the neighbour toward zero in units of the fp16 spacing there
- * and u = (r >> 8) / 2^24 for a random word r; magnitudes beyond 65504
- * saturate.  r for state element e (its index in the pool) is word e % 4 of
- * Philox-4x32 with philox_rounds rounds (10 = the published Philox-4x32-10),
- * key = seed, counter = (e / 4 as 64 bits, offset as 64 bits).  Callers pass
- * a fresh offset per call (e.g. the decode step).  A NULL ssm_rounding
- * pointer means round to nearest even.
+ * and u = r16 / 2^16 for 16 random bits r16; magnitudes beyond 65504
+ * saturate.  The 16 bits of state element e (its index in the pool) are half
+ * e % 2 (0 = the low half) of 32-bit word (e % 8) / 2 of one Philox-4x32
+ * output with philox_rounds rounds (10 = the published Philox-4x32-10),
+ * key = seed (low word first), counter = (e / 8 as 64 bits, offset as 64
+ * bits; low words first), so one generator call serves 8 adjacent elements.
+ * Callers pass a fresh offset per call (e.g. the decode step).  A NULL
+ * ssm_rounding pointer means round to nearest even.
  */
 typedef struct {
     uint64_t seed;
@@ -138,6 +144,16 @@ SSM_API int ssm_version(void);
  *   products are carried as fp16 (exact for |v| < 65504) so that derived
  *   operands (decay-masked C.B^T, decay-weighted x, the carried state) keep
  *   11 significant bits.
+ * Range of the tensor-core path (bf16 x/B/C, head_dim 64, d_state 128,
+ *   chunk 128, an even number of heads per group): x, B, C, every
+ *   decay-masked C.B^T entry dt_j exp(cs_i - cs_j) C_i.B_j and every carried
+ *   state entry must stay below 65504 in magnitude.  Beyond it an fp16
+ *   operand becomes infinite, y of the affected chunks is not valid, and the
+ *   kernel writes SSM_ERR_RANGE to *status_dev (the final state, computed
+ *   from x, B and the decay weights only, stays valid unless x or B is out of
+ *   range).  Values below 2^-14 keep an absolute precision of 2^-25.  Every
+ *   other shape and fp32 inputs run in fp32 on the CUDA cores, without this
+ *   limit.
  * D: device [nheads] or NULL (no skip term).
  * initial_state: device fp32 [nseq][nheads][head_dim][d_state] or NULL (zero).
  *   It may be the same pointer as final_state (in-place update of a state

@@ -18,6 +18,38 @@ from hybrid_mamba_ssm_b200 import inputs as synth
 
 TOL = 2e-3
 
+# Canary guard bands: every output buffer a parity test hands to the library
+# sits between two GUARD-byte bands filled with SENTINEL; after the call the
+# bands must be untouched (no stray write before or after an output, e.g. by a
+# TMA store of a partial tile or a slot-indexed write).
+GUARD = 4096
+SENTINEL = 0x5A
+
+
+class Guarded:
+    """A device tensor of ``shape`` inside a larger buffer with guard bands."""
+
+    def __init__(self, shape, dtype, device="cuda", init=None):
+        es = torch.empty((), dtype=dtype).element_size()
+        n = int(np.prod(shape)) if len(shape) else 1
+        g = GUARD // es
+        self.buf = torch.empty(n + 2 * g, dtype=dtype, device=device)
+        self.buf.view(torch.uint8).fill_(SENTINEL)
+        self.t = self.buf[g:g + n].view(*shape)
+        if init is not None:
+            self.t.copy_(init)
+
+    def check(self, name="output"):
+        b = self.buf.view(torch.uint8)
+        head, tail = b[:GUARD], b[b.numel() - GUARD:]
+        assert bool((head == SENTINEL).all()), f"write before {name}"
+        assert bool((tail == SENTINEL).all()), f"write after {name}"
+
+
+def guarded_like(t, init=True):
+    """A guarded copy of tensor t (its contents copied in when init)."""
+    return Guarded(tuple(t.shape), t.dtype, t.device, init=t if init else None)
+
 
 def dev_tensor(t: synth.Tensor16, device="cuda"):
     if t.bits is None:
@@ -52,8 +84,12 @@ def to_np(t):
 
 
 def scan_on_gpu(inp: synth.ScanInputs, chunk=128, y_dtype=torch.bfloat16, varlen=None,
-                initial_state=True, inplace=False, use_D=True):
-    """Run ssd_chunk_scan on the inputs; returns (y, final_state) tensors."""
+                initial_state=True, inplace=False, use_D=True, expect_status=0):
+    """Run ssd_chunk_scan on the inputs; returns (y, final_state) tensors.
+
+    y and the final state are written into guarded buffers whose guard bands
+    are checked after the call; the device status word must read
+    ``expect_status`` (0 unless a test provokes a device-side status)."""
     from hybrid_mamba_ssm_b200 import ssm
     T, nseq = inp.T, inp.nseq
     lens = np.diff(inp.cu_seqlens)
@@ -64,25 +100,35 @@ def scan_on_gpu(inp: synth.ScanInputs, chunk=128, y_dtype=torch.bfloat16, varlen
     Bt, Ct = dev_tensor(inp.B), dev_tensor(inp.C)
     dt = dev_f32(inp.dt)
     A, D = dev_f32(inp.A), dev_f32(inp.D) if use_D else None
-    h0 = dev_f32(inp.h0) if (initial_state and inp.h0 is not None) else None
+    H, P = x.shape[1], x.shape[2]
+    G, N = Bt.shape[1], Bt.shape[2]
+    h0g = None
+    if initial_state and inp.h0 is not None:
+        h0g = guarded_like(dev_f32(inp.h0))
+    h0 = None if h0g is None else h0g.t
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    yg = Guarded((T, H, P), y_dtype)
+    if inplace and h0g is not None:
+        hg = h0g
+    else:
+        hg = Guarded((nseq, H, P, N), torch.float32)
     if varlen:
         cu = torch.from_numpy(inp.cu_seqlens.astype(np.int32)).cuda()
-        fs = h0 if (inplace and h0 is not None) else None
         y, hT = ssm.ssd_chunk_scan(x, dt, A, Bt, Ct, D, h0, cu_seqlens=cu, chunk_size=chunk,
-                                   y_dtype=y_dtype, final_state=fs, status=status)
+                                   y=yg.t, final_state=hg.t, status=status)
     else:
         L = int(lens[0]) if nseq else 0
-        H, P = x.shape[1], x.shape[2]
-        G, N = Bt.shape[1], Bt.shape[2]
-        fs = h0 if (inplace and h0 is not None) else None
         y, hT = ssm.ssd_chunk_scan(x.view(nseq, L, H, P), dt.view(nseq, L, H), A,
                                    Bt.view(nseq, L, G, N), Ct.view(nseq, L, G, N), D, h0,
-                                   chunk_size=chunk, y_dtype=y_dtype, final_state=fs,
-                                   status=status)
+                                   chunk_size=chunk, y=yg.t.view(nseq, L, H, P),
+                                   final_state=hg.t, status=status)
         y = y.view(T, H, P)
     torch.cuda.synchronize()
-    assert int(status.item()) == 0
+    yg.check("y")
+    hg.check("final_state")
+    if h0g is not None:
+        h0g.check("initial_state")
+    assert int(status.item()) == expect_status, (int(status.item()), expect_status)
     return y, hT
 
 

@@ -1,4 +1,4 @@
-"""The C ABI: the library loads, exports every symbol include/ssm.h declares,
+"""The C ABI: the library loads, exports every symbol include/*.h declares,
 and rejects bad arguments on the host before launching anything.
 
 No test here launches a kernel: every call either fails validation (which
@@ -14,6 +14,8 @@ from hybrid_mamba_ssm_b200 import build as ssm_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "ssm.h")
+HEADERS = sorted(os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+                 if f.endswith(".h"))
 
 OK, INVALID, UNSUPPORTED, MISALIGNED = 0, 1, 2, 3
 F32, BF16 = 0, 1
@@ -38,8 +40,10 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    return re.findall(r"SSM_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    names = []
+    for h in HEADERS:
+        names += re.findall(r"SSM_API\s+[\w\s\*]+?\b(\w+)\s*\(", open(h).read())
+    return names
 
 
 def test_header_declares_the_entry_points():
@@ -55,8 +59,9 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(9):
         assert lib.ssm_status_string(code)
+        assert b"unknown" not in lib.ssm_status_string(code)
     assert b"unknown" in lib.ssm_status_string(99)
 
 
@@ -357,3 +362,26 @@ def test_gated_rmsnorm_rejects(lib):
     assert call(out=0x200000 + 64) == INVALID    # out overlaps z
     assert call(out=0x100000 + 2, od=BF16) == MISALIGNED
     assert call(rows=0, y=None, z=None, w=None, out=None) == OK
+
+
+def test_testing_hooks_validate_on_the_host(lib):
+    u64 = ctypes.c_ulonglong
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    lib.ssm_testing_scan_stalled.restype = i
+    lib.ssm_testing_scan_stalled.argtypes = [i, i, i, i, vp, vp, vp, vp, vp, vp, u64, vp, vp]
+    lib.ssm_testing_conv1d_stalled.restype = i
+    lib.ssm_testing_conv1d_stalled.argtypes = [i, i, i, i, vp, vp, vp, u64, vp, vp]
+    args = (A16, A16b, A16c, 0x40000, 0x50000, 0x60000)
+    # the status word is required, the wait limit bounded, the pointers aligned
+    assert lib.ssm_testing_scan_stalled(1, 256, 4, 2, *args, 10**6, None, None) == INVALID
+    assert lib.ssm_testing_scan_stalled(1, 256, 4, 2, *args, 10, 0x80000, None) == INVALID
+    assert lib.ssm_testing_scan_stalled(1, 256, 4, 2, *args, 10**11, 0x80000, None) == INVALID
+    assert lib.ssm_testing_scan_stalled(1, 256, 3, 2, *args, 10**6, 0x80000, None) == INVALID
+    assert lib.ssm_testing_scan_stalled(1, 256, 4, 2, ODD, *args[1:], 10**6, 0x80000,
+                                        None) == MISALIGNED
+    assert lib.ssm_testing_conv1d_stalled(1, 64, 100, 4, A16, A16b, A16c, 10**6, 0x80000,
+                                          None) == INVALID            # dim % 8
+    assert lib.ssm_testing_conv1d_stalled(1, 64, 128, 9, A16, A16b, A16c, 10**6, 0x80000,
+                                          None) == INVALID            # width
+    assert lib.ssm_testing_conv1d_stalled(1, 64, 128, 4, A16, A16b, A16c, 10**6, None,
+                                          None) == INVALID            # no status word

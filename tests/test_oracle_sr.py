@@ -94,3 +94,26 @@ def test_round_state_draw_layout():
         ref.append(1.0 + 2.0**-10 if r16 < 32768 else 1.0)
     assert list(got) == ref
     assert 0 < sum(g > 1.0 for g in got) < 24
+
+
+def test_header_states_the_pinned_draw_layout():
+    """The public header's description of the draw layout (ssm_rounding in
+    include/ssm.h) is the one the oracle follows and the test above pins:
+    its numbers are read from the comment and checked against the oracle."""
+    import re
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    text = open(os.path.join(root, "include", "ssm.h")).read()
+    block = text[text.index("Stochastic rounding of an fp16 state pool"):
+                 text.index("uint64_t seed;")]
+    block = " ".join(block.replace("*", " ").split())
+    bits, scale = map(int, re.search(r"u = r(\d+) / 2\^(\d+)", block).groups())
+    halves = int(re.search(r"half e % (\d+)", block).group(1))
+    per_call, per_word = map(int, re.search(r"word \(e % (\d+)\) / (\d+)", block).groups())
+    ctr_div = int(re.search(r"counter = \(e / (\d+)", block).group(1))
+    assert (bits, scale, halves, per_call, per_word, ctr_div) == (16, 16, 2, 8, 2, 8)
+    v = np.full(24, 1.0 + 2.0**-11)
+    got = oracle.round_state_f16(v, np.arange(24), 11, 5)
+    for e in range(24):
+        w = oracle.philox4x32((e // ctr_div, 0, 5, 0), (11, 0), 10)[(e % per_call) // per_word]
+        r = (w >> (bits * (e % halves))) & ((1 << bits) - 1)
+        assert got[e] == (1.0 + 2.0**-10 if r < (1 << (scale - 1)) else 1.0), e

@@ -4,7 +4,7 @@ import pytest
 import torch
 
 from hybrid_mamba_ssm_b200 import inputs as synth
-from tests.gpu_helpers import TOL, dev_f32, dev_tensor, rel_err, to_np
+from tests.gpu_helpers import TOL, Guarded, dev_f32, dev_tensor, guarded_like, rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -14,22 +14,25 @@ def run_steps(batch, H, P, N, G, dtype, y_dtype, steps, seed, use_D=True, sample
     from hybrid_mamba_ssm_b200 import ssm
     A, D = synth.make_head_params(seed, H)
     state0 = synth.make_state(seed + 1, (batch, H, P, N))
-    st_gpu = dev_f32(state0)
+    st_g = guarded_like(dev_f32(state0))
+    st_gpu = st_g.t
     At, Dt = dev_f32(A), (dev_f32(D) if use_D else None)
+    y_g = Guarded((batch, H, P), y_dtype)
     ref = state0.astype(np.float64)
     bs = slice(None) if sample is None else sample
     worst_y = worst_s = 0.0
     for k in range(steps):
         inp = synth.make_decode_step(seed + 100 + k, batch, H, P, N, G, dtype)
         y = ssm.ssm_state_update(st_gpu, dev_tensor(inp.x), dev_f32(inp.dt), At,
-                                 dev_tensor(inp.B), dev_tensor(inp.C), Dt,
-                                 y_dtype=y_dtype)
+                                 dev_tensor(inp.B), dev_tensor(inp.C), Dt, y=y_g.t)
         y_ref, ref_new = oracle.state_update(ref[bs], inp.x.values[bs], inp.dt[bs], A,
                                              inp.B.values[bs], inp.C.values[bs],
                                              D if use_D else None)
         ref = ref_new if sample is None else _put(ref, bs, ref_new)
         worst_y = max(worst_y, rel_err(to_np(y)[bs], y_ref, bf16=y_dtype == torch.bfloat16))
     torch.cuda.synchronize()
+    st_g.check("state")
+    y_g.check("y")
     worst_s = rel_err(to_np(st_gpu)[bs], ref[bs])
     return worst_y, worst_s
 

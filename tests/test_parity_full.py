@@ -25,8 +25,11 @@ def _workload_inputs(name):
                                   init_state=w["init_state"])
 
 
-@pytest.mark.parametrize("name,heads", [("prefill_4x4096", [0, 17, 66, 127]),
-                                        ("prefill_ultra_32k", [0, 95, 200, 255])])
+# One whole group of heads (all heads sharing one B, C), plus heads of other
+# groups: group 1 of the 128-head workload (heads 16..31), group 6 of the
+# 256-head one (heads 192..223).
+@pytest.mark.parametrize("name,heads", [("prefill_4x4096", list(range(16, 32)) + [0, 66, 127]),
+                                        ("prefill_ultra_32k", list(range(192, 224)) + [0, 95])])
 def test_full_prefill_sampled_heads(name, heads):
     inp = _workload_inputs(name)
     y, hT = scan_on_gpu(inp, chunk=128, y_dtype=torch.bfloat16)
