@@ -95,7 +95,14 @@ const char *ssm_status_string(int status)
 
 int ssm_version(void) { return 200; }
 
-size_t ssd_chunk_scan_workspace_size(int, int, int, int, int, int, int) { return 0; }
+size_t ssd_chunk_scan_workspace_size(int nseq, int seqlen, int nheads, int head_dim, int d_state,
+                                     int ngroups, int chunk_size)
+{
+    if (nseq <= 0 || seqlen <= 0 || !ssm::scan_tc_shape(head_dim, d_state, chunk_size, nheads, ngroups))
+        return 0;
+    const int runs = ssm::scan_tc_balanced_runs(nseq, seqlen, nheads);
+    return runs ? ssm::scan_tc_handoff_bytes(runs) : 0;
+}
 
 int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
                    int nheads, int head_dim, int d_state, int ngroups,
@@ -107,7 +114,6 @@ int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
                    void *workspace, size_t workspace_bytes,
                    int *status_dev, cudaStream_t stream)
 {
-    (void)workspace; (void)workspace_bytes;
     if (nseq < 0 || seqlen < 0 || nheads <= 0 || ngroups <= 0 || nheads % ngroups)
         return SSM_ERR_INVALID_ARG;
     if (!valid_dtype(in_dtype) || !valid_dtype(y_dtype)) return SSM_ERR_INVALID_ARG;
@@ -163,8 +169,25 @@ int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
     a.initial_state = initial_state; a.y = y; a.final_state = final_state;
     a.status_dev = status_dev;
     a.slot_idx = nullptr; a.has_initial = nullptr; a.max_slots = 0;
-    const cudaError_t e = ssm::scan_tc_supports(a) ? ssm::launch_scan_tc(a, stream)
-                                                   : ssm::launch_scan_simt(a, stream);
+    const bool tc = ssm::scan_tc_supports(a);
+    if (tc && !cu_seqlens && workspace && workspace_bytes) {
+        // balanced schedule: the carried state crosses the cuts through the workspace
+        const int runs = ssm::scan_tc_balanced_runs(nseq, seqlen, nheads);
+        const size_t need = runs ? ssm::scan_tc_handoff_bytes(runs) : 0;
+        if (runs && workspace_bytes >= need) {
+            if (!aligned16(workspace)) return SSM_ERR_MISALIGNED;
+            const Range rw = range_of(workspace, need);
+            const Range outs[] = {ry, rhT};
+            for (const Range &r : ins)
+                if (overlap(rw, r)) return SSM_ERR_INVALID_ARG;
+            for (const Range &r : outs)
+                if (overlap(rw, r)) return SSM_ERR_INVALID_ARG;
+            a.runs = runs;
+            a.handoff = static_cast<float *>(workspace);
+            a.handoff_flags = reinterpret_cast<int *>(static_cast<char *>(workspace) + (need - runs * sizeof(int)));
+        }
+    }
+    const cudaError_t e = tc ? ssm::launch_scan_tc(a, stream) : ssm::launch_scan_simt(a, stream);
     return e == cudaSuccess ? SSM_OK : SSM_ERR_CUDA;
 }
 

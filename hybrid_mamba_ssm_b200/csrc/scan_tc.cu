@@ -19,38 +19,29 @@
 // The diagonal j = i belongs to M because the output reads the updated state.
 //
 // Work decomposition: one CTA per (sequence, pair of heads of one group),
-// sweeping the sequence's chunks in order, with three warp roles that work on
-// different chunks at the same time (640 threads, 20 warps):
-//   * compute warpgroups (warps 4-19): head 2k + (wg & 1), column half wg >> 1;
-//     thread i owns TMEM lane i (row i of G, M, Y, Yoff; d_state index i of
-//     S^T and of the carried state, 32 of whose 64 head_dim entries it keeps
-//     in fp32 registers for the whole sequence).  Per chunk: the next chunk's
-//     cumulative decay (published for the converters), state update, decay
-//     mask, new H^T tile, the next chunk's C converted into TMEM (the A
-//     operand of C.B^T and C.H^T, double-buffered), output epilogue;
-//   * converter warps (warps 0-2): one chunk ahead of the compute warps, they
-//     convert the chunk's bf16 B and x tiles to fp16 in place in shared
-//     memory and form the decay-weighted x (w o x) from the published decay;
-//   * issuing warp (warp 3): lane 0 issues the TMA loads and stores and the
-//     MMAs as their operands become ready.
-// Every hand-off between roles is an mbarrier with a bounded wait (no named
-// barrier spans two roles), so a wait that never completes cannot hang the
-// kernel: it raises a CTA-wide abort flag instead.  20 warps keep 5 warps on
-// each SM sub-partition, so every thread gets 96 registers.
+// sweeping the sequence's chunks in order.  544 threads: four compute
+// warpgroups and one issuing warp.  Compute warpgroup wg works on head
+// 2k + (wg & 1) and on half (wg >> 1) of the columns: thread i of it owns TMEM
+// lane i (row i of G, M, Y, Yoff; d_state index i of S^T and of the carried
+// state, 32 of whose 64 head_dim entries it keeps in fp32 registers for the
+// whole sequence).  Lane 0 of the issuing warp issues TMA and the MMAs; the
+// products shared by both heads (C.B^T, and B^T or C against the two heads'
+// operands side by side) are single N = 128 MMAs.
 //
-// Per chunk k, the issuing thread runs
-//   S_k = B^T [wX_a|wX_b]  (once Y_{k-1} has read M_{k-1}, whose TMEM S reuses)
-//   G_k = C B^T            (once the epilogue of k-1 has read Y_{k-1})
-//   Yoff_k = C [H_a^T|H_b^T] (once H_{k-1}^T is in shared memory)
-//   Y_k = M_k X_k          (once the mask of chunk k is in TMEM)
-// while the compute warps work through chunk k and the converters prepare
-// chunk k+1.
+// Pipeline per chunk (single-buffered tiles, with prefetch where a buffer
+// frees early):
+//   wait TMA(x), TMA(B, C) -> convert bf16 -> fp16 (C into TMEM and B in
+//   place, a quarter of d_state per warpgroup; x and w o x per head)
+//   -> issue TMA(x of next chunk) into the raw x buffers
+//   -> MMA S^T (2 heads), G  [commit] , Yoff (2 heads) [commit]
+//   -> the next chunk's cumulative decay (while the MMAs run)
+//   -> issue TMA(B, C of next chunk) once S^T and G are done
+//   -> state update from S^T, decay mask M per head (overlap the Yoff MMAs)
+//   -> MMA Y (2 heads) [commit] -> epilogue y.
 //
 // Precision: bf16 inputs are converted to fp16 (exact for |v| < 65504) so the
 // derived operands M, w o x and H (rounded to fp16, 11 significant bits) keep
-// the result within ~3e-4 of the fp64 recurrence; accumulation is fp32.  An
-// operand beyond the fp16 range makes some output non-finite; the epilogue
-// detects that and the kernel reports SSM_ERR_RANGE.
+// the result within ~3e-4 of the fp64 recurrence; accumulation is fp32.
 //
 // Decay factors are never ratios of exponentials.  With block ends r_K =
 // 32K+31, exp(cs_i - cs_j) = exp(cs_i - cs_{r_I}) exp(cs_{r_I} - cs_{r_J})
@@ -70,65 +61,35 @@ namespace {
 constexpr int kQ = 128;       // chunk length
 constexpr int kP = 64;        // head_dim
 constexpr int kN = 128;       // d_state
-constexpr int kConvThreads = 96;       // converter warps 0-2 (lane-free work)
-constexpr int kIssuerBase = 96;        // warp 3
-constexpr int kComputeBase = 128;      // compute warpgroups: warps 4-19
-constexpr int kCompute = 512;
-constexpr int kThreads = kComputeBase + kCompute;      // 640
+constexpr int kThreads = 544;   // 16 compute warps + 1 issuing warp
 
 // Shared memory (bytes from the 1024-aligned dynamic base).  16-bit tiles use
 // the 128B-swizzled layout TMA writes and the MMA descriptors read: rows of 64
 // elements (128 B), 8-row groups of 1024 B, 16-byte chunk c of row r stored at
 // c ^ (r % 8).  128-wide tiles are two 64-column halves 16 KB apart.
 constexpr uint32_t HALF = 16384;
-constexpr uint32_t OFF_C = 0;            // C [128 i][128 n] bf16 (TMA target; fp16 copy in TMEM)
-constexpr uint32_t OFF_B = 32768;        // B buffer 0 [128 j][128 n] (bf16 -> fp16 in place)
-constexpr uint32_t OFF_X = 65536;        // x, 2 buffers x 2 heads x [128 j][64 p] (bf16 -> fp16 in
-                                         // place; after Y_k, the staging of y_k for its TMA store)
-constexpr uint32_t XBUF = 32768;
-constexpr uint32_t OFF_W = 131072;       // w o x, 2 heads x [128 j][64 p] fp16
-constexpr uint32_t OFF_H = 163840;       // H^T fp16, 2 heads x [128 n][64 p]
-constexpr uint32_t OFF_B1 = 196608;      // B buffer 1
+constexpr uint32_t OFF_C = 0;            // C [128 i][128 n]  bf16 (TMA target; fp16 copy in TMEM)
+constexpr uint32_t OFF_B = 32768;        // B [128 j][128 n]  (bf16 -> fp16 in place)
+constexpr uint32_t OFF_XR = 65536;       // raw x, 2 heads x [128 j][64 p] bf16 (TMA target)
+constexpr uint32_t OFF_XH = 98304;       // x as fp16, 2 heads
+constexpr uint32_t OFF_WM = 131072;      // w o x, 2 heads x [128 j][64 p]
+constexpr uint32_t OFF_MB = 163840;      // y staging, 2 heads x [128 t][64 p] bf16
+constexpr uint32_t OFF_H = 196608;       // H^T fp16, 2 heads x [128 n][64 p]
 constexpr uint32_t OFF_MISC = 229376;
 constexpr uint32_t OFF_VD = OFF_MISC;              // float[2 buffers][2 heads][128]: column factors vd
-constexpr uint32_t OFF_WF = OFF_VD + 2048;         // float[2 buffers][2 heads][4]: exp(cs_last - cs_{r_J})
-constexpr uint32_t OFF_CSBT = OFF_WF + 64;         // float[2 buffers][2 heads][8]: block-end cs, cs_last
-constexpr uint32_t OFF_CSB = OFF_CSBT + 128;       // float[4][8]: scan scratch per compute warpgroup
-constexpr uint32_t OFF_PART = OFF_CSB + 128;       // float[4][4]: compute warp partial sums
-constexpr uint32_t OFF_BAR = OFF_PART + 64;        // mbarriers (8 B each)
-constexpr uint32_t NBAR = 18;
-constexpr uint32_t OFF_TM = OFF_BAR + 8 * NBAR;    // TMEM base address (4 B)
+constexpr uint32_t OFF_CSBT = OFF_VD + 2048;       // float[2 buffers][2 heads][8]: block-end cs, cs_last
+constexpr uint32_t OFF_CSB = OFF_CSBT + 128;       // float[4][8]: scan scratch per warpgroup
+constexpr uint32_t OFF_PART = OFF_CSB + 128;       // float[4][4] warp partial sums
+constexpr uint32_t OFF_BAR = OFF_PART + 64;        // 6 mbarriers
+constexpr uint32_t OFF_TM = OFF_BAR + 48;          // TMEM base address (4 B)
 constexpr uint32_t OFF_ABORT = OFF_TM + 4;         // CTA-wide abort flag (int)
 constexpr uint32_t OFF_RANGE = OFF_TM + 8;         // set when an output is not finite (int)
 constexpr uint32_t SMEM_BYTES = OFF_TM + 16;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-
-// mbarrier indices (address OFF_BAR + 8 * index).  A barrier that serves
-// alternate chunks (x buffers, converter hand-off, decay tables) comes in a
-// pair indexed by chunk parity, so that no waiter can ever be two phases
-// behind the barrier it waits on.
-enum : uint32_t {
-    BAR_X0 = 0, BAR_X1 = 1,   // x tiles of buffer 0 / 1 landed (TMA)
-    BAR_CT = 2,               // C tile landed (TMA)
-    BAR_BT0 = 3, BAR_BT1 = 4, // B tile of buffer 0 / 1 landed (TMA)
-    BAR_CRAW = 5,             // compute warps have read the C tile (16 warp arrivals)
-    BAR_CV0 = 6, BAR_CV1 = 7, // converters done with a chunk of parity 0 / 1 (3 warp arrivals)
-    BAR_DC0 = 8, BAR_DC1 = 9, // decay tables of a chunk of parity 0 / 1 published (8 warp arrivals)
-    BAR_S = 10,               // S MMAs of a chunk done (commit): w o x may be rewritten
-    BAR_SG = 11,              // S and G MMAs of a chunk done (commit)
-    BAR_YO = 12,              // Yoff MMAs done (commit)
-    BAR_Y = 13,               // Y MMAs done (commit)
-    BAR_MASK = 14,            // decay mask written (16 compute-warp arrivals)
-    BAR_STATE = 15,           // H^T tile written (16 compute-warp arrivals)
-    BAR_EPI = 16,             // epilogue done and next C in TMEM (16 compute-warp arrivals)
-    BAR_DRAIN = 17            // abort path: every issued MMA done (commit)
-};
 
 // TMEM columns (fp32 accumulators, lane = row).
 // G and Y share columns: the y MMAs write Y only after the mask has read G,
 // and the next chunk's G is issued only after the epilogue has read Y.  C
-// (fp16, two values per column, double-buffered) is the TMEM A operand of
-// C.B^T and C.H^T.
+// (fp16, two values per column) is the TMEM A operand of C.B^T and C.H^T.
 constexpr uint32_t TM_G = 0, TM_Y = 0, TM_S = 128, TM_YO = 256, TM_C = 384;
 constexpr uint32_t TM_COLS = 512;
 
@@ -138,39 +99,6 @@ constexpr uint32_t IDESC_YO2 = tc::idesc_f16_f32(128, 128, 0, 1); // C (K-major)
 constexpr uint32_t IDESC_Y = tc::idesc_f16_f32(128, 64, 0, 1);    // M (TMEM) x X (MN-major)
 
 constexpr float kSafeBlockDecay = 80.f;   // max exp argument taken by the factorised path
-
-// Named barriers (never shared between roles): 1..4 per compute warpgroup,
-// 5 all compute warps.
-constexpr uint32_t NB_COMPUTE = 5;
-
-extern __shared__ __align__(1024) uint8_t smem[];
-
-__device__ __forceinline__ volatile int &abort_flag() {
-    return *reinterpret_cast<volatile int *>(smem + OFF_ABORT);
-}
-__device__ __forceinline__ volatile int &range_flag() {
-    return *reinterpret_cast<volatile int *>(smem + OFF_RANGE);
-}
-__device__ __forceinline__ uint64_t wait_limit(unsigned long long wait_ns) {
-    return wait_ns ? wait_ns : kDefaultWaitNs;
-}
-
-// Bounded mbarrier wait: when it expires (or the abort flag is already up)
-// `ok` turns false, the CTA-wide abort flag goes up, and every later wait of
-// this thread returns at once.  The roles then run to the end of their loops
-// without waiting, the issuing thread drains what it has in flight, and the
-// kernel reports SSM_ERR_TIMEOUT.
-__device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, bool &ok,
-                                              unsigned long long wait_ns) {
-    if (ok && abort_flag()) ok = false;
-    if (ok && !tc::mbar_wait_bounded(bar, parity, ok, wait_limit(wait_ns))) abort_flag() = 1;
-}
-
-// One arrival per warp on an mbarrier, after every lane's prior writes.
-__device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
-    __syncwarp();
-    if (lane == 0) tc::mbar_arrive(bar);
-}
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
@@ -212,6 +140,30 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
 
 __device__ __forceinline__ void wg_sync(int wg) {
     asm volatile("bar.sync %0, 128;" ::"r"(wg + 1) : "memory");
+}
+
+// Bounded mbarrier wait that, when it expires, raises the CTA-wide abort
+// flag: the issuing warp stops issuing TMA loads and MMAs, and every other
+// thread skips its remaining waits (it reads the flag after the next named
+// barrier).  The kernel then drains what is in flight and exits, reporting
+// SSM_ERR_TIMEOUT.
+extern __shared__ __align__(1024) uint8_t smem[];
+
+__device__ __forceinline__ int flag_get(uint32_t off) {
+    int v;
+    asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(tc::smem_u32(smem) + off) : "memory");
+    return v;
+}
+__device__ __forceinline__ void flag_set(uint32_t off, int v) {
+    asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(tc::smem_u32(smem) + off), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t wait_limit(unsigned long long wait_ns) {
+    return wait_ns ? wait_ns : kDefaultWaitNs;
+}
+
+__device__ __forceinline__ void wait_or_abort(uint32_t bar, uint32_t parity, bool &ok,
+                                              unsigned long long wait_ns) {
+    if (ok && !tc::mbar_wait_bounded(bar, parity, ok, wait_limit(wait_ns))) flag_set(OFF_ABORT, 1);
 }
 
 __device__ __forceinline__ void store16(float *dst, const float (&v)[16]) {
@@ -294,7 +246,20 @@ __device__ __noinline__ void mask_block_exact(uint32_t g_taddr, uint32_t m_taddr
 //   diagonal (jc == wq):     j <= i only, plus D on j == i
 //   above (jc > wq):         zeros
 // with vd[j] = exp(cs_{r_J} - cs_j) dt_j (J = j's block) from shared memory.
-__device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, const float *sVD,
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, uint32_t sVD,
                                            int jc, int wq, int lane, float ua,
                                            bool block_safe, float cs, float dtv, float Dh)
 {
@@ -309,7 +274,7 @@ __device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, c
         mask_block_exact(g_taddr, m_taddr, jc, lane, cs, dtv, Dh);
         return;
     }
-    const float4 *vd4 = reinterpret_cast<const float4 *>(sVD + jc * 32);
+    const uint32_t vd4 = sVD + jc * 128;
 #pragma unroll
     for (int qq = 0; qq < 2; ++qq) {   // 16 columns at a time
         uint32_t r[16];
@@ -318,7 +283,7 @@ __device__ __forceinline__ void mask_block(uint32_t g_taddr, uint32_t m_taddr, c
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
             const int q = qq * 2 + q2;   // 8-column chunk within the block
-            const float4 v0 = vd4[2 * q], v1 = vd4[2 * q + 1];
+            const float4 v0 = lds_f32x4(vd4 + 32 * q), v1 = lds_f32x4(vd4 + 32 * q + 16);
             const float vd[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
             float m[8];
             if (jc < wq) {
@@ -372,30 +337,28 @@ struct ChunkDecay {
     float cs;        // inclusive cumulative dt*A at row i
     float dtv;       // dt of row i (0 past the chunk end)
     float uaA, uaB;  // exp(cs_i - cs_{r_K}) for this thread's two column blocks
+    float w;         // exp(cs_last - cs_i) dt_i   (weights of the chunk state)
     float e;         // exp(cs_i)                  (decay of the carried state to row i)
     float a_last;    // exp(cs_last)               (decay over the whole chunk)
     bool safe;       // the row block's own decay fits the factorised path
 };
 
 // Raw dt of row i of the chunk starting at c0 (0 past the sequence end t1),
-// loaded ahead of use: the compute and converter loops keep two chunks of it
-// in flight.
+// loaded ahead of use: the compute loop keeps two chunks of it in flight.
 __device__ __forceinline__ float load_dt(const ScanArgs &a, int H, int hh, long c0, long t1, int i) {
     return (c0 + i < t1) ? __ldg(a.dt + (size_t)(c0 + i) * H + hh) : 0.f;
 }
 
 // Cumulative decay of head hh over a chunk of Lc tokens whose raw dt for row
-// i is dt_raw (warpgroup-wide); returns (cs_i, dt_i).  The warpgroup with
-// ch == 0 publishes the chunk's tables, read later by the compute warps
-// (decay_derive, the mask) and by the converters (w o x):
-//   vd[j]   = exp(cs_{r_J} - cs_j) dt_j, J = j's 32-row block (column factors)
-//   wf[J]   = exp(cs_last - cs_{r_J})      (so the chunk-state weight is
-//                                          w_j = wf[J] vd_j: two factors <= 1)
-//   csb[J]  = cs_{r_J} (J < 4), csb[4] = cs_last
-__device__ __forceinline__ float2 decay_scan(const ScanArgs &a, int hh, float Ah, float dt_raw,
+// i is dt_raw (warpgroup-wide).  Returns row i's (cs_i, dt_i, w_i) with the
+// chunk-state weight w_i = exp(cs_last - cs_i) dt_i.  The warpgroup with
+// ch == 0 also publishes the chunk's tables for decay_derive and the mask:
+//   vd[j]  = exp(cs_{r_J} - cs_j) dt_j, J = j's 32-row block (column factors)
+//   csb[J] = cs_{r_J} (J < 4), csb[4] = cs_last
+__device__ __forceinline__ float3 decay_scan(const ScanArgs &a, int hh, float Ah, float dt_raw,
                                              int Lc, int i, int wq, int lane, int wg, int ch,
-                                             float *sPART, float *sCSB, float *vd_out,
-                                             float *wf_out, float *csb_out)
+                                             uint32_t sPART, uint32_t sCSB, uint32_t vd_out,
+                                             uint32_t csb_out)
 {
     const float dtv = (i < Lc) ? dt_apply(a.dtp, dt_raw, hh) : 0.f;
     float v = dtv * Ah;
@@ -404,117 +367,232 @@ __device__ __forceinline__ float2 decay_scan(const ScanArgs &a, int hh, float Ah
         const float u = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += u;
     }
-    if (lane == 31) sPART[wq] = v;
+    if (lane == 31) sts_f32(sPART + 4 * wq, v);
     wg_sync(wg);
     float pre = 0.f;
-    for (int w = 0; w < wq; ++w) pre += sPART[w];
+    for (int w = 0; w < wq; ++w) pre += lds_f32(sPART + 4 * w);
     const float cs = v + pre;
-    if (lane == 31) sCSB[wq] = cs;
-    if (i == Lc - 1) sCSB[4] = cs;
+    if (lane == 31) sts_f32(sCSB + 4 * wq, cs);
+    if (i == Lc - 1) sts_f32(sCSB + 16, cs);
     wg_sync(wg);
+    const float cs_last = lds_f32(sCSB + 16);
     if (ch == 0) {
-        const float cs_last = sCSB[4];
-        vd_out[i] = exp_dec(sCSB[wq] - cs) * dtv;   // <= dt
-        if (i < 4) wf_out[i] = exp_dec(cs_last - sCSB[i]);
-        if (i < 5) csb_out[i] = sCSB[i];
+        sts_f32(vd_out + 4 * i, exp_dec(lds_f32(sCSB + 4 * wq) - cs) * dtv);   // <= dt
+        if (i < 5) sts_f32(csb_out + 4 * i, lds_f32(sCSB + 4 * i));
     }
-    return make_float2(cs, dtv);
+    return make_float3(cs, dtv, (i < Lc) ? exp_dec(cs_last - cs) * dtv : 0.f);
 }
 
-// The per-row decay quantities of ChunkDecay from row i's (cs, dt) and the
-// chunk's published block ends csb.
-__device__ __forceinline__ ChunkDecay decay_derive(float2 csdt, const float *csb, int wq, int ch) {
+// The per-row decay quantities of ChunkDecay from row i's (cs, dt, w) and
+// the chunk's published block ends csb.
+__device__ __forceinline__ ChunkDecay decay_derive(float3 csdtw, uint32_t csb, int wq, int ch) {
     ChunkDecay d;
-    d.cs = csdt.x;
-    d.dtv = csdt.y;
+    d.cs = csdtw.x;
+    d.dtv = csdtw.y;
+    d.w = csdtw.z;
     const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
-    d.uaA = (kA <= wq) ? exp_dec(d.cs - csb[kA]) : 0.f;
-    d.uaB = (kB <= wq) ? exp_dec(d.cs - csb[kB]) : 0.f;
-    d.safe = (__shfl_sync(0xffffffffu, d.cs, 0) - csb[wq]) <= kSafeBlockDecay;
+    d.uaA = (kA <= wq) ? exp_dec(d.cs - lds_f32(csb + 4 * kA)) : 0.f;
+    d.uaB = (kB <= wq) ? exp_dec(d.cs - lds_f32(csb + 4 * kB)) : 0.f;
+    d.safe = (__shfl_sync(0xffffffffu, d.cs, 0) - lds_f32(csb + 4 * wq)) <= kSafeBlockDecay;
     d.e = exp_dec(d.cs);
-    d.a_last = exp_dec(csb[4]);
+    d.a_last = exp_dec(lds_f32(csb + 16));
     return d;
 }
 
-template <typename TOut>
+// Named barriers: 1..4 per-warpgroup; the compute warps signal the issuing
+// warp with bar.arrive on 5 (operands ready), 6 (decay mask ready) and 7 (y
+// staged); 8 is compute-warps-only.
+constexpr uint32_t BAR_OPERANDS = 5, BAR_MASK = 6, BAR_YSTAGED = 7, BAR_COMPUTE = 8;
+constexpr uint32_t kCompute = 512;
+
+// The chunks one CTA sweeps.  Chains are (sequence, pair of heads): chain c
+// = sequence c / pairs, heads 2 (c % pairs) and 2 (c % pairs) + 1.
+//   * one CTA per chain (runs == 0): chain blockIdx.x, all of its chunks;
+//   * balanced (runs > 0, fixed-length sequences of nch chunks): the chains
+//     laid end to end are cut into `runs` runs of equal chunk counts, and run
+//     r covers global chunks [lo, hi).  It sweeps the head of its last chain
+//     cl (chunks [0, kl), ending at a cut: its carried state is handed on
+//     through slot r), then its whole chains, then the tail of its first
+//     chain cf (chunks [kf, nch), starting at a cut: its state comes from slot
+//     r - 1).  A tail is swept last and a head first, so a hand-off has long
+//     been written when it is read; a run inside one chain (cf == cl) reads
+//     at its start a state that the previous run wrote first, after a head of
+//     fewer chunks than one run.
+struct Sweep {
+    int nch;          // chunks per chain (balanced) or of this CTA's chain
+    int cf, kf;       // first chain and its first chunk
+    int cl, kl;       // last chain and the end (exclusive) of its chunks
+    int total;        // chunks swept
+};
+
+// Piece p of a sweep: chain and its chunk range [k0, k1).  Pieces are the
+// head of the last chain, the whole chains between, and the tail of the
+// first chain (one piece when the run lies in one chain).
+__device__ __forceinline__ void sweep_piece(const Sweep &w, int p, int &chain, int &k0, int &k1) {
+    if (w.cf == w.cl) { chain = w.cf; k0 = w.kf; k1 = w.kl; }
+    else if (p == 0) { chain = w.cl; k0 = 0; k1 = w.kl; }
+    else if (p < w.cl - w.cf) { chain = w.cf + p; k0 = 0; k1 = w.nch; }
+    else { chain = w.cf; k0 = w.kf; k1 = w.nch; }
+}
+
+// Position of a sweep: piece p, chunk k of its chain, and the chunk's token
+// rows.  step() moves to the next chunk; it divides (chain -> sequence) only
+// when it enters a new piece.
+struct Item {
+    int p, k, k1;   // piece, chunk, end (exclusive) of the piece's chunks
+    int s, pair;    // sequence and head pair of the chunk's chain
+    int t1, c0;     // end of the sequence's tokens; first token of the chunk
+};
+// Where a chain's tokens lie: [t0, t1) of the packed token axis.
+__device__ __forceinline__ void chain_span(const ScanArgs &a, int s, long &t0, long &t1) {
+    if (a.cu_seqlens) {
+        t0 = a.cu_seqlens[s];
+        t1 = a.cu_seqlens[s + 1];
+    } else {
+        t0 = (long)s * a.seqlen;
+        t1 = t0 + a.seqlen;
+    }
+}
+
+// The first chunk of piece p.
+__device__ __forceinline__ Item piece_item(const ScanArgs &a, const Sweep &w, int p, int pairs) {
+    Item it;
+    int chain, k0;
+    it.p = p;
+    sweep_piece(w, p, chain, k0, it.k1);
+    it.k = k0;
+    it.s = chain / pairs;
+    it.pair = chain - it.s * pairs;
+    long t0, t1;
+    chain_span(a, it.s, t0, t1);
+    it.t1 = (int)t1;
+    it.c0 = (int)(t0 + (long)k0 * kQ);
+    return it;
+}
+
+// The next chunk of the sweep.
+__device__ __forceinline__ void step(const ScanArgs &a, const Sweep &w, Item &it, int pairs) {
+    if (it.k + 1 < it.k1) {
+        ++it.k;
+        it.c0 += kQ;
+    } else {
+        it = piece_item(a, w, it.p + 1, pairs);
+    }
+}
+
+// Bounded acquire-spin on a hand-off flag written by another CTA.
+__device__ __forceinline__ bool wait_flag(const int *flag, unsigned long long wait_ns) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v) return true;
+    const uint64_t t0 = tc::globaltimer_ns(), lim = wait_limit(wait_ns);
+    for (;;) {
+        __nanosleep(256);
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v) return true;
+        if (tc::globaltimer_ns() - t0 > lim) return false;
+    }
+}
+
+// kPieces = false: one CTA per (sequence, head pair) chain, sweeping its
+// chunks in order.  kPieces = true (fixed-length batches, no slot pools): CTA
+// r sweeps run r of the chains laid end to end, cut into one run per CTA, and
+// hands the carried state across each cut through the caller's workspace.
+// Both instantiations share the per-chunk phases below; only the walk over
+// chunks differs.
+template <typename TOut, bool kPieces>
 __global__ void __launch_bounds__(kThreads, 1)
 scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y,
                const ScanArgs a)
 {
-    // bf16 y of full chunks is staged in shared memory and written by TMA;
+    // bf16 y of full chunks is staged in shared memory (the M tile of head 1,
+    // free between the y MMAs and the next chunk's mask) and written by TMA;
     // fp32 y and partial chunks are stored row by row.
     constexpr bool kStoreByTma = sizeof(TOut) == 2;
     const uint32_t sbase = tc::smem_u32(smem);
     const int tid = threadIdx.x;
+    const bool issuer = tid >= (int)kCompute;  // warp 16: TMA and MMA issue
+    const int wg = (tid >> 7) & 3;       // compute warpgroup 0..3
+    const int hd = wg & 1;               // head slot of the pair
+    const int ch = wg >> 1;              // column half
+    const int i = tid & 127;             // row / TMEM lane / d_state index
+    const int wq = i >> 5;               // warp within the warpgroup = 32-row block
     const int lane = tid & 31;
 
     const int H = a.nheads, G = a.ngroups;
     const int hpg = H / G;
     const int pairs = H >> 1;
-    const int s = blockIdx.x / pairs;
-    const int h0 = (blockIdx.x - s * pairs) * 2;
-    const int g = h0 / hpg;
 
-    if (sbase & 1023u) {                 // the swizzled layouts need 1024-B alignment
+    if (sbase & 1023u || (kPieces && (a.cu_seqlens || a.slot_idx || a.runs <= 0))) {
+        // the swizzled layouts need 1024-B alignment; runs cover fixed-length
+        // batches without slot pools only
         if (tid == 0) report_status(a.status_dev, kStatusInternal);
         return;
     }
 
-    long t0, t1;
-    if (a.cu_seqlens) {
-        const int c0 = a.cu_seqlens[0], cs0 = a.cu_seqlens[s], cs1 = a.cu_seqlens[s + 1];
-        const int cend = a.cu_seqlens[a.nseq];
-        if (c0 != 0 || cs1 < cs0 || cs0 < 0 || cend != a.seqlen || cs1 > a.seqlen) {
-            if (tid == 0) report_status(a.status_dev, kStatusDeviceInput);
-            return;
-        }
-        t0 = cs0; t1 = cs1;
-    } else {
-        t0 = (long)s * a.seqlen; t1 = t0 + a.seqlen;
-    }
-    const int nch = (int)((t1 - t0 + kQ - 1) / kQ);   // chunks of this sequence
-
-    size_t srow = (size_t)s;   // state row of this sequence
+    // ---- what this CTA sweeps ----
+    Sweep sw{};                 // kPieces: run r of the chains laid end to end
+    int s = 0, h0 = 0;          // otherwise: sequence s, heads h0, h0 + 1 ...
+    long t0 = 0, t1 = 0;        // ... over tokens [t0, t1)
+    size_t srow = 0;            // ... with state row srow
     bool load_init = a.initial_state != nullptr;
-    if (a.slot_idx) {
-        const int slot = a.slot_idx[s];
-        if (slot < 0 || slot >= a.max_slots) {
-            if (tid == 0) report_status(a.status_dev, kStatusDeviceInput);
+    if constexpr (kPieces) {
+        const int r = blockIdx.x;
+        sw.nch = (a.seqlen + kQ - 1) / kQ;
+        const long ctot = (long)a.nseq * pairs * sw.nch;
+        const long lo = ctot * r / a.runs, hi = ctot * (r + 1) / a.runs;
+        sw.cf = (int)(lo / sw.nch);
+        sw.kf = (int)(lo - (long)sw.cf * sw.nch);
+        sw.cl = (int)((hi - 1) / sw.nch);
+        sw.kl = (int)(hi - (long)sw.cl * sw.nch);
+        sw.total = (int)(hi - lo);
+        if (sw.total <= 0) {   // the host cuts at most one run per chunk
+            if (tid == 0) report_status(a.status_dev, kStatusInternal);
             return;
         }
-        srow = (size_t)slot;
-        if (a.has_initial && a.has_initial[s] == 0) load_init = false;
+    } else {
+        s = blockIdx.x / pairs;
+        h0 = (blockIdx.x - s * pairs) * 2;
+        if (a.cu_seqlens) {
+            const int c0 = a.cu_seqlens[0], cs0 = a.cu_seqlens[s], cs1 = a.cu_seqlens[s + 1];
+            const int cend = a.cu_seqlens[a.nseq];
+            if (c0 != 0 || cs1 < cs0 || cs0 < 0 || cend != a.seqlen || cs1 > a.seqlen) {
+                if (tid == 0) report_status(a.status_dev, kStatusDeviceInput);
+                return;
+            }
+        }
+        chain_span(a, s, t0, t1);
+        srow = (size_t)s;
+        if (a.slot_idx) {
+            const int slot = a.slot_idx[s];
+            if (slot < 0 || slot >= a.max_slots) {
+                if (tid == 0) report_status(a.status_dev, kStatusDeviceInput);
+                return;
+            }
+            srow = (size_t)slot;
+            if (a.has_initial && a.has_initial[s] == 0) load_init = false;
+        }
     }
 
-    const uint32_t bar0 = sbase + OFF_BAR;
-    auto bar = [&](uint32_t idx) { return bar0 + 8u * idx; };
+    const uint32_t sCSB = sbase + OFF_CSB + wg * 32;
+    const uint32_t sPART = sbase + OFF_PART + wg * 16;
+    const uint32_t bar_x = sbase + OFF_BAR, bar_cb = bar_x + 8, bar_sg = bar_x + 16;
+    const uint32_t bar_yo = bar_x + 24, bar_y = bar_x + 32, bar_drain = bar_x + 40;
 
     if (tid < 32) {
         tc::tmem_alloc(sbase + OFF_TM, TM_COLS);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(bar(BAR_X0), 1);
-        tc::mbar_init(bar(BAR_X1), 1);
-        tc::mbar_init(bar(BAR_CT), 1);
-        tc::mbar_init(bar(BAR_BT0), 1);
-        tc::mbar_init(bar(BAR_BT1), 1);
-        tc::mbar_init(bar(BAR_S), 1);
-        tc::mbar_init(bar(BAR_CRAW), 16);
-        tc::mbar_init(bar(BAR_CV0), 3);
-        tc::mbar_init(bar(BAR_CV1), 3);
-        tc::mbar_init(bar(BAR_DC0), 8);
-        tc::mbar_init(bar(BAR_DC1), 8);
-        tc::mbar_init(bar(BAR_SG), 1);
-        tc::mbar_init(bar(BAR_YO), 1);
-        tc::mbar_init(bar(BAR_Y), 1);
-        tc::mbar_init(bar(BAR_MASK), 16);
-        tc::mbar_init(bar(BAR_STATE), 16);
-        tc::mbar_init(bar(BAR_EPI), 16);
-        tc::mbar_init(bar(BAR_DRAIN), 1);
-        abort_flag() = 0;
-        range_flag() = 0;
+        tc::mbar_init(bar_x, 1);
+        tc::mbar_init(bar_cb, 1);
+        tc::mbar_init(bar_sg, 1);
+        tc::mbar_init(bar_yo, 1);
+        tc::mbar_init(bar_y, 1);
+        tc::mbar_init(bar_drain, 1);
+        flag_set(OFF_ABORT, 0);
+        flag_set(OFF_RANGE, 0);
         tc::fence_mbar_init();
     }
     tc::tc_fence_before();
@@ -522,331 +600,225 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     tc::tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_TM);
     bool ok = true;
-    float *vd_tab = reinterpret_cast<float *>(smem + OFF_VD);   // [2 buffers][2 heads][128]
-    float *wf_tab = reinterpret_cast<float *>(smem + OFF_WF);   // [2 buffers][2 heads][4]
 
-    if (tid >= kIssuerBase && tid < kComputeBase) {
-        // ================= TMA / MMA issuing thread =================
-        if (lane == 0) {
-            const bool produce = a.stall_producer == 0;
-            // Work in flight, for the drain after an abort: phases armed on the
-            // TMA barriers, and whether any MMA was issued.
-            uint32_t armed_x[2] = {0, 0}, armed_b[2] = {0, 0}, armed_c = 0;
-            bool mma_issued = false;
-            auto tile_row = [&](int k) { return (int)(t0 + (long)k * kQ); };
-            auto load_x = [&](int k) {
-                const uint32_t b = (uint32_t)k & 1u;
-                tc::mbar_arrive_expect_tx(bar(BAR_X0 + b), 2 * HALF);
-                tc::tma_load_3d(sbase + OFF_X + b * XBUF, &map_x, bar(BAR_X0 + b), 0, h0, tile_row(k));
-                tc::tma_load_3d(sbase + OFF_X + b * XBUF + HALF, &map_x, bar(BAR_X0 + b), 0, h0 + 1, tile_row(k));
-                ++armed_x[b];
-            };
-            auto load_c = [&](int k) {
-                tc::mbar_arrive_expect_tx(bar(BAR_CT), 2 * HALF);
-                tc::tma_load_3d(sbase + OFF_C, &map_c, bar(BAR_CT), 0, g, tile_row(k));
-                tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar(BAR_CT), 64, g, tile_row(k));
-                ++armed_c;
-            };
-            auto load_b = [&](int k) {
-                const uint32_t b = (uint32_t)k & 1u;
-                const uint32_t dst = b ? sbase + OFF_B1 : sbase + OFF_B;
-                tc::mbar_arrive_expect_tx(bar(BAR_BT0 + b), 2 * HALF);
-                tc::tma_load_3d(dst, &map_b, bar(BAR_BT0 + b), 0, g, tile_row(k));
-                tc::tma_load_3d(dst + HALF, &map_b, bar(BAR_BT0 + b), 64, g, tile_row(k));
-                ++armed_b[b];
-            };
-            auto store_y = [&](int k) {   // y tiles of full chunk k, staged in its x buffer
-                const uint32_t src = sbase + OFF_X + ((uint32_t)k & 1u) * XBUF;
-                tc::tma_store_3d(&map_y, src, 0, h0, tile_row(k));
-                tc::tma_store_3d(&map_y, src + HALF, 0, h0 + 1, tile_row(k));
-                tc::bulk_commit();
-            };
-            if (produce && nch > 0) {
-                load_c(0);
-                load_x(0);
-                load_b(0);
-                if (nch > 1) {
-                    load_x(1);
-                    load_b(1);
-                }
-                wait_or_abort(bar(BAR_CRAW), 0, ok, a.wait_ns);   // compute warps read C_0
-                if (ok && nch > 1) load_c(1);
-            }
-            for (int k = 0; k < nch && produce && ok; ++k) {
-                const uint32_t b = (uint32_t)k & 1u;
-                const uint32_t ph = (uint32_t)k & 1u;
-                // chunk k converted (B and x in fp16, w o x)
-                wait_or_abort(bar(BAR_CV0 + b), ((uint32_t)k >> 1) & 1u, ok, a.wait_ns);
-                // S_k overwrites TMEM that held M_{k-1}: Y_{k-1} must be done
-                if (k > 0) wait_or_abort(bar(BAR_Y), ph ^ 1u, ok, a.wait_ns);
-                if (!ok) break;
+    if (issuer) {
+        // ================= TMA / MMA issuing warp =================
+        const bool leader = lane == 0;
+        // descriptors (start-address field advanced by offset >> 4 per K step)
+        const uint64_t dBmn = tc::sdesc_sw128(sbase + OFF_B, HALF, 1024);   // B^T, MN-major
+        const uint64_t dW = tc::sdesc_sw128(sbase + OFF_WM, HALF, 1024);    // [wX_a | wX_b]
+        const uint64_t dBk = tc::sdesc_sw128(sbase + OFF_B, 16, 1024);      // B, K-major
+        const uint64_t dH = tc::sdesc_sw128(sbase + OFF_H, HALF, 1024);     // [H_a^T | H_b^T]
+        const uint64_t dXa = tc::sdesc_sw128(sbase + OFF_XH, HALF, 1024);
+        const uint64_t dXb = dXa + (HALF >> 4);
+        // Work in flight, for the drain after an abort: phases armed on the
+        // two load barriers, and whether any MMA was issued.
+        uint32_t nx_armed = 0, ncb_armed = 0;
+        bool mma_issued = false;
+        const bool produce = a.stall_producer == 0;
+        // x of heads hp, hp + 1 and C, B of group gg for the chunk at token row
+        auto load_x = [&](int hp, int row) {
+            tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
+            tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, hp, row);
+            tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, hp + 1, row);
+            ++nx_armed;
+        };
+        auto load_cb = [&](int gg, int row) {
+            tc::mbar_arrive_expect_tx(bar_cb, 4 * HALF);
+            tc::tma_load_3d(sbase + OFF_C, &map_c, bar_cb, 0, gg, row);
+            tc::tma_load_3d(sbase + OFF_C + HALF, &map_c, bar_cb, 64, gg, row);
+            tc::tma_load_3d(sbase + OFF_B, &map_b, bar_cb, 0, gg, row);
+            tc::tma_load_3d(sbase + OFF_B + HALF, &map_b, bar_cb, 64, gg, row);
+            ++ncb_armed;
+        };
+        // One chunk: S^T and G, then Yoff, once the operands are ready (the
+        // next chunk's x and C, B loads go out as their buffers free); Y once
+        // the decay mask is in TMEM; the y tiles once staged.
+        auto issue_chunk = [&](uint32_t phase, bool has_next, int hp_n, int row_n, int hp, int row,
+                               bool full) {
+            tc::named_sync(BAR_OPERANDS, kCompute + 32);
+            if (flag_get(OFF_ABORT)) ok = false;   // a compute warp's wait expired: issue nothing more
+            if (leader && ok && produce) {
+                tc::bulk_wait_read();   // previous y staging (in the M tiles) was read
+                if (has_next) load_x(hp_n, row_n);
                 tc::tc_fence_after();
-                const uint32_t sB = b ? sbase + OFF_B1 : sbase + OFF_B;
-                {
-                    const uint64_t dBmn = tc::sdesc_sw128(sB, HALF, 1024);               // B^T, MN-major
-                    const uint64_t dW = tc::sdesc_sw128(sbase + OFF_W, HALF, 1024);    // [wX_a | wX_b]
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_f16_ss(tmem + TM_S, dBmn + kk * 128, dW + kk * 128, IDESC_S2, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ss(tmem + TM_S, dBmn + kk * 128, dW + kk * 128, IDESC_S2, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
+                    tc::mma_f16_ts(tmem + TM_G, tmem + TM_C + kk * 8, dBk + ko, IDESC_G, kk > 0);
                 }
-                tc::mma_commit(bar(BAR_S));
+                tc::mma_commit(bar_sg);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ts(tmem + TM_YO, tmem + TM_C + kk * 8, dH + kk * 128, IDESC_YO2, kk > 0);
+                tc::mma_commit(bar_yo);
                 mma_issued = true;
-                // G_k overwrites Y_{k-1}, Yoff_k overwrites Yoff_{k-1}, and G_k needs C_k
-                // in TMEM: the epilogue of k-1 (which converts C_k) must be done
-                wait_or_abort(bar(BAR_EPI), ph, ok, a.wait_ns);
-                if (!ok) break;
-                if (k > 0 && kStoreByTma) store_y(k - 1);   // chunk k-1 is full (chunk k follows it)
-                tc::tc_fence_after();
-                const uint32_t tC = tmem + TM_C + 64u * b;
-                {
-                    const uint64_t dBk = tc::sdesc_sw128(sB, 16, 1024);                  // B, K-major
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t ko = (kk >> 2) * (HALF >> 4) + (kk & 3) * 2;
-                        tc::mma_f16_ts(tmem + TM_G, tC + kk * 8, dBk + ko, IDESC_G, kk > 0);
-                    }
-                }
-                tc::mma_commit(bar(BAR_SG));
-                // x of chunk k+1 into the buffer of chunk k-1, once Y_{k-1} has read
-                // x_{k-1} and the store of y_{k-1} (staged there) has read it
-                if (k > 0 && k + 1 < nch) {
-                    tc::bulk_wait_read();
-                    load_x(k + 1);
-                }
-                // Yoff_k reads H_{k-1}^T (the initial state's for k = 0)
-                wait_or_abort(bar(BAR_STATE), ph, ok, a.wait_ns);
-                if (!ok) break;
-                tc::tc_fence_after();
-                {
-                    const uint64_t dH = tc::sdesc_sw128(sbase + OFF_H, HALF, 1024);     // [H_a^T | H_b^T]
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_f16_ts(tmem + TM_YO, tC + kk * 8, dH + kk * 128, IDESC_YO2, kk > 0);
-                }
-                tc::mma_commit(bar(BAR_YO));
-                // B of chunk k+2 into this buffer once S_k and G_k have read B_k
-                wait_or_abort(bar(BAR_SG), ph, ok, a.wait_ns);
-                if (!ok) break;
-                if (k + 2 < nch) load_b(k + 2);
-                // Y_k needs the mask
-                wait_or_abort(bar(BAR_MASK), ph, ok, a.wait_ns);
-                if (!ok) break;
-                tc::tc_fence_after();
-                {
-                    const uint64_t dX = tc::sdesc_sw128(sbase + OFF_X + b * XBUF, HALF, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_f16_ts(tmem + TM_Y, tmem + TM_S + kk * 8, dX + kk * 128, IDESC_Y, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_f16_ts(tmem + TM_Y + 64, tmem + TM_S + 64 + kk * 8,
-                                       dX + (HALF >> 4) + kk * 128, IDESC_Y, kk > 0);
-                }
-                tc::mma_commit(bar(BAR_Y));
-                // C of chunk k+2 once the compute warps have read C_{k+1}
-                if (k + 2 < nch) {
-                    wait_or_abort(bar(BAR_CRAW), ((uint32_t)k + 1u) & 1u, ok, a.wait_ns);
-                    if (!ok) break;
-                    load_c(k + 2);
-                }
+                // The compute warps read C from shared memory before the operand
+                // barrier; B is read by the S and G MMAs only: both tiles are free
+                // once those complete.
+                wait_or_abort(bar_sg, phase, ok, a.wait_ns);
+                if (has_next && ok) load_cb(hp_n / hpg, row_n);
             }
-            // y of the last chunk
-            if (ok && produce && nch > 0) {
-                wait_or_abort(bar(BAR_EPI), (uint32_t)nch & 1u, ok, a.wait_ns);
-                if (ok && kStoreByTma && t0 + (long)nch * kQ <= t1) store_y(nch - 1);
+            __syncwarp();
+            tc::named_sync(BAR_MASK, kCompute + 32);
+            if (flag_get(OFF_ABORT)) ok = false;
+            if (leader && ok && produce) {
+                tc::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ts(tmem + TM_Y, tmem + TM_S + kk * 8, dXa + kk * 128, IDESC_Y, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_f16_ts(tmem + TM_Y + 64, tmem + TM_S + 64 + kk * 8, dXb + kk * 128, IDESC_Y, kk > 0);
+                tc::mma_commit(bar_y);
             }
+            __syncwarp();
+            tc::named_sync(BAR_YSTAGED, kCompute + 32);
+            if (flag_get(OFF_ABORT)) ok = false;
+            if (kStoreByTma && leader && ok && produce && full) {
+                // full chunk: both heads' y tiles by TMA
+                tc::tma_store_3d(&map_y, sbase + OFF_MB, 0, hp, row);
+                tc::tma_store_3d(&map_y, sbase + OFF_MB + HALF, 0, hp + 1, row);
+                tc::bulk_commit();
+            }
+            __syncwarp();
+        };
+        if constexpr (kPieces) {
+            Item itq = piece_item(a, sw, 0, pairs);   // the chunk being computed
+            if (leader && sw.total > 0 && produce) {
+                load_x(2 * itq.pair, itq.c0);
+                load_cb(2 * itq.pair / hpg, itq.c0);
+            }
+            uint32_t phase = 0;
+            for (int q = 0; q < sw.total; ++q, phase ^= 1u) {
+                const bool has_next = q + 1 < sw.total;
+                Item itn = itq;
+                if (has_next) step(a, sw, itn, pairs);
+                issue_chunk(phase, has_next, 2 * itn.pair, itn.c0, 2 * itq.pair, itq.c0,
+                            itq.c0 + kQ <= itq.t1);
+                itq = itn;
+            }
+        } else {
+            if (leader && t1 > t0 && produce) {
+                load_x(h0, (int)t0);
+                load_cb(h0 / hpg, (int)t0);
+            }
+            uint32_t phase = 0;
+            for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u) {
+                const long c1 = c0 + kQ;
+                issue_chunk(phase, c1 < t1, h0, (int)c1, h0, (int)c0, c1 <= t1);
+            }
+        }
+        if (leader) {
             if (!ok) {
                 // Aborted: wait (bounded) for every MMA issued and for the last
                 // phase armed on each load barrier, so that nothing writes TMEM
                 // or shared memory after they are released.
-                const uint64_t lim = wait_limit(a.wait_ns);
                 bool dok = true;
                 if (mma_issued) {
-                    tc::mma_commit(bar(BAR_DRAIN));
-                    tc::mbar_wait_bounded(bar(BAR_DRAIN), 0, dok, lim);
+                    tc::mma_commit(bar_drain);
+                    tc::mbar_wait_bounded(bar_drain, 0, dok, wait_limit(a.wait_ns));
                 }
-                for (int b = 0; b < 2; ++b) {
-                    bool xok = true;
-                    if (armed_x[b]) tc::mbar_wait_bounded(bar(BAR_X0 + b), (armed_x[b] - 1) & 1u, xok, lim);
-                }
-                for (int b = 0; b < 2; ++b) {
-                    bool bok = true;
-                    if (armed_b[b]) tc::mbar_wait_bounded(bar(BAR_BT0 + b), (armed_b[b] - 1) & 1u, bok, lim);
-                }
-                bool cok = true;
-                if (armed_c) tc::mbar_wait_bounded(bar(BAR_CT), (armed_c - 1) & 1u, cok, lim);
+                bool xok = true, cbok = true;
+                if (nx_armed) tc::mbar_wait_bounded(bar_x, (nx_armed - 1) & 1u, xok, wait_limit(a.wait_ns));
+                if (ncb_armed) tc::mbar_wait_bounded(bar_cb, (ncb_armed - 1) & 1u, cbok, wait_limit(a.wait_ns));
             }
             tc::bulk_wait_all();
         }
         __syncwarp();
-    } else if (tid < kConvThreads) {
-        // ================= converter warps: one chunk ahead =================
-        // 4096 jobs of one 16-byte chunk (8 values) per tile row: jobs 0..2047
-        // are x (head, row, chunk): x -> fp16 in place and w o x; jobs
-        // 2048..4095 are B (half, row, chunk) -> fp16 in place.  Thread t takes
-        // jobs t, t + 96, ...; a warp's 32 consecutive jobs cover 4 whole rows,
-        // so its 16-byte accesses hit every bank once per 128 bytes.
-        for (int k = 0; k < nch; ++k) {
-            const uint32_t b = (uint32_t)k & 1u;
-            const long c0 = t0 + (long)k * kQ;
-            const int Lc = (int)min((long)kQ, t1 - c0);
-            const uint32_t xt = sbase + OFF_X + b * XBUF;
-            wait_or_abort(bar(BAR_X0 + b), ((uint32_t)k >> 1) & 1u, ok, a.wait_ns);
-            wait_or_abort(bar(BAR_DC0 + b), ((uint32_t)k >> 1) & 1u, ok, a.wait_ns);
-            // w o x overwrites the tile S_{k-1} read
-            if (k >= 1) wait_or_abort(bar(BAR_S), ((uint32_t)k - 1u) & 1u, ok, a.wait_ns);
-            const float *vd = vd_tab + b * 256;
-            const float *wf = wf_tab + b * 8;
-#pragma unroll 4
-            for (int j = tid; j < 2048; j += kConvThreads) {
-                const int hd = j >> 10, row = (j >> 3) & 127, q = j & 7;
-                const uint32_t off = hd * HALF + sw128(row, q);
-                if (row < Lc) {
-                    const float w = wf[hd * 4 + (row >> 5)] * vd[hd * 128 + row];
-                    const uint4 v = lds128(xt + off);
-                    sts128(xt + off, cvt_chunk(v));
-                    sts128(sbase + OFF_W + off, cvt_chunk_scaled(v, w));
-                } else {
-                    sts128(xt + off, make_uint4(0, 0, 0, 0));
-                    sts128(sbase + OFF_W + off, make_uint4(0, 0, 0, 0));
-                }
-            }
-            wait_or_abort(bar(BAR_BT0 + b), ((uint32_t)k >> 1) & 1u, ok, a.wait_ns);
-            const uint32_t bt = b ? sbase + OFF_B1 : sbase + OFF_B;
-#pragma unroll 4
-            for (int j = tid; j < 2048; j += kConvThreads) {
-                const int hf = j >> 10, row = (j >> 3) & 127, q = j & 7;
-                const uint32_t addr = bt + hf * HALF + sw128(row, q);
-                sts128(addr, row < Lc ? cvt_chunk(lds128(addr)) : make_uint4(0, 0, 0, 0));
-            }
-            tc::fence_proxy_async_smem();
-            warp_arrive(bar(BAR_CV0 + b), lane);
-        }
-    } else if (tid >= kComputeBase) {
+    } else {
         // ================= compute warpgroups =================
-        const int ctid = tid - kComputeBase;
-        const int wg = ctid >> 7;            // compute warpgroup 0..3
-        const int hd = wg & 1;               // head slot of the pair
-        const int ch = wg >> 1;              // column half
-        const int i = ctid & 127;            // row / TMEM lane / d_state index
-        const int wq = i >> 5;               // warp within the warpgroup = 32-row block
-        const int hh = h0 + hd;
         const uint32_t tlane = (uint32_t)(wq * 32) << 16;
-        float *sCSB = reinterpret_cast<float *>(smem + OFF_CSB) + wg * 8;
-        float *sPART = reinterpret_cast<float *>(smem + OFF_PART) + wg * 4;
-        const size_t state_off = (srow * H + hh) * (size_t)(kP * kN) + (size_t)(32 * ch) * kN + i;
+        const uint32_t vd_tab = sbase + OFF_VD;     // float [2 buffers][2 heads][128]
+        const uint32_t csb_tab = sbase + OFF_CSBT;  // float [2 buffers][2 heads][8]
+        TOut *y = static_cast<TOut *>(a.y);
+        float Hs[32];   // carried state: d_state row i, head_dim entries 32 ch ..
 
-        // Row i's quarter wg of C_k (d_state n in [32 wg, 32 wg + 32)) as fp16
-        // pairs into TMEM C[k & 1] (lane i, columns 16 wg ..): the A operand
-        // of C.B^T and C.H^T.  Rows past the chunk end are zero.
-        auto convert_c = [&](int k) {
-            const long ck = t0 + (long)k * kQ;
-            const bool live_c = i < (int)min((long)kQ, t1 - ck);
-            wait_or_abort(bar(BAR_CT), (uint32_t)k & 1u, ok, a.wait_ns);
+        // ---- operands to fp16 (rows past the chunk end zeroed) ----
+        auto convert = [&](uint32_t phase, bool live, float w) {
+            wait_or_abort(bar_x, phase, ok, a.wait_ns);
+            wait_or_abort(bar_cb, phase, ok, a.wait_ns);
+            // warpgroup wg takes d_state columns n in [32 wg, 32 wg + 32) of row i:
+            // C as fp16 pairs into TMEM (lane i, columns 16 wg ..), B in place
             const uint32_t ctile = sbase + OFF_C + (wg >> 1) * HALF;
-            uint4 v[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                v[q] = live_c ? lds128(ctile + sw128(i, 4 * (wg & 1) + q)) : make_uint4(0, 0, 0, 0);
-            warp_arrive(bar(BAR_CRAW), lane);   // the C tile may be reloaded
+            const uint32_t btile = sbase + OFF_B + (wg >> 1) * HALF;
             uint32_t pc[16];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint4 u = cvt_chunk(v[q]);
-                pc[4 * q] = u.x; pc[4 * q + 1] = u.y; pc[4 * q + 2] = u.z; pc[4 * q + 3] = u.w;
+                const uint4 v = live ? cvt_chunk(lds128(ctile + sw128(i, 4 * (wg & 1) + q)))
+                                     : make_uint4(0, 0, 0, 0);
+                pc[4 * q] = v.x;
+                pc[4 * q + 1] = v.y;
+                pc[4 * q + 2] = v.z;
+                pc[4 * q + 3] = v.w;
             }
-            tc::tmem_st16(tmem + tlane + TM_C + 64u * ((uint32_t)k & 1u) + 16 * wg, pc);
-            tc::tmem_st_wait();
-        };
-
-        float Hs[32];
+            tc::tmem_st16(tmem + tlane + TM_C + 16 * wg, pc);
 #pragma unroll
-        for (int p = 0; p < 32; ++p)
-            Hs[p] = load_init ? state_load1(a.initial_state, state_off + (size_t)p * kN, a.rp) : 0.f;
-        write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
-        tc::fence_proxy_async_smem();
-        warp_arrive(bar(BAR_STATE), lane);     // H_{-1}^T ready for Yoff_0
-
-        const float Ah = a.A[hh];
-        const float Dh = a.D ? a.D[hh] : 0.f;
-        TOut *y = static_cast<TOut *>(a.y);
-        float *csb_tab = reinterpret_cast<float *>(smem + OFF_CSBT);   // [2 buffers][2 heads][8]
-        float2 cs_cur = make_float2(0.f, 0.f);   // (cs_i, dt_i) of the current chunk
-        if (nch > 0) {
-            convert_c(0);
-            tc::tc_fence_before();
-            warp_arrive(bar(BAR_EPI), lane);   // C_0 in TMEM for G_0
-            cs_cur = decay_scan(a, hh, Ah, load_dt(a, H, hh, t0, t1, i), (int)min((long)kQ, t1 - t0),
-                                i, wq, lane, wg, ch, sPART, sCSB, vd_tab + hd * 128, wf_tab + hd * 4,
-                                csb_tab + hd * 8);
-            if (ch == 0) warp_arrive(bar(BAR_DC0), lane);
-        }
-        tc::named_sync(NB_COMPUTE, kCompute);   // chunk 0's tables visible to every compute warp
-        float dt_n1 = load_dt(a, H, hh, t0 + kQ, t1, i);   // raw dt of the next chunk
-        for (int k = 0; k < nch; ++k) {
-            const uint32_t ph = (uint32_t)k & 1u, vb = (uint32_t)k & 1u;
-            const long c0 = t0 + (long)k * kQ;
-            const int Lc = (int)min((long)kQ, t1 - c0);
-            const long c1 = c0 + kQ;
-            const bool has_next = c1 < t1;
-            const bool live = i < Lc;
-            // dt two chunks ahead, so its load has a whole chunk to land
-            const float dt_n2 = load_dt(a, H, hh, c0 + 2 * kQ, t1, i);
-
-            const ChunkDecay cur = decay_derive(cs_cur, csb_tab + vb * 16 + hd * 8, wq, ch);
-            // ---- next chunk's decay, published for the converters (while S_k, G_k run) ----
-            float2 cs_nxt = make_float2(0.f, 0.f);
-            if (has_next) {
-                cs_nxt = decay_scan(a, hh, Ah, dt_n1, (int)min((long)kQ, t1 - c1), i, wq, lane, wg, ch,
-                                    sPART, sCSB, vd_tab + (vb ^ 1u) * 256 + hd * 128,
-                                    wf_tab + (vb ^ 1u) * 8 + hd * 4, csb_tab + (vb ^ 1u) * 16 + hd * 8);
-                if (ch == 0) warp_arrive(bar(BAR_DC0 + (vb ^ 1u)), lane);
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t addr = btile + sw128(i, 4 * (wg & 1) + q);
+                sts128(addr, live ? cvt_chunk(lds128(addr)) : make_uint4(0, 0, 0, 0));
             }
-
-            // ---- carried state: H <- exp(cs_L) H + S (d_state row i, p half ch) ----
-            wait_or_abort(bar(BAR_SG), ph, ok, a.wait_ns);
+#pragma unroll
+            for (int k = 4 * ch; k < 4 * ch + 4; ++k) {
+                const uint32_t off = hd * HALF + sw128(i, k);
+                if (live) {
+                    const uint4 r = lds128(sbase + OFF_XR + off);
+                    sts128(sbase + OFF_XH + off, cvt_chunk(r));
+                    sts128(sbase + OFF_WM + off, cvt_chunk_scaled(r, w));
+                } else {
+                    sts128(sbase + OFF_XH + off, make_uint4(0, 0, 0, 0));
+                    sts128(sbase + OFF_WM + off, make_uint4(0, 0, 0, 0));
+                }
+            }
+            tc::tmem_st_wait();
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            tc::named_arrive(BAR_OPERANDS, kCompute + 32);
+        };
+        // ---- carried state: H <- exp(cs_L) H + S (d_state row i, p half ch) ----
+        auto update_state = [&](uint32_t phase, float a_last) {
+            wait_or_abort(bar_sg, phase, ok, a.wait_ns);
             tc::tc_fence_after();
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-                uint32_t rr[16];
-                tc::tmem_ld16(tmem + tlane + TM_S + hd * 64 + ch * 32 + q * 16, rr);
+                uint32_t r[16];
+                tc::tmem_ld16(tmem + tlane + TM_S + hd * 64 + ch * 32 + q * 16, r);
                 tc::tmem_ld_wait();
-                const float2 al2 = make_float2(cur.a_last, cur.a_last);
+                const float2 al2 = make_float2(a_last, a_last);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float2 h2 = __ffma2_rn(al2, make_float2(Hs[q * 16 + 2 * e], Hs[q * 16 + 2 * e + 1]),
-                                                 make_float2(__uint_as_float(rr[2 * e]), __uint_as_float(rr[2 * e + 1])));
+                                                 make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])));
                     Hs[q * 16 + 2 * e] = h2.x;
                     Hs[q * 16 + 2 * e + 1] = h2.y;
                 }
             }
             tc::tc_fence_before();
-            tc::named_sync(NB_COMPUTE, kCompute);   // every S column read: M may overwrite them
+            tc::named_sync(BAR_COMPUTE, kCompute);   // every S column read: M may overwrite them
             tc::tc_fence_after();
-
-            // ---- decay mask M of head hd into TMEM (over S of this head) ----
-            {
-                const float *vd = vd_tab + vb * 256 + hd * 128;
-                const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
-                const uint32_t m_taddr = tmem + tlane + TM_S + hd * 64;
-                mask_block(tmem + tlane + TM_G, m_taddr, vd, kA, wq, lane, cur.uaA, cur.safe, cur.cs, cur.dtv, Dh);
-                mask_block(tmem + tlane + TM_G, m_taddr, vd, kB, wq, lane, cur.uaB, cur.safe, cur.cs, cur.dtv, Dh);
-                tc::tmem_st_wait();
-            }
+            if (flag_get(OFF_ABORT)) ok = false;
+        };
+        // ---- decay mask M of head hd into TMEM (over S of this head) ----
+        auto build_mask = [&](const ChunkDecay &cur, uint32_t vb, float Dh) {
+            const uint32_t vd = vd_tab + vb * 1024 + hd * 512;
+            const int kA = ch == 0 ? 0 : 1, kB = ch == 0 ? 3 : 2;
+            const uint32_t m_taddr = tmem + tlane + TM_S + hd * 64;
+            mask_block(tmem + tlane + TM_G, m_taddr, vd, kA, wq, lane, cur.uaA, cur.safe, cur.cs, cur.dtv, Dh);
+            mask_block(tmem + tlane + TM_G, m_taddr, vd, kB, wq, lane, cur.uaB, cur.safe, cur.cs, cur.dtv, Dh);
+            tc::tmem_st_wait();
             tc::tc_fence_before();
-            warp_arrive(bar(BAR_MASK), lane);
-
-            // ---- new H^T tile for the next chunk (Yoff_k read the old one) ----
-            wait_or_abort(bar(BAR_YO), ph, ok, a.wait_ns);
-            write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
-            tc::fence_proxy_async_smem();
-            warp_arrive(bar(BAR_STATE), lane);
-
-            // ---- C of the next chunk into TMEM (while the y MMAs run) ----
-            if (has_next) convert_c(k + 1);
-
-            // ---- y = Y + exp(cs_i) Yoff (row i, p half ch; D x is inside Y) ----
-            wait_or_abort(bar(BAR_Y), ph, ok, a.wait_ns);
+            tc::named_arrive(BAR_MASK, kCompute + 32);
+        };
+        // ---- y = Y + exp(cs_i) Yoff (row i, p half ch; D x is inside Y) ----
+        // An fp16 operand out of range (a bf16 input, a decay-masked C.B^T
+        // entry or a carried-state entry beyond 65504) turns some output into
+        // inf or NaN; each group of 16 outputs is summed and the range flag
+        // raised when a sum is not finite.
+        auto epilogue = [&](uint32_t phase, float e, bool full, bool live, TOut *yrow) {
+            wait_or_abort(bar_y, phase, ok, a.wait_ns);
             tc::tc_fence_after();
 #pragma unroll
             for (int q = 0; q < 2; ++q) {   // 16 columns at a time
@@ -855,7 +827,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 tc::tmem_ld16(tmem + tlane + TM_YO + hd * 64 + ch * 32 + q * 16, ro);
                 tc::tmem_ld_wait();
                 float out[16];
-                const float2 e2 = make_float2(cur.e, cur.e);
+                const float2 e2 = make_float2(e, e);
                 float2 ysum = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
@@ -865,22 +837,184 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                     out[2 * c + 1] = o2.y;
                     ysum = __fadd2_rn(ysum, o2);
                 }
-                if (!isfinite(ysum.x + ysum.y)) range_flag() = 1;
-                if (kStoreByTma && Lc == kQ) {   // into x_k's buffer: Y_k has read it
-                    stage16_bf16(sbase + OFF_X + vb * XBUF + hd * HALF, i, 4 * ch + 2 * q, out);
+                if (!isfinite(ysum.x + ysum.y)) flag_set(OFF_RANGE, 1);
+                if (kStoreByTma && full) {
+                    stage16_bf16(sbase + OFF_MB + hd * HALF, i, 4 * ch + 2 * q, out);
                 } else if (live) {
-                    store16(y + ((size_t)(c0 + i) * H + hh) * kP + 32 * ch + 16 * q, out);
+                    store16(yrow + 32 * ch + 16 * q, out);
                 }
             }
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
-            warp_arrive(bar(BAR_EPI), lane);
-            cs_cur = cs_nxt;
-            dt_n1 = dt_n2;
-        }
-        if (a.final_state) {
+            tc::named_arrive(BAR_YSTAGED, kCompute + 32);
+        };
+
+        if constexpr (!kPieces) {
+            const int hh = h0 + hd;
+            const size_t state_off = (srow * H + hh) * (size_t)(kP * kN) + (size_t)(32 * ch) * kN + i;
 #pragma unroll
-            for (int p = 0; p < 32; ++p) state_store1(a.final_state, state_off + (size_t)p * kN, Hs[p], a.rp);
+            for (int p = 0; p < 32; ++p)
+                Hs[p] = load_init ? state_load1(a.initial_state, state_off + (size_t)p * kN, a.rp) : 0.f;
+            write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+
+            const float Ah = a.A[hh];
+            const float Dh = a.D ? a.D[hh] : 0.f;
+            float3 dcur = make_float3(0.f, 0.f, 0.f);   // (cs_i, dt_i, w_i) of the current chunk
+            if (t1 > t0)
+                dcur = decay_scan(a, hh, Ah, load_dt(a, H, hh, t0, t1, i), (int)min((long)kQ, t1 - t0),
+                                  i, wq, lane, wg, ch, sPART, sCSB, vd_tab + hd * 512, csb_tab + hd * 32);
+            float dt_n1 = load_dt(a, H, hh, t0 + kQ, t1, i);   // raw dt of the next chunk
+            tc::named_sync(BAR_COMPUTE, kCompute);
+            uint32_t phase = 0, vb = 0;
+            for (long c0 = t0; c0 < t1; c0 += kQ, phase ^= 1u, vb ^= 1u) {
+                const int Lc = (int)min((long)kQ, t1 - c0);
+                const long c1 = c0 + kQ;
+                const bool has_next = c1 < t1;
+                const bool live = i < Lc;
+                const ChunkDecay cur = decay_derive(dcur, csb_tab + vb * 64 + hd * 32, wq, ch);
+
+                // dt two chunks ahead, so its load has a whole chunk to land
+                const float dt_n2 = load_dt(a, H, hh, c0 + 2 * kQ, t1, i);
+
+                convert(phase, live, cur.w);
+
+                // ---- next chunk's decay while the MMAs run ----
+                float3 dnxt = make_float3(0.f, 0.f, 0.f);
+                if (has_next)
+                    dnxt = decay_scan(a, hh, Ah, dt_n1, (int)min((long)kQ, t1 - c1), i, wq, lane, wg, ch,
+                                      sPART, sCSB, vd_tab + (vb ^ 1u) * 1024 + hd * 512,
+                                      csb_tab + (vb ^ 1u) * 64 + hd * 32);
+
+                update_state(phase, cur.a_last);
+                build_mask(cur, vb, Dh);
+
+                // ---- new H^T tile for the next chunk (Yoff of this chunk read the old one) ----
+                wait_or_abort(bar_yo, phase, ok, a.wait_ns);
+                write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+
+                epilogue(phase, cur.e, Lc == kQ, live, y + ((size_t)(c0 + i) * H + hh) * kP);
+                dcur = dnxt;
+                dt_n1 = dt_n2;
+            }
+            if (a.final_state) {
+#pragma unroll
+                for (int p = 0; p < 32; ++p) state_store1(a.final_state, state_off + (size_t)p * kN, Hs[p], a.rp);
+            }
+        } else {
+            const int r = blockIdx.x;
+            // This thread's 32 values of the state row of sequence sq, head hh.
+            auto state_at = [&](int sq, int hh) {
+                return ((size_t)sq * H + hh) * (size_t)(kP * kN) + (size_t)(32 * ch) * kN + i;
+            };
+            // Hand-off slot of cut rr: [2 heads][64 p][128 n] fp32; this thread's
+            // 32 values sit at (hd * 64 + 32 ch + p) * 128 + i.
+            auto slot_at = [&](int rr) {
+                return a.handoff + (size_t)rr * (2 * kP * kN) + (size_t)(hd * kP + 32 * ch) * kN + i;
+            };
+            // Carried state at the start of a piece: the initial state (or zero)
+            // at a chain start, else the state handed over through slot r - 1.
+            auto load_piece_state = [&](const Item &it) {
+                if (it.k == 0) {
+                    const size_t off = state_at(it.s, 2 * it.pair + hd);
+#pragma unroll
+                    for (int p = 0; p < 32; ++p)
+                        Hs[p] = load_init ? state_load1(a.initial_state, off + (size_t)p * kN, a.rp) : 0.f;
+                } else {
+                    if (tid == 0 && ok && !wait_flag(a.handoff_flags + (r - 1), a.wait_ns)) flag_set(OFF_ABORT, 1);
+                    tc::named_sync(BAR_COMPUTE, kCompute);
+                    const float *src = slot_at(r - 1);
+#pragma unroll
+                    for (int p = 0; p < 32; ++p) Hs[p] = __ldcg(src + (size_t)p * kN);
+                }
+            };
+            // Carried state at the end of a piece: the final state at a chain end,
+            // else handed on through slot r (written, fenced, then flagged).
+            auto store_piece_state = [&](const Item &it) {
+                if (it.c0 + kQ >= it.t1) {
+                    if (a.final_state) {
+                        const size_t off = state_at(it.s, 2 * it.pair + hd);
+#pragma unroll
+                        for (int p = 0; p < 32; ++p) state_store1(a.final_state, off + (size_t)p * kN, Hs[p], a.rp);
+                    }
+                } else {
+                    float *dst = slot_at(r);
+#pragma unroll
+                    for (int p = 0; p < 32; ++p) __stcg(dst + (size_t)p * kN, Hs[p]);
+                    __threadfence();
+                    tc::named_sync(BAR_COMPUTE, kCompute);
+                    if (tid == 0)
+                        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(a.handoff_flags + r), "r"(1) : "memory");
+                }
+            };
+
+            Item it = piece_item(a, sw, 0, pairs);
+            int hh = 2 * it.pair + hd;
+            float Ah = a.A[hh];
+            float Dh = a.D ? a.D[hh] : 0.f;
+            load_piece_state(it);
+            write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+            float3 dcur = decay_scan(a, hh, Ah, load_dt(a, H, hh, it.c0, it.t1, i), min(kQ, it.t1 - it.c0),
+                                     i, wq, lane, wg, ch, sPART, sCSB, vd_tab + hd * 512, csb_tab + hd * 32);
+            // first chunk of the next piece (the chunk after this piece's last)
+            const int npieces = sw.cf == sw.cl ? 1 : sw.cl - sw.cf + 1;
+            Item nxp = npieces > 1 ? piece_item(a, sw, 1, pairs) : it;
+            tc::named_sync(BAR_COMPUTE, kCompute);
+            uint32_t phase = 0, vb = 0;
+            int q = 0;
+            // Outer loop over pieces (the carried state is stored, handed on and
+            // loaded between them); the inner loop over a piece's chunks keeps the
+            // next chunk's operands and decay in flight across piece boundaries.
+            for (int pc_ = 0; pc_ < npieces; ++pc_) {
+                for (; it.k < it.k1; ++it.k, it.c0 += kQ, ++q, phase ^= 1u, vb ^= 1u) {
+                    const int c0 = it.c0;
+                    const int Lc = min(kQ, it.t1 - c0);
+                    const bool has_next = q + 1 < sw.total;
+                    const bool live = i < Lc;
+                    const ChunkDecay cur = decay_derive(dcur, csb_tab + vb * 64 + hd * 32, wq, ch);
+                    // the next chunk: in this piece, or the first of the next piece
+                    const bool same = it.k + 1 < it.k1;
+                    const int hh_n = same ? hh : 2 * nxp.pair + hd;
+                    const int c0_n = same ? c0 + kQ : nxp.c0;
+                    const int t1_n = same ? it.t1 : nxp.t1;
+                    // its raw dt, a whole conversion ahead of its decay
+                    const float dt_n1 = has_next ? load_dt(a, H, hh_n, c0_n, t1_n, i) : 0.f;
+
+                    convert(phase, live, cur.w);
+
+                    // ---- next chunk's decay while the MMAs run ----
+                    const float Ah_n = same ? Ah : a.A[hh_n];
+                    float3 dnxt = make_float3(0.f, 0.f, 0.f);
+                    if (has_next)
+                        dnxt = decay_scan(a, hh_n, Ah_n, dt_n1, min(kQ, t1_n - c0_n), i, wq, lane, wg, ch,
+                                          sPART, sCSB, vd_tab + (vb ^ 1u) * 1024 + hd * 512,
+                                          csb_tab + (vb ^ 1u) * 64 + hd * 32);
+
+                    update_state(phase, cur.a_last);
+                    build_mask(cur, vb, Dh);
+
+                    // ---- new H^T tile for the next chunk (Yoff of this chunk read the old one) ----
+                    wait_or_abort(bar_yo, phase, ok, a.wait_ns);
+                    write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+
+                    epilogue(phase, cur.e, Lc == kQ, live, y + ((size_t)(c0 + i) * H + hh) * kP);
+                    dcur = dnxt;
+                }
+                // ---- piece boundary: store or hand on the state, start the next piece
+                // (its H^T tile replaces the one the last chunk wrote before the next
+                // chunk's operands are released to the MMAs) ----
+                it.k = it.k1 - 1;
+                it.c0 -= kQ;
+                store_piece_state(it);
+                if (pc_ + 1 < npieces) {
+                    it = nxp;
+                    hh = 2 * it.pair + hd;
+                    Ah = a.A[hh];
+                    Dh = a.D ? a.D[hh] : 0.f;
+                    load_piece_state(it);
+                    write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+                    if (pc_ + 2 < npieces) nxp = piece_item(a, sw, pc_ + 2, pairs);
+                }
+            }
         }
     }
     tc::tc_fence_before();
@@ -889,9 +1023,9 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, TM_COLS);
     }
-    if (abort_flag()) {
+    if (flag_get(OFF_ABORT)) {
         if (tid == 0) report_status(a.status_dev, kStatusTimeout);
-    } else if (tid == 0 && range_flag()) {
+    } else if (tid == 0 && flag_get(OFF_RANGE)) {
         report_status(a.status_dev, kStatusRange);
     }
 }
@@ -944,21 +1078,77 @@ cudaError_t launch_tc_t(const ScanArgs &a, cudaStream_t stream)
     } else {
         my = mx;   // unused: fp32 y is stored row by row
     }
-    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<TOut>,
+    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel<TOut, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    if (a.runs > 0) {
+        e = cudaFuncSetAttribute(scan_tc_kernel<TOut, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        // Balanced: every run must be resident at once (a run may wait for a
+        // state another run hands over), which a cooperative launch
+        // guarantees or refuses; the hand-off flags start at zero.
+        e = cudaMemsetAsync(a.handoff_flags, 0, (size_t)a.runs * sizeof(int), stream);
+        if (e != cudaSuccess) return e;
+        ScanArgs ac = a;
+        void *args[] = {&mx, &mb, &mc, &my, &ac};
+        e = cudaLaunchCooperativeKernel((const void *)scan_tc_kernel<TOut, true>, dim3((unsigned)a.runs),
+                                        dim3(kThreads), args, SMEM_BYTES, stream);
+        if (e == cudaSuccess) return cudaSuccess;
+        (void)cudaGetLastError();   // not resident all at once: one CTA per chain instead
+    }
+    ScanArgs a1 = a;
+    a1.runs = 0;
     const dim3 grid((unsigned)((size_t)a.nseq * (a.nheads / 2)));
-    scan_tc_kernel<TOut><<<grid, kThreads, SMEM_BYTES, stream>>>(mx, mb, mc, my, a);
+    scan_tc_kernel<TOut, false><<<grid, kThreads, SMEM_BYTES, stream>>>(mx, mb, mc, my, a1);
     return cudaGetLastError();
+}
+
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
 }
 
 }  // namespace
 
+bool scan_tc_shape(int head_dim, int d_state, int chunk_size, int nheads, int ngroups)
+{
+    return head_dim == kP && d_state == kN && chunk_size == kQ && ngroups > 0 &&
+           nheads % ngroups == 0 && (nheads / ngroups) % 2 == 0;
+}
+
 bool scan_tc_supports(const ScanArgs &a)
 {
     const long long T = a.cu_seqlens ? (long long)a.seqlen : (long long)a.nseq * a.seqlen;
-    return a.in_dtype == 1 && a.head_dim == kP && a.d_state == kN && a.chunk_size == kQ &&
-           (a.nheads / a.ngroups) % 2 == 0 && T > 0 && encode_fn() != nullptr;
+    return a.in_dtype == 1 && scan_tc_shape(a.head_dim, a.d_state, a.chunk_size, a.nheads, a.ngroups) &&
+           T > 0 && encode_fn() != nullptr;
+}
+
+int scan_tc_balanced_runs(int nseq, int seqlen, int nheads)
+{
+    // One CTA per (sequence, head pair) chain leaves SMs idle when the chains
+    // do not fill whole waves; cutting the chains into one run per SM fills
+    // them.  A chain's chunks stay a sequential recurrence whichever runs
+    // sweep them, so with no more chains than SMs (one wave, each chain its
+    // own critical path) the cut gains nothing and is not used.
+    const int sms = sm_count();
+    const long long chains = (long long)nseq * (nheads / 2);
+    const long long nch = ((long long)seqlen + kQ - 1) / kQ;
+    if (sms <= 0 || chains <= sms || nch <= 0) return 0;
+    // A run's chunks cost about a tenth more than one chain's (the hand-offs,
+    // and a compute loop that also walks pieces): cut only when the last wave
+    // leaves more than a tenth of the SM slots idle.
+    const long long waves = (chains + sms - 1) / sms;
+    if (chains * 10 >= waves * sms * 9) return 0;
+    return sms;
+}
+
+size_t scan_tc_handoff_bytes(int runs)
+{
+    return (size_t)runs * (2 * kP * kN * sizeof(float)) + (size_t)runs * sizeof(int);
 }
 
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t stream)

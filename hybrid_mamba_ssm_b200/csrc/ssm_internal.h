@@ -83,6 +83,15 @@ struct ScanArgs {
     // (0 = the 2 s default), and a producer that issues no load or MMA.
     unsigned long long wait_ns;
     int stall_producer;
+    // Balanced schedule of the tensor-core scan (fixed-length batches only):
+    // `runs` CTAs split the chains (sequence, head pair) laid end to end into
+    // runs of equal chunk counts, handing the carried state across each cut
+    // through `handoff` (runs slots of 2 x head_dim x d_state fp32) and
+    // `handoff_flags` (runs ints, zeroed before the launch).  runs == 0: one
+    // CTA per chain.
+    int runs;
+    float *handoff;
+    int *handoff_flags;
 };
 
 // Causal depthwise conv1d (prefill over packed sequences, or one decode token
@@ -135,6 +144,12 @@ cudaError_t launch_scan_simt(const ScanArgs &a, cudaStream_t stream);
 // Tensor-core (tcgen05 / TMEM / TMA) chunked scan.  Returns
 // cudaErrorNotSupported, launching nothing, for shapes it does not cover.
 bool scan_tc_supports(const ScanArgs &a);
+bool scan_tc_shape(int head_dim, int d_state, int chunk_size, int nheads, int ngroups);
 cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t stream);
+// Balanced schedule: the number of runs (CTAs) for fixed-length sequences of
+// these sizes on the current device (0: one CTA per chain), and the hand-off
+// workspace it needs.
+int scan_tc_balanced_runs(int nseq, int seqlen, int nheads);
+size_t scan_tc_handoff_bytes(int runs);
 
 }  // namespace ssm

@@ -161,8 +161,17 @@ SSM_API int ssm_version(void);
  * y: device [T][nheads][head_dim], y_dtype (SSM_F32 or SSM_BF16, round to
  *   nearest even).  Must not overlap any input.
  * final_state: device fp32 [nseq][nheads][head_dim][d_state] or NULL.
- * workspace / workspace_bytes: reserved; pass NULL / 0 (the required size,
- *   ssd_chunk_scan_workspace_size, is 0 in this version).
+ * workspace / workspace_bytes: optional device scratch of at least
+ *   ssd_chunk_scan_workspace_size(...) bytes (16-byte aligned, not overlapping
+ *   any argument), or NULL / 0.  With it, fixed-length batches on the
+ *   tensor-core path run a balanced schedule: the (sequence, head pair)
+ *   chains laid end to end are cut into one run per SM, and the carried state
+ *   crosses each cut through the workspace (one fp32 [2][head_dim][d_state]
+ *   slot and one flag per run; the flags are zeroed on `stream` before the
+ *   launch).  Without it, or for packed varlen input, each chain runs in one
+ *   CTA.  The results are identical either way (the same chunk arithmetic in
+ *   the same order).  Calls that share a workspace must not overlap on the
+ *   GPU.
  * status_dev: device int32 or NULL; the kernels only ever write a nonzero
  *   status into it (the caller zeroes it).
  * stream: the CUDA stream to enqueue on (0 = legacy default stream).
@@ -178,7 +187,10 @@ SSM_API int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
                    void *workspace, size_t workspace_bytes,
                    int *status_dev, cudaStream_t stream);
 
-/* Workspace bytes ssd_chunk_scan needs for these shapes (0 in this version). */
+/* Workspace bytes ssd_chunk_scan can use for these shapes on the current
+ * device.  0 when no workspace helps: other shapes; no more chains than SMs
+ * (one wave, where every chain is already its own critical path); or chains
+ * that fill their last wave of SMs to nine tenths or more. */
 SSM_API size_t ssd_chunk_scan_workspace_size(int nseq, int seqlen, int nheads,
                                      int head_dim, int d_state, int ngroups,
                                      int chunk_size);

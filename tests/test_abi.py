@@ -65,8 +65,16 @@ def test_status_strings(lib):
     assert b"unknown" in lib.ssm_status_string(99)
 
 
-def test_workspace_size_is_zero(lib):
-    assert lib.ssd_chunk_scan_workspace_size(4, 4096, 128, 64, 128, 8, 128) == 0
+def test_workspace_size(lib):
+    # no workspace for shapes off the tensor-core path, nor for empty input
+    assert lib.ssd_chunk_scan_workspace_size(4, 4096, 128, 32, 128, 8, 128) == 0
+    assert lib.ssd_chunk_scan_workspace_size(4, 4096, 128, 64, 128, 8, 64) == 0
+    assert lib.ssd_chunk_scan_workspace_size(4, 4096, 12, 64, 128, 4, 128) == 0   # 3 heads per group
+    assert lib.ssd_chunk_scan_workspace_size(0, 4096, 128, 64, 128, 8, 128) == 0
+    # otherwise one 2 x 64 x 128 fp32 slot and one flag per run (per SM of the
+    # current device; no device here means no runs)
+    n = lib.ssd_chunk_scan_workspace_size(4, 4096, 128, 64, 128, 8, 128)
+    assert n % (65536 + 4) == 0
 
 
 # Fake, never-dereferenced device addresses: validation rejects the call first.
