@@ -730,6 +730,10 @@ def run_ours(args, world, rank, local, pg):
     phT = torch.empty((p["nseq"], p["H"], p["P"], p["N"]), dtype=torch.float32, device=dev)
     host_pre = dict(x=bf16(pin.x, True), dt=f32(pin.dt, True), B=bf16(pin.B, True),
                     C=bf16(pin.C, True))
+    # scan workspace: the balanced schedule, where the chains do not fill whole
+    # waves of SMs (both legs' scans run on one stream, so they share it)
+    n_ws = ssm.ssd_chunk_scan_workspace_size(p["nseq"], L, p["H"], p["P"], p["N"], p["G"], p["Q"])
+    pws = torch.empty(n_ws, dtype=torch.uint8, device=dev) if n_ws else None
 
     # decode: state, per-head params, a ring of per-step inputs
     dA, dD = synth.make_head_params(1001 + 7919 * rank, d["H"])
@@ -748,7 +752,8 @@ def run_ours(args, world, rank, local, pg):
     def prefill(x=px, dt=pdt, B=pB, C=pC):
         ssm.ssd_chunk_scan(shp(x, p["H"], p["P"]), shp(dt, p["H"]), pA,
                            shp(B, p["G"], p["N"]), shp(C, p["G"], p["N"]), pD, None,
-                           chunk_size=p["Q"], y=py, final_state=phT, stream=stream)
+                           chunk_size=p["Q"], y=py, final_state=phT, stream=stream,
+                           workspace=pws)
 
     def decode(k, inp=None):
         x, dt, B, C = inp if inp is not None else ring[k % RING]
@@ -826,7 +831,8 @@ def run_ours(args, world, rank, local, pg):
             stream.wait_event(ev_out[k % 2])             # outputs of step k-2 copied out
         ssm.ssd_chunk_scan(shp(sl["x"], p["H"], p["P"]), shp(sl["dt"], p["H"]), pA,
                            shp(sl["B"], p["G"], p["N"]), shp(sl["C"], p["G"], p["N"]), pD, None,
-                           chunk_size=p["Q"], y=sl["y"], final_state=sl["hT"], stream=stream)
+                           chunk_size=p["Q"], y=sl["y"], final_state=sl["hT"], stream=stream,
+                           workspace=pws)
         x, dt, B, C = sl["dec"]
         ssm.ssm_state_update(state, x, dt, dA, B, C, dD, y=sl["dy"], stream=stream)
         ev_comp[k % 2].record(stream)

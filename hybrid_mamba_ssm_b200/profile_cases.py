@@ -1,6 +1,7 @@
 """Small, self-contained launches of each kernel for profiling (ncu).
 
     python -m hybrid_mamba_ssm_b200.profile_cases prefill --nseq 1 --seqlen 4096 --heads 128
+    python -m hybrid_mamba_ssm_b200.profile_cases prefill --nseq 4 --seqlen 4096 --workspace
     python -m hybrid_mamba_ssm_b200.profile_cases decode --batch 16 --heads 256
     python -m hybrid_mamba_ssm_b200.profile_cases conv --nseq 1 --seqlen 8192
     python -m hybrid_mamba_ssm_b200.profile_cases conv_update --batch 64
@@ -42,8 +43,13 @@ def prefill(args, dev):
     A, D = _f32(inp.A, dev), _f32(inp.D, dev)
     y = torch.empty_like(x)
     hT = torch.empty((n, args.heads, args.head_dim, args.d_state), dtype=torch.float32, device=dev)
+    ws = None
+    if args.workspace:   # the balanced schedule, where it applies to these shapes
+        nb = ssm.ssd_chunk_scan_workspace_size(n, L, args.heads, args.head_dim, args.d_state,
+                                               args.groups, args.chunk)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
     return lambda: ssm.ssd_chunk_scan(x, dt, A, B, C, D, None, chunk_size=args.chunk, y=y,
-                                      final_state=hT)
+                                      final_state=hT, workspace=ws)
 
 
 def decode(args, dev):
@@ -115,6 +121,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--launches", type=int, default=1)
     ap.add_argument("--graph", action="store_true")
+    ap.add_argument("--workspace", action="store_true",
+                    help="prefill: pass the scan workspace (balanced schedule)")
     args = ap.parse_args()
     if args.heads is None:
         args.heads = 128 if args.case in ("prefill", "conv") else 256

@@ -157,14 +157,6 @@ def _dev(t, name, dtype=None):
     return t
 
 
-def scan_workspace_size(nseq, seqlen, nheads, head_dim=64, d_state=128, ngroups=8,
-                        chunk_size=128) -> int:
-    """Bytes of optional workspace ssd_chunk_scan can use for these shapes on the
-    current device (the balanced schedule of fixed-length batches); 0 if none."""
-    return int(lib.ssd_chunk_scan_workspace_size(nseq, seqlen, nheads, head_dim, d_state,
-                                                  ngroups, chunk_size))
-
-
 def ssd_chunk_scan(x, dt, A, B, C, D=None, initial_state=None, cu_seqlens=None,
                    chunk_size: int = 128, y=None, final_state=None, y_dtype=None,
                    return_final_state: bool = True, status=None, stream=None, workspace=None):
@@ -177,7 +169,7 @@ def ssd_chunk_scan(x, dt, A, B, C, D=None, initial_state=None, cu_seqlens=None,
     initial_state : [nseq, H, P, N] fp32 or None (zeros); may be ``final_state``
     cu_seqlens : int32 [nseq+1] CUDA tensor of packed offsets, or None
     y / final_state : optional preallocated outputs
-    workspace : optional CUDA tensor of at least scan_workspace_size(...) bytes
+    workspace : optional CUDA tensor of at least ssd_chunk_scan_workspace_size(...) bytes
         (fixed-length batches then run the balanced schedule)
     Returns (y, final_state) -- final_state is None if not requested.
     """
@@ -219,6 +211,8 @@ def ssd_chunk_scan(x, dt, A, B, C, D=None, initial_state=None, cu_seqlens=None,
 
 def ssd_chunk_scan_workspace_size(nseq, seqlen, nheads, head_dim, d_state, ngroups,
                                   chunk_size=128) -> int:
+    """Bytes of optional workspace ssd_chunk_scan can use for these shapes on the
+    current device (the balanced schedule of fixed-length batches); 0 if none."""
     return int(lib.ssd_chunk_scan_workspace_size(nseq, seqlen, nheads, head_dim, d_state,
                                                  ngroups, chunk_size))
 

@@ -84,12 +84,14 @@ def to_np(t):
 
 
 def scan_on_gpu(inp: synth.ScanInputs, chunk=128, y_dtype=torch.bfloat16, varlen=None,
-                initial_state=True, inplace=False, use_D=True, expect_status=0):
+                initial_state=True, inplace=False, use_D=True, expect_status=0, workspace=False):
     """Run ssd_chunk_scan on the inputs; returns (y, final_state) tensors.
 
     y and the final state are written into guarded buffers whose guard bands
     are checked after the call; the device status word must read
-    ``expect_status`` (0 unless a test provokes a device-side status)."""
+    ``expect_status`` (0 unless a test provokes a device-side status).  With
+    ``workspace`` a fixed-length call also gets the (guarded) scan workspace,
+    as bench.py passes it, where the shapes can use one."""
     from hybrid_mamba_ssm_b200 import ssm
     T, nseq = inp.T, inp.nseq
     lens = np.diff(inp.cu_seqlens)
@@ -118,11 +120,19 @@ def scan_on_gpu(inp: synth.ScanInputs, chunk=128, y_dtype=torch.bfloat16, varlen
                                    y=yg.t, final_state=hg.t, status=status)
     else:
         L = int(lens[0]) if nseq else 0
+        wsg = None
+        if workspace:
+            n = ssm.ssd_chunk_scan_workspace_size(nseq, L, H, P, N, G, chunk)
+            wsg = Guarded((n,), torch.uint8) if n else None
         y, hT = ssm.ssd_chunk_scan(x.view(nseq, L, H, P), dt.view(nseq, L, H), A,
                                    Bt.view(nseq, L, G, N), Ct.view(nseq, L, G, N), D, h0,
                                    chunk_size=chunk, y=yg.t.view(nseq, L, H, P),
-                                   final_state=hg.t, status=status)
+                                   final_state=hg.t, status=status,
+                                   workspace=None if wsg is None else wsg.t)
         y = y.view(T, H, P)
+        if wsg is not None:
+            torch.cuda.synchronize()
+            wsg.check("workspace")
     torch.cuda.synchronize()
     yg.check("y")
     hg.check("final_state")

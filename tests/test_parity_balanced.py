@@ -31,7 +31,7 @@ def _run(inp, nseq, L, H, G, workspace, y_dtype=torch.bfloat16):
     hg = Guarded((nseq, H, P, N), torch.float32)
     wsg = None
     if workspace:
-        n = ssm.scan_workspace_size(nseq, L, H, P, N, G, 128)
+        n = ssm.ssd_chunk_scan_workspace_size(nseq, L, H, P, N, G, 128)
         assert n > 0, "the balanced schedule should apply to this shape"
         wsg = Guarded((n,), torch.uint8)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")

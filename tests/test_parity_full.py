@@ -1,5 +1,6 @@
-"""Full-size workloads in the benchmark's launch configuration, checked on
-sampled heads (and batch rows) that the oracle computes one by one.
+"""Full-size workloads in the benchmark's launch configuration (the prefill
+with the scan workspace, as bench.py passes it), checked on sampled heads (and
+batch rows) that the oracle computes one by one.
 
 * prefill 4 x 4096 tokens, 128 heads (bf16 in, bf16 y, zero initial state);
 * long prefill 1 x 32768 tokens, 256 heads, nonzero initial state;
@@ -32,7 +33,7 @@ def _workload_inputs(name):
                                         ("prefill_ultra_32k", list(range(192, 224)) + [0, 95])])
 def test_full_prefill_sampled_heads(name, heads):
     inp = _workload_inputs(name)
-    y, hT = scan_on_gpu(inp, chunk=128, y_dtype=torch.bfloat16)
+    y, hT = scan_on_gpu(inp, chunk=128, y_dtype=torch.bfloat16, workspace=True)
     y = y[:, heads]
     hT = hT[:, heads]
     y_ref, h_ref = oracle_scan(inp, heads=heads)
