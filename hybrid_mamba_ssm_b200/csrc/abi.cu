@@ -89,6 +89,7 @@ const char *ssm_status_string(int status)
     case SSM_ERR_DEVICE_INPUT: return "SSM_ERR_DEVICE_INPUT: inconsistent cu_seqlens or slot index";
     case SSM_ERR_RANGE: return "SSM_ERR_RANGE: a value beyond the fp16 range of the tensor-core operands";
     case SSM_ERR_INTERNAL: return "SSM_ERR_INTERNAL: launch configuration broke a kernel layout rule";
+    case SSM_ERR_SCRATCH_LIMIT: return "SSM_ERR_SCRATCH_LIMIT: workspace needed exceeds the built-in scratch";
     default: return "unknown ssm status";
     }
 }

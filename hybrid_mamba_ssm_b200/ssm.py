@@ -37,6 +37,9 @@ def _load():
     lib.ssd_chunk_scan.restype = i
     lib.ssd_chunk_scan.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp,
                                    vp, vp, i, vp, vp, vp, sz, vp, vp]
+    lib.ssd_chunk_scan_noalloc.restype = i
+    lib.ssd_chunk_scan_noalloc.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp,
+                                           vp, vp, i, vp, vp, vp, vp]
     lib.ssd_chunk_scan_workspace_size.restype = sz
     lib.ssd_chunk_scan_workspace_size.argtypes = [i] * 7
     lib.ssm_state_update.restype = i
@@ -206,6 +209,43 @@ def ssd_chunk_scan(x, dt, A, B, C, D=None, initial_state=None, cu_seqlens=None,
                             0 if workspace is None else workspace.numel() * workspace.element_size(),
                             _ptr(status), _stream(stream))
     _check(st, "ssd_chunk_scan")
+    return y, final_state
+
+
+def ssd_chunk_scan_noalloc(x, dt, A, B, C, y, final_state=None, D=None, initial_state=None,
+                           cu_seqlens=None, chunk_size: int = 128, status=None, stream=None):
+    """ssd_chunk_scan with its workspace taken from the library's built-in
+    scratch; nothing here allocates, so y (and final_state, if wanted) must be
+    given.  Layouts as for ssd_chunk_scan.  For callers that must not allocate
+    device memory (a pool owned by another framework, or no allocator at
+    hand).  The first call on a device looks up the scratch's address; calls
+    whose launches overlap on the GPU race on the one scratch per device."""
+    _dev(x, "x")
+    in_code = _dtype_code(x.dtype)
+    if cu_seqlens is not None:
+        _dev(cu_seqlens, "cu_seqlens", torch.int32)
+        T, H, P = x.shape
+        nseq = cu_seqlens.shape[0] - 1
+        seqlen = T
+    else:
+        nseq, seqlen, H, P = x.shape
+    G, N = B.shape[-2], B.shape[-1]
+    _dev(dt, "dt", torch.float32)
+    _dev(A, "A", torch.float32)
+    _dev(B, "B", x.dtype)
+    _dev(C, "C", x.dtype)
+    _dev(D, "D", torch.float32)
+    _dev(initial_state, "initial_state", torch.float32)
+    if y is None:
+        raise ValueError("ssd_chunk_scan_noalloc: y must be preallocated")
+    _dev(y, "y", y.dtype)
+    _dev(final_state, "final_state", torch.float32)
+    _dev(status, "status", torch.int32)
+    st = lib.ssd_chunk_scan_noalloc(nseq, seqlen, _ptr(cu_seqlens), H, P, N, G, int(chunk_size),
+                                    in_code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
+                                    _ptr(D), _ptr(initial_state), _dtype_code(y.dtype), _ptr(y),
+                                    _ptr(final_state), _ptr(status), _stream(stream))
+    _check(st, "ssd_chunk_scan_noalloc")
     return y, final_state
 
 

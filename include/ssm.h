@@ -62,8 +62,10 @@ typedef enum {
     SSM_ERR_DEVICE_INPUT = 6,  /* written to status_dev: bad cu_seqlens or slot index */
     SSM_ERR_RANGE = 7,         /* written to status_dev: a value beyond the fp16 range of the
                                   tensor-core operands made y non-finite (see ssd_chunk_scan) */
-    SSM_ERR_INTERNAL = 8       /* written to status_dev: a launch broke a kernel's own layout
+    SSM_ERR_INTERNAL = 8,      /* written to status_dev: a launch broke a kernel's own layout
                                   rule (e.g. shared-memory alignment); nothing was computed */
+    SSM_ERR_SCRATCH_LIMIT = 9  /* ssd_chunk_scan_noalloc: the shapes need more workspace than
+                                  the library's built-in scratch holds; nothing launched */
 } ssm_status;
 
 typedef enum {
@@ -194,6 +196,50 @@ SSM_API int ssd_chunk_scan(int nseq, int seqlen, const int32_t *cu_seqlens,
 SSM_API size_t ssd_chunk_scan_workspace_size(int nseq, int seqlen, int nheads,
                                      int head_dim, int d_state, int ngroups,
                                      int chunk_size);
+
+/* Size of the scratch built into the library for ssd_chunk_scan_noalloc
+ * (one static device array per device the library runs on). */
+#define SSM_NOALLOC_SCRATCH_BYTES ((size_t)10 << 20)
+
+/*
+ * ssd_chunk_scan_noalloc -- ssd_chunk_scan whose workspace comes from scratch
+ * memory built into the library rather than from the caller.  The method has
+ * no counterpart to this: it is a convenience of the library.
+ *
+ * It exists for callers that cannot provide device memory: C or C++ hosts
+ * that have no device allocator of their own, and serving processes whose
+ * device memory is already reserved by another framework's pool, where a
+ * cudaMalloc would take memory outside that pool and a cudaFree would
+ * synchronise the device.  Nothing in this call allocates.  The balanced
+ * schedule's hand-off slots and flags (ssd_chunk_scan_workspace_size bytes)
+ * live in a static device array of SSM_NOALLOC_SCRATCH_BYTES.
+ *
+ * Arguments, layouts, results and statuses are those of ssd_chunk_scan with
+ * that scratch as the workspace; the results are identical.  Shapes that
+ * need no workspace run as ssd_chunk_scan does without one.  Shapes whose
+ * workspace would exceed the scratch return SSM_ERR_SCRATCH_LIMIT and
+ * launch nothing.
+ *
+ * Setup: the first call on each device, made with that device current,
+ * looks up the scratch's device address with cudaGetSymbolAddress (which
+ * loads the library's device code on that device if it is not loaded yet)
+ * and keeps it for later calls; a failed lookup returns SSM_ERR_CUDA.  Make
+ * that first call before any stream capture begins.  Each call zeroes the
+ * hand-off flags on `stream` with a memset before its launch; the slots need
+ * no clearing.
+ *
+ * There is one scratch per device: calls whose work overlaps on the GPU
+ * (launched on different streams, or from different host threads, without
+ * ordering between them) race on it, so the caller must order them.
+ */
+SSM_API int ssd_chunk_scan_noalloc(int nseq, int seqlen, const int32_t *cu_seqlens,
+                           int nheads, int head_dim, int d_state, int ngroups,
+                           int chunk_size, int in_dtype,
+                           const void *x, const float *dt, const float *A,
+                           const void *B, const void *C, const float *D,
+                           const float *initial_state,
+                           int y_dtype, void *y, float *final_state,
+                           int *status_dev, cudaStream_t stream);
 
 /*
  * ssm_state_update -- decode: one token per batch element, applied in place

@@ -59,7 +59,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(9):
+    for code in range(10):
         assert lib.ssm_status_string(code)
         assert b"unknown" not in lib.ssm_status_string(code)
     assert b"unknown" in lib.ssm_status_string(99)
@@ -75,6 +75,27 @@ def test_workspace_size(lib):
     # current device; no device here means no runs)
     n = lib.ssd_chunk_scan_workspace_size(4, 4096, 128, 64, 128, 8, 128)
     assert n % (65536 + 4) == 0
+
+
+def test_noalloc_validates_like_ssd_chunk_scan(lib):
+    # Without a device no shape needs the built-in scratch, so the call goes
+    # straight to ssd_chunk_scan's host validation (nothing is launched).
+    f = lib.ssd_chunk_scan_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    f.restype = i
+    f.argtypes = [i, i, vp, i, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp]
+    args = [1, 128, None, 4, 64, 128, 1, 128, BF16, 0x10000, 0x20000, 0x30000, 0x40000,
+            0x50000, None, None, BF16, 0x60000, 0x70000, None, None]
+    bad = list(args)
+    bad[0] = -1                       # nseq
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[3], bad[6] = 6, 4             # heads not a multiple of groups
+    assert f(*bad) == INVALID
+    bad = list(args)
+    bad[17] = 0x60008                 # y only 8-byte aligned
+    assert f(*bad) == MISALIGNED
+    assert b"SCRATCH" in lib.ssm_status_string(9)
 
 
 # Fake, never-dereferenced device addresses: validation rejects the call first.
