@@ -738,7 +738,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         float Hs[32];   // carried state: d_state row i, head_dim entries 32 ch ..
 
         // ---- operands to fp16 (rows past the chunk end zeroed) ----
-        auto convert = [&](uint32_t phase, bool live, float w) {
+        // (w o x already written when wm_ready: see convert_wm)
+        auto convert = [&](uint32_t phase, bool live, float w, bool wm_ready) {
             wait_or_abort(bar_x, phase, ok, a.wait_ns);
             wait_or_abort(bar_cb, phase, ok, a.wait_ns);
             // warpgroup wg takes d_state columns n in [32 wg, 32 wg + 32) of row i:
@@ -767,16 +768,28 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 if (live) {
                     const uint4 r = lds128(sbase + OFF_XR + off);
                     sts128(sbase + OFF_XH + off, cvt_chunk(r));
-                    sts128(sbase + OFF_WM + off, cvt_chunk_scaled(r, w));
+                    if (!wm_ready) sts128(sbase + OFF_WM + off, cvt_chunk_scaled(r, w));
                 } else {
                     sts128(sbase + OFF_XH + off, make_uint4(0, 0, 0, 0));
-                    sts128(sbase + OFF_WM + off, make_uint4(0, 0, 0, 0));
+                    if (!wm_ready) sts128(sbase + OFF_WM + off, make_uint4(0, 0, 0, 0));
                 }
             }
             tc::tmem_st_wait();
             tc::fence_proxy_async_smem();
             tc::tc_fence_before();
             tc::named_arrive(BAR_OPERANDS, kCompute + 32);
+        };
+        // ---- w o x of the next chunk while this chunk's Y MMAs run: its raw x
+        // has landed by then (requested at this chunk's operand barrier), and
+        // the S MMA that read this chunk's w o x has completed ----
+        auto convert_wm = [&](uint32_t phase_n, bool live_n, float w_n) {
+            wait_or_abort(bar_x, phase_n, ok, a.wait_ns);
+#pragma unroll
+            for (int k = 4 * ch; k < 4 * ch + 4; ++k) {
+                const uint32_t off = hd * HALF + sw128(i, k);
+                sts128(sbase + OFF_WM + off, live_n ? cvt_chunk_scaled(lds128(sbase + OFF_XR + off), w_n)
+                                                    : make_uint4(0, 0, 0, 0));
+            }
         };
         // ---- carried state: H <- exp(cs_L) H + S (d_state row i, p half ch) ----
         auto update_state = [&](uint32_t phase, float a_last) {
@@ -876,7 +889,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 // dt two chunks ahead, so its load has a whole chunk to land
                 const float dt_n2 = load_dt(a, H, hh, c0 + 2 * kQ, t1, i);
 
-                convert(phase, live, cur.w);
+                convert(phase, live, cur.w, c0 != t0);
 
                 // ---- next chunk's decay while the MMAs run ----
                 float3 dnxt = make_float3(0.f, 0.f, 0.f);
@@ -891,6 +904,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 // ---- new H^T tile for the next chunk (Yoff of this chunk read the old one) ----
                 wait_or_abort(bar_yo, phase, ok, a.wait_ns);
                 write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+                if (has_next) convert_wm(phase ^ 1u, c1 + i < t1, dnxt.z);
 
                 epilogue(phase, cur.e, Lc == kQ, live, y + ((size_t)(c0 + i) * H + hh) * kP);
                 dcur = dnxt;
@@ -979,7 +993,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                     // its raw dt, a whole conversion ahead of its decay
                     const float dt_n1 = has_next ? load_dt(a, H, hh_n, c0_n, t1_n, i) : 0.f;
 
-                    convert(phase, live, cur.w);
+                    convert(phase, live, cur.w, q > 0);
 
                     // ---- next chunk's decay while the MMAs run ----
                     const float Ah_n = same ? Ah : a.A[hh_n];
@@ -995,6 +1009,7 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                     // ---- new H^T tile for the next chunk (Yoff of this chunk read the old one) ----
                     wait_or_abort(bar_yo, phase, ok, a.wait_ns);
                     write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
+                    if (has_next) convert_wm(phase ^ 1u, c0_n + i < t1_n, dnxt.z);
 
                     epilogue(phase, cur.e, Lc == kQ, live, y + ((size_t)(c0 + i) * H + hh) * kP);
                     dcur = dnxt;
