@@ -172,3 +172,30 @@ def test_verify_only_against_oracle(ntok, dtype, P):
     yn = to_np(y)
     assert rel_err(yn[live], y_ref) < TOL
     assert (yn[~live] == 7.0).all()
+
+
+def test_verify_only_many_slices():
+    """The y-only verify at a size where every SM runs many (row, head)
+    slices: 24 rows of 128 heads in 8 groups, a shuffled slot map with
+    padding rows between live ones; all heads against the oracle."""
+    from hybrid_mamba_ssm_b200 import ssm
+    H, P, N, G, ntok, max_slots = 128, 64, 128, 8, 4, 30
+    rng = np.random.default_rng(291)
+    slots = rng.permutation(max_slots)[:24].astype(np.int32)
+    slots[[5, 17]] = -1                                   # padding rows
+    batch = slots.shape[0]
+    A, D = synth.make_head_params(292, H)
+    pool0 = synth.make_state(293, (max_slots, H, P, N))
+    (x, dt, B, C), (xd, dtd, Bd, Cd) = _draft(294, batch, ntok, H, P, N, G, "bf16")
+    pool = dev_f32(pool0)
+    y = torch.full((batch, ntok, H, P), 7.0, device="cuda")
+    ssm.ssm_state_update_multi(pool, xd, dtd, dev_f32(A), Bd, Cd, dev_f32(D),
+                               slot_idx=torch.from_numpy(slots).cuda(), y=y)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(pool), pool0.astype(np.float64))   # only read
+    live = slots >= 0
+    y_ref, _, _ = oracle.state_update_multi(pool0[slots[live]], x[live], dt[live], A, B[live],
+                                            C[live], D)
+    yn = to_np(y)
+    assert rel_err(yn[live], y_ref) < TOL
+    assert (yn[~live] == 7.0).all()
