@@ -18,8 +18,11 @@
 //   y    = Y + exp(cs_i) Yoff,   H <- exp(cs_{L-1}) H + S
 // The diagonal j = i belongs to M because the output reads the updated state.
 //
-// Work decomposition: one CTA per (sequence, pair of heads of one group),
-// sweeping the sequence's chunks in order.  544 threads: four compute
+// Work decomposition: a CTA sweeps the chunks of (sequence, pair of heads of
+// one group) chains in order: one chain per CTA, or (with the caller's
+// workspace, for fixed-length batches with more chains than SMs) one run per
+// SM of the chains laid end to end, the carried state crossing each cut
+// through the workspace.  544 threads: four compute
 // warpgroups and one issuing warp.  Compute warpgroup wg works on head
 // 2k + (wg & 1) and on half (wg >> 1) of the columns: thread i of it owns TMEM
 // lane i (row i of G, M, Y, Yoff; d_state index i of S^T and of the carried
@@ -31,13 +34,14 @@
 // Pipeline per chunk (single-buffered tiles, with prefetch where a buffer
 // frees early):
 //   wait TMA(x), TMA(B, C) -> convert bf16 -> fp16 (C into TMEM and B in
-//   place, a quarter of d_state per warpgroup; x and w o x per head)
+//   place, a quarter of d_state per warpgroup; x per head)
 //   -> issue TMA(x of next chunk) into the raw x buffers
 //   -> MMA S^T (2 heads), G  [commit] , Yoff (2 heads) [commit]
 //   -> the next chunk's cumulative decay (while the MMAs run)
 //   -> issue TMA(B, C of next chunk) once S^T and G are done
 //   -> state update from S^T, decay mask M per head (overlap the Yoff MMAs)
-//   -> MMA Y (2 heads) [commit] -> epilogue y.
+//   -> MMA Y (2 heads) [commit]; meanwhile w o x of the next chunk, whose
+//      raw x has landed -> epilogue y.
 //
 // Precision: bf16 inputs are converted to fp16 (exact for |v| < 65504) so the
 // derived operands M, w o x and H (rounded to fp16, 11 significant bits) keep
