@@ -620,11 +620,14 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
         uint32_t nx_armed = 0, ncb_armed = 0;
         bool mma_issued = false;
         const bool produce = a.stall_producer == 0;
+        // x and y are touched once (evict-first in L2); B and C are read by
+        // every head pair of their group, and keep the default policy.
+        const uint64_t once = tc::l2_evict_first_policy();
         // x of heads hp, hp + 1 and C, B of group gg for the chunk at token row
         auto load_x = [&](int hp, int row) {
             tc::mbar_arrive_expect_tx(bar_x, 2 * HALF);
-            tc::tma_load_3d(sbase + OFF_XR, &map_x, bar_x, 0, hp, row);
-            tc::tma_load_3d(sbase + OFF_XR + HALF, &map_x, bar_x, 0, hp + 1, row);
+            tc::tma_load_3d_hint(sbase + OFF_XR, &map_x, bar_x, 0, hp, row, once);
+            tc::tma_load_3d_hint(sbase + OFF_XR + HALF, &map_x, bar_x, 0, hp + 1, row, once);
             ++nx_armed;
         };
         auto load_cb = [&](int gg, int row) {
@@ -684,8 +687,8 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             if (flag_get(OFF_ABORT)) ok = false;
             if (kStoreByTma && leader && ok && produce && full) {
                 // full chunk: both heads' y tiles by TMA
-                tc::tma_store_3d(&map_y, sbase + OFF_MB, 0, hp, row);
-                tc::tma_store_3d(&map_y, sbase + OFF_MB + HALF, 0, hp + 1, row);
+                tc::tma_store_3d_hint(&map_y, sbase + OFF_MB, 0, hp, row, once);
+                tc::tma_store_3d_hint(&map_y, sbase + OFF_MB + HALF, 0, hp + 1, row, once);
                 tc::bulk_commit();
             }
             __syncwarp();
