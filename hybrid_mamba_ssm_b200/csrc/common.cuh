@@ -139,7 +139,7 @@ __device__ __forceinline__ float state_load1(const void *base, size_t e, const R
 }
 __device__ __forceinline__ void state_store1(void *base, size_t e, float v, const RoundParams &p) {
     if (!p.f16) {
-        static_cast<float *>(base)[e] = v;
+        __stcs(static_cast<float *>(base) + e, v);   // written once: streaming (evict-first)
         return;
     }
     uint32_t r = 0;
