@@ -108,9 +108,21 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
+// bf16 pair (low half first) -> two floats, exactly: a mixed-precision add of
+// -0 to each bf16 half, which runs on the FMA pipes and needs no unpacking
+// shifts or masks on the ALU (the compute warps' busiest pipe).
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
+    float lo, hi;
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.bf16 %0, l, 0f80000000;\n\t"
+        "add.rn.f32.bf16 %1, h, 0f80000000;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(v));
+    return make_float2(lo, hi);
+}
+
 __device__ __forceinline__ uint32_t bf2_to_h2(uint32_t v, float scale) {
-    const float2 p = __fmul2_rn(make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u)),
-                                make_float2(scale, scale));
+    const float2 p = __fmul2_rn(bf2_to_f2(v), make_float2(scale, scale));
     __half2 h = __floats2half2_rn(p.x, p.y);
     return *reinterpret_cast<uint32_t *>(&h);
 }
@@ -191,7 +203,8 @@ __device__ __forceinline__ void store16(__nv_bfloat16 *dst, const float (&v)[16]
 
 // bf16 pair -> fp16 pair (exact for |v| < 65504).
 __device__ __forceinline__ uint32_t bf2h(uint32_t v) {
-    return f2_to_h2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+    const float2 f = bf2_to_f2(v);
+    return f2_to_h2(f.x, f.y);
 }
 
 __device__ __forceinline__ uint4 cvt_chunk(uint4 r) {
