@@ -88,6 +88,7 @@ constexpr uint32_t OFF_BAR = OFF_PART + 64;        // 6 mbarriers
 constexpr uint32_t OFF_TM = OFF_BAR + 48;          // TMEM base address (4 B)
 constexpr uint32_t OFF_ABORT = OFF_TM + 4;         // CTA-wide abort flag (int)
 constexpr uint32_t OFF_RANGE = OFF_TM + 8;         // set when an output is not finite (int)
+constexpr uint32_t OFF_SEQ = OFF_TM + 12;          // sequence this CTA sweeps (packed varlen)
 constexpr uint32_t SMEM_BYTES = OFF_TM + 16;
 
 // TMEM columns (fp32 accumulators, lane = row).
@@ -103,6 +104,7 @@ constexpr uint32_t IDESC_YO2 = tc::idesc_f16_f32(128, 128, 0, 1); // C (K-major)
 constexpr uint32_t IDESC_Y = tc::idesc_f16_f32(128, 64, 0, 1);    // M (TMEM) x X (MN-major)
 
 constexpr float kSafeBlockDecay = 80.f;   // max exp argument taken by the factorised path
+constexpr int kLongestFirstSeqs = 64;     // packed batches up to this many sequences run longest first
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
@@ -571,6 +573,23 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
     } else {
         s = blockIdx.x / pairs;
         h0 = (blockIdx.x - s * pairs) * 2;
+        if (a.cu_seqlens && a.nseq <= kLongestFirstSeqs) {
+            // Packed sequences of mixed lengths: the CTAs take the sequences
+            // longest first (ties by index), so the long chains start in the
+            // first wave and the short ones fill in behind them.  Rank r of
+            // the order goes to CTAs [r pairs, (r + 1) pairs).
+            if (tid < a.nseq) {
+                const int len = __ldg(a.cu_seqlens + tid + 1) - __ldg(a.cu_seqlens + tid);
+                int rank = 0;
+                for (int q = 0; q < a.nseq; ++q) {
+                    const int lq = __ldg(a.cu_seqlens + q + 1) - __ldg(a.cu_seqlens + q);
+                    rank += (lq > len) || (lq == len && q < tid);
+                }
+                if (rank == s) flag_set(OFF_SEQ, tid);
+            }
+            __syncthreads();
+            s = flag_get(OFF_SEQ);
+        }
         if (a.cu_seqlens) {
             const int c0 = a.cu_seqlens[0], cs0 = a.cu_seqlens[s], cs1 = a.cu_seqlens[s + 1];
             const int cend = a.cu_seqlens[a.nseq];
