@@ -49,6 +49,8 @@ __host__ __device__ inline SimtSmem simt_smem(int Q, int P, int N)
     return s;
 }
 
+constexpr int kSimtLongestFirstSeqs = 64;   // packed batches up to this many sequences run longest first
+
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kSimtThreads)
 scan_simt_kernel(ScanArgs a)
@@ -62,10 +64,26 @@ scan_simt_kernel(ScanArgs a)
     float *Hs = smem + L.Hs, *Ms = smem + L.Ms;
     float *cs = smem + L.cs, *ex = smem + L.ex, *w = smem + L.w, *dts = smem + L.dts;
 
-    const int s = blockIdx.x / H;
+    const int tid = threadIdx.x;
+    int s = blockIdx.x / H;
     const int h = blockIdx.x - s * H;
     const int g = h / (H / G);
-    const int tid = threadIdx.x;
+    if (a.cu_seqlens && a.nseq <= kSimtLongestFirstSeqs) {
+        // Packed sequences of mixed lengths run longest first (ties by
+        // index): CTAs [r H, (r + 1) H) take the sequence of length rank r.
+        __shared__ int s_seq;
+        if (tid < a.nseq) {
+            const int len = __ldg(a.cu_seqlens + tid + 1) - __ldg(a.cu_seqlens + tid);
+            int rank = 0;
+            for (int q = 0; q < a.nseq; ++q) {
+                const int lq = __ldg(a.cu_seqlens + q + 1) - __ldg(a.cu_seqlens + q);
+                rank += (lq > len) || (lq == len && q < tid);
+            }
+            if (rank == s) s_seq = tid;
+        }
+        __syncthreads();
+        s = s_seq;
+    }
 
     long t0, t1;
     if (a.cu_seqlens) {
