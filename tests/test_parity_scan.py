@@ -113,3 +113,23 @@ def test_scan_large_dt_decays_to_zero(dt):
     inp.A[:] = -16.0
     ey, eh, _ = check(inp, y_dtype=torch.float32)
     assert ey < TOL and eh < TOL, (ey, eh)
+
+
+@pytest.mark.parametrize("nseq", [64, 65])   # longest-first order, and index order
+@pytest.mark.parametrize("dtype,P,N", [("bf16", 64, 128), ("f32", 32, 64)])
+def test_scan_packed_order_both_sides_of_cutoff(nseq, dtype, P, N):
+    """Packed batches of up to 64 sequences are swept longest first (each CTA
+    ranks the lengths), larger ones in index order.  Lengths with ties,
+    empty sequences and ragged tails, on the tensor-core and CUDA-core
+    kernels; every element against the oracle, empty sequences bit-exact."""
+    rng = np.random.default_rng(16 + nseq)
+    lens = [int(v) for v in rng.integers(0, 300, nseq)]
+    lens[3] = lens[7] = 0
+    lens[10] = lens[11] = lens[12] = 129
+    inp = synth.make_scan_inputs(17 + nseq, lens, 4, P, N, 2, dtype=dtype, init_state=True)
+    y, hT = scan_on_gpu(inp, y_dtype=torch.float32, varlen=True)
+    y_ref, h_ref = oracle_scan(inp)
+    assert rel_err(to_np(y), y_ref) < TOL
+    assert rel_err(to_np(hT), h_ref) < TOL
+    for s in (3, 7):
+        np.testing.assert_array_equal(to_np(hT)[s], inp.h0[s].astype(np.float64))
