@@ -162,7 +162,7 @@ def _dev(t, name, dtype=None):
 
 def ssd_chunk_scan(x, dt, A, B, C, D=None, initial_state=None, cu_seqlens=None,
                    chunk_size: int = 128, y=None, final_state=None, y_dtype=None,
-                   return_final_state: bool = True, status=None, stream=None, workspace=None):
+                   return_final_state: bool = True, status=None, stream=None, workspace="auto"):
     """Chunked SSD prefill scan.
 
     x  : [nseq, L, H, P] (fixed length) or [T, H, P] with ``cu_seqlens``
@@ -172,8 +172,10 @@ def ssd_chunk_scan(x, dt, A, B, C, D=None, initial_state=None, cu_seqlens=None,
     initial_state : [nseq, H, P, N] fp32 or None (zeros); may be ``final_state``
     cu_seqlens : int32 [nseq+1] CUDA tensor of packed offsets, or None
     y / final_state : optional preallocated outputs
-    workspace : optional CUDA tensor of at least ssd_chunk_scan_workspace_size(...) bytes
-        (fixed-length batches then run the balanced schedule)
+    workspace : CUDA tensor of at least ssd_chunk_scan_workspace_size(...) bytes (a
+        fixed-length batch then runs the balanced schedule), None for none, or
+        "auto" (the default): one is allocated through torch when these shapes
+        can use it
     Returns (y, final_state) -- final_state is None if not requested.
     """
     _dev(x, "x")
@@ -202,6 +204,13 @@ def ssd_chunk_scan(x, dt, A, B, C, D=None, initial_state=None, cu_seqlens=None,
         final_state = torch.empty((nseq, H, P, N), dtype=torch.float32, device=x.device)
     _dev(final_state, "final_state", torch.float32)
     _dev(status, "status", torch.int32)
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError('workspace must be a CUDA tensor, None or "auto"')
+        n = 0 if cu_seqlens is not None else ssd_chunk_scan_workspace_size(
+            nseq, seqlen, H, P, N, G, chunk_size)
+        workspace = torch.empty(n, dtype=torch.uint8, device=x.device) if n else None
+    _dev(workspace, "workspace")
     st = lib.ssd_chunk_scan(nseq, seqlen, _ptr(cu_seqlens), H, P, N, G, int(chunk_size),
                             in_code, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
                             _ptr(D), _ptr(initial_state), _dtype_code(y.dtype), _ptr(y),

@@ -70,3 +70,24 @@ def test_balanced_schedule_matches_oracle():
     yg = to_np(y).reshape(nseq * L, H, 64)[:, heads]
     assert rel_err(yg, y_ref) < TOL
     assert rel_err(to_np(hT)[:, heads], h_ref) < TOL
+
+
+def test_python_binding_allocates_the_workspace_by_default():
+    """Without a workspace argument the binding allocates one where the shapes
+    can use it; the result is bit-identical to passing one explicitly, and to
+    passing none (one CTA per chain)."""
+    from hybrid_mamba_ssm_b200 import ssm
+    nseq, L, H, G = 2, 8192, 160, 8
+    inp = synth.make_scan_inputs(421, [L] * nseq, H, 64, 128, G, dtype="bf16", init_state=True)
+    x = dev_tensor(inp.x).view(nseq, L, H, 64)
+    B = dev_tensor(inp.B).view(nseq, L, G, 128)
+    C = dev_tensor(inp.C).view(nseq, L, G, 128)
+    dt = dev_f32(inp.dt).view(nseq, L, H)
+    A, D, h0 = dev_f32(inp.A), dev_f32(inp.D), dev_f32(inp.h0)
+    y_auto, h_auto = ssm.ssd_chunk_scan(x, dt, A, B, C, D, h0)
+    y_none, h_none = ssm.ssd_chunk_scan(x, dt, A, B, C, D, h0, workspace=None)
+    torch.cuda.synchronize()
+    assert ssm.ssd_chunk_scan_workspace_size(nseq, L, H, 64, 128, G) > 0
+    assert torch.equal(y_auto, y_none) and torch.equal(h_auto, h_none)
+    with pytest.raises(ValueError):
+        ssm.ssd_chunk_scan(x, dt, A, B, C, D, h0, workspace="always")
