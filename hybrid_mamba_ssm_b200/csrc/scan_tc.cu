@@ -89,7 +89,8 @@ constexpr uint32_t OFF_TM = OFF_BAR + 48;          // TMEM base address (4 B)
 constexpr uint32_t OFF_ABORT = OFF_TM + 4;         // CTA-wide abort flag (int)
 constexpr uint32_t OFF_RANGE = OFF_TM + 8;         // set when an output is not finite (int)
 constexpr uint32_t OFF_SEQ = OFF_TM + 12;          // sequence this CTA sweeps (packed varlen)
-constexpr uint32_t SMEM_BYTES = OFF_TM + 16;
+constexpr uint32_t OFF_NXP = OFF_TM + 16;          // balanced: first chunk of the next piece (3 ints)
+constexpr uint32_t SMEM_BYTES = OFF_TM + 32;
 
 // TMEM columns (fp32 accumulators, lane = row).
 // G and Y share columns: the y MMAs write Y only after the mask has read G,
@@ -1008,9 +1009,19 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
             write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
             float3 dcur = decay_scan(a, hh, Ah, load_dt(a, H, hh, it.c0, it.t1, i), min(kQ, it.t1 - it.c0),
                                      i, wq, lane, wg, ch, sPART, sCSB, vd_tab + hd * 512, csb_tab + hd * 32);
-            // first chunk of the next piece (the chunk after this piece's last)
+            // The first chunk of the next piece (needed only at a piece's last
+            // chunk) is kept in shared memory, not in registers across the chunk
+            // loop: its first head, first token and sequence end.
             const int npieces = sw.cf == sw.cl ? 1 : sw.cl - sw.cf + 1;
-            Item nxp = npieces > 1 ? piece_item(a, sw, 1, pairs) : it;
+            auto publish_next = [&](int p) {
+                if (tid == 0) {
+                    const Item n = piece_item(a, sw, p, pairs);
+                    flag_set(OFF_NXP, 2 * n.pair);
+                    flag_set(OFF_NXP + 4, n.c0);
+                    flag_set(OFF_NXP + 8, n.t1);
+                }
+            };
+            if (npieces > 1) publish_next(1);
             tc::named_sync(BAR_COMPUTE, kCompute);
             uint32_t phase = 0, vb = 0;
             int q = 0;
@@ -1026,16 +1037,20 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                     const ChunkDecay cur = decay_derive(dcur, csb_tab + vb * 64 + hd * 32, wq, ch);
                     // the next chunk: in this piece, or the first of the next piece
                     const bool same = it.k + 1 < it.k1;
-                    const int hh_n = same ? hh : 2 * nxp.pair + hd;
-                    const int c0_n = same ? c0 + kQ : nxp.c0;
-                    const int t1_n = same ? it.t1 : nxp.t1;
+                    int hh_n = hh, c0_n = c0 + kQ, t1_n = it.t1;
+                    float Ah_n = Ah;
+                    if (!same && has_next) {
+                        hh_n = flag_get(OFF_NXP) + hd;
+                        c0_n = flag_get(OFF_NXP + 4);
+                        t1_n = flag_get(OFF_NXP + 8);
+                        Ah_n = a.A[hh_n];
+                    }
                     // its raw dt, a whole conversion ahead of its decay
                     const float dt_n1 = has_next ? load_dt(a, H, hh_n, c0_n, t1_n, i) : 0.f;
 
                     convert(phase, live, cur.w, q > 0);
 
                     // ---- next chunk's decay while the MMAs run ----
-                    const float Ah_n = same ? Ah : a.A[hh_n];
                     float3 dnxt = make_float3(0.f, 0.f, 0.f);
                     if (has_next)
                         dnxt = decay_scan(a, hh_n, Ah_n, dt_n1, min(kQ, t1_n - c0_n), i, wq, lane, wg, ch,
@@ -1060,13 +1075,16 @@ scan_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant_
                 it.c0 -= kQ;
                 store_piece_state(it);
                 if (pc_ + 1 < npieces) {
-                    it = nxp;
+                    it = piece_item(a, sw, pc_ + 1, pairs);
                     hh = 2 * it.pair + hd;
                     Ah = a.A[hh];
                     Dh = a.D ? a.D[hh] : 0.f;
                     load_piece_state(it);
                     write_state_half(sbase + OFF_H + hd * HALF, i, ch, Hs);
-                    if (pc_ + 2 < npieces) nxp = piece_item(a, sw, pc_ + 2, pairs);
+                    if (pc_ + 2 < npieces) publish_next(pc_ + 2);
+                    // (every thread has read the previous value: the last chunk's
+                    // state-update barrier lies between; this one publishes the new)
+                    tc::named_sync(BAR_COMPUTE, kCompute);
                 }
             }
         }
