@@ -217,7 +217,8 @@ def barrier(pg, device=None):
 # ---------------------------------------------------------------------------
 def oracle_step_sample(rank_seed, prefill_tokens, prefill_heads, decode_rows):
     """Time the oracle on a bounded sample of one step; returns (seconds for a
-    full step, description, threads)."""
+    full step, scaled from the sample, description, threads, seconds the
+    sample itself took)."""
     import oracle
     from hybrid_mamba_ssm_b200 import inputs as synth
     oracle.set_num_threads(os.cpu_count() or 1)
@@ -239,7 +240,7 @@ def oracle_step_sample(rank_seed, prefill_tokens, prefill_heads, decode_rows):
     step_s = t_pre * scale_pre + t_dec * scale_dec
     desc = (f"prefill {prefill_tokens} tokens x {prefill_heads} heads (of 16384 x 128) and "
             f"decode {decode_rows} of 64 batch rows x 256 heads, scaled to one full step")
-    return step_s, desc, oracle.num_threads()
+    return step_s, desc, oracle.num_threads(), t_pre + t_dec
 
 
 CONV_PREFILL = dict(nseq=4, seqlen=4096, dim=128 * 64 + 2 * 8 * 128, width=4)
@@ -677,15 +678,19 @@ def run_reference(args, world, rank, pg):
     tokens_per_step = PREFILL["nseq"] * PREFILL["seqlen"] + DECODE["batch"]
     for _ in range(args.warmup):
         oracle_step_sample(2000, 256, 4, 1)
-    total = 0.0
+    total = measured = 0.0
     desc = cores = None
     for k in range(args.steps):
-        s, desc, cores = oracle_step_sample(2000 + k, 256, 4, 1)
+        s, desc, cores, took = oracle_step_sample(2000 + k, 256, 4, 1)
         total += s
+        measured += took
     value = tokens_per_step * args.steps / total
+    # ms_per_step is what each (sample) step took on the host; the value is the
+    # full workload's tokens/s, the sample's time scaled to a whole step.
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "ms_per_step": 1e3 * measured / args.steps,
+            "full_step_ms_equivalent": 1e3 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
             "config": {"workload": "prefill 4x4096 H128 P64 N128 G8 Q128 + decode 64x256x64x128 G8",
@@ -935,7 +940,7 @@ def run_ours(args, world, rank, local, pg):
         line["mixed_varlen"] = {"prefill_tokens_per_s": r3(mixed["prefill"]["tokens_per_s"]),
                                 "decode_steps_per_s": r3(mixed["decode_steps_per_s"])}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        step_s, desc, cores = oracle_step_sample(3000, 1024, 8, 4)
+        step_s, desc, cores, _ = oracle_step_sample(3000, 1024, 8, 4)
         line["cpu_baseline"] = {"value": tok_step / step_s, "unit": "tokens/s", "cores": cores,
                                 "kind": "oracle", "sample": desc}
     if rank == 0:

@@ -86,3 +86,13 @@ def test_traffic_entry_requires_matching_source_hash(tmp_path, monkeypatch):
     # a kernel whose source changed since the capture reports no traffic
     monkeypatch.setattr(bench, "kernel_source_hash", lambda f: "0000000000000000")
     assert bench.measured_traffic("ssd_chunk_scan", "scan_tc.cu") is None
+
+
+def test_oracle_sample_reports_measured_and_scaled_time():
+    """The reference arm's step is a bounded sample: the sample's own time
+    (what ms_per_step reports) and its scaling to one full step (what the
+    tokens/s value uses) both come back, the second at least the first."""
+    import bench
+    step_s, desc, cores, took = bench.oracle_step_sample(5, 64, 2, 1)
+    assert 0 < took <= step_s
+    assert cores >= 1 and "scaled to one full step" in desc
