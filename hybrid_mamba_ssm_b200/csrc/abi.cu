@@ -590,6 +590,12 @@ int ssm_gated_rmsnorm(int rows, int dim, int group_size, int y_dtype, const void
 
 
 // ---------------------------------------------------------------- testing hooks
+int ssm_testing_balanced_runs(int nseq, int seqlen, int nheads, int sms)
+{
+    if (nseq <= 0 || seqlen <= 0 || nheads <= 0 || sms <= 0) return 0;
+    return ssm::scan_tc_balanced_runs_for(nseq, seqlen, nheads, sms);
+}
+
 int ssm_testing_scan_stalled(int nseq, int seqlen, int nheads, int ngroups,
                              const void *x, const float *dt, const float *A,
                              const void *B, const void *C, void *y,

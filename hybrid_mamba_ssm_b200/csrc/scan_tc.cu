@@ -1201,12 +1201,16 @@ bool scan_tc_supports(const ScanArgs &a)
 
 int scan_tc_balanced_runs(int nseq, int seqlen, int nheads)
 {
+    return scan_tc_balanced_runs_for(nseq, seqlen, nheads, sm_count());
+}
+
+int scan_tc_balanced_runs_for(int nseq, int seqlen, int nheads, int sms)
+{
     // One CTA per (sequence, head pair) chain leaves SMs idle when the chains
     // do not fill whole waves; cutting the chains into one run per SM fills
     // them.  A chain's chunks stay a sequential recurrence whichever runs
     // sweep them, so with no more chains than SMs (one wave, each chain its
     // own critical path) the cut gains nothing and is not used.
-    const int sms = sm_count();
     const long long chains = (long long)nseq * (nheads / 2);
     const long long nch = ((long long)seqlen + kQ - 1) / kQ;
     if (sms <= 0 || chains <= sms || nch <= 0) return 0;

@@ -150,6 +150,8 @@ cudaError_t launch_scan_tc(const ScanArgs &a, cudaStream_t stream);
 // these sizes on the current device (0: one CTA per chain), and the hand-off
 // workspace it needs.
 int scan_tc_balanced_runs(int nseq, int seqlen, int nheads);
+// The same decision for a device of `sms` SMs (pure host arithmetic).
+int scan_tc_balanced_runs_for(int nseq, int seqlen, int nheads, int sms);
 size_t scan_tc_handoff_bytes(int runs);
 
 }  // namespace ssm

@@ -20,6 +20,10 @@
  * they write are meaningless.  The operation itself has no counterpart in
  * the pages the library follows: it exists to exercise the timeout path
  * without faulting or hanging a GPU.
+ *
+ * ssm_testing_balanced_runs exposes, for host-only tests, the rule by which
+ * ssd_chunk_scan_workspace_size decides whether a fixed-length batch gets
+ * the balanced schedule, for a device of a given SM count.
  */
 #ifndef LIBSSM_SSM_TESTING_H
 #define LIBSSM_SSM_TESTING_H
@@ -56,6 +60,16 @@ SSM_API int ssm_testing_scan_stalled(int nseq, int seqlen, int nheads, int ngrou
  * [dim][width] (width 1..8), no conv state, no bias, no activation.
  * wait_ns and status_dev as above.
  */
+/*
+ * ssm_testing_balanced_runs -- the number of runs (one per SM) into which
+ * ssd_chunk_scan cuts the (sequence, head pair) chains of a fixed-length
+ * batch of nseq sequences of seqlen tokens and nheads heads on a device of
+ * `sms` SMs, or 0 when it keeps one CTA per chain: with no more chains than
+ * SMs, or when the last wave of chains fills at least nine tenths of the
+ * SMs.  Host arithmetic only; no device is used.
+ */
+SSM_API int ssm_testing_balanced_runs(int nseq, int seqlen, int nheads, int sms);
+
 SSM_API int ssm_testing_conv1d_stalled(int nseq, int seqlen, int dim, int width,
                                        const void *x, const float *weight, void *y,
                                        unsigned long long wait_ns, int *status_dev,

@@ -414,3 +414,22 @@ def test_testing_hooks_validate_on_the_host(lib):
                                           None) == INVALID            # width
     assert lib.ssm_testing_conv1d_stalled(1, 64, 128, 4, A16, A16b, A16c, 10**6, None,
                                           None) == INVALID            # no status word
+
+
+def test_balanced_schedule_rule(lib):
+    """When a fixed-length batch is cut into one run per SM (host arithmetic,
+    for a device of a given SM count): more chains than SMs, and a last wave
+    of chains less than nine tenths full; one run per SM."""
+    f = lib.ssm_testing_balanced_runs
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 4
+    assert f(4, 4096, 128, 148) == 148       # 256 chains: a second wave 108 wide
+    assert f(2, 8192, 160, 148) == 148       # 160 chains
+    assert f(1, 32768, 256, 148) == 0        # 128 chains: one wave, each its own critical path
+    assert f(9, 1024, 32, 148) == 0          # 144 chains
+    assert f(37, 1024, 16, 148) == 0         # 296 chains: two whole waves
+    assert f(266, 512, 2, 148) == 148        # last wave 118 of 148 (< 9/10)
+    assert f(267, 512, 2, 148) == 0          # last wave 119 of 148 (>= 9/10)
+    assert f(4, 4096, 128, 132) == 0         # 132 SMs: last wave 124 of 132 (>= 9/10)
+    assert f(4, 4096, 128, 160) == 160       # 160 SMs: last wave 96 of 160
+    assert f(0, 4096, 128, 148) == 0 and f(4, 0, 128, 148) == 0 and f(4, 4096, 128, 0) == 0
