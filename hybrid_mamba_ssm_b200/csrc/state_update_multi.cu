@@ -201,8 +201,11 @@ state_update_multi_kernel(MultiUpdateArgs a)
 // arithmetic per state element drops from ~3 operations per token to 1.
 constexpr int kVerifyMaxTok = 8;
 
-template <typename TIn, typename TOut>
-__global__ void __launch_bounds__(kMultiWarps * 32, 4)
+// Tokens padded to a power of two, for the joint reduction of y.
+constexpr int verify_pad(int nt) { return nt <= 1 ? 1 : nt <= 2 ? 2 : nt <= 4 ? 4 : 8; }
+
+template <typename TIn, typename TOut, int NT>
+__global__ void __launch_bounds__(kMultiWarps * 32, (NT <= 2 ? 4 : NT <= 4 ? 3 : 2))
 state_verify_kernel(MultiUpdateArgs a)
 {
     constexpr int N = 128;
@@ -210,7 +213,8 @@ state_verify_kernel(MultiUpdateArgs a)
     __shared__ float sX[kVerifyMaxTok][64], sDt[kVerifyMaxTok], sCs[kVerifyMaxTok];
     __shared__ float sL[kVerifyMaxTok][kVerifyMaxTok];
 
-    const int H = a.nheads, P = a.head_dim, nt = a.ntok;
+    constexpr int nt = NT;   // draft tokens (a.ntok)
+    const int H = a.nheads, P = a.head_dim;
     const int bh = blockIdx.x;
     const int b = bh / H;
     const int h = bh - b * H;
@@ -280,37 +284,56 @@ state_verify_kernel(MultiUpdateArgs a)
     }
     __syncthreads();
 
-    for (int t = 0; t < nt; ++t) {
-        const float4 c4 = *reinterpret_cast<const float4 *>(&sC[t][lane * 4]);
-        float part[kMultiUnroll];
+    // y of every token at once: this lane's partial dot products of its 8
+    // rows with each C_t (index k NP + t), then one transpose-reduction over
+    // all (row, token) pairs: each level keeps half of the values (the upper
+    // half in the lanes whose bit `off` is set) and adds the partner's other
+    // half, so the tokens share 5 dependent shuffle rounds instead of 5 each.
+    constexpr int NP = verify_pad(NT);
+    constexpr int M = kMultiUnroll * NP;                       // values per lane
+    constexpr int LEVELS = M >= 32 ? 5 : (M == 16 ? 4 : 3);    // lane bits folded with halving
+    float part[M];
+#pragma unroll
+    for (int t = 0; t < NP; ++t) {
+        const float4 c4 = t < NT ? *reinterpret_cast<const float4 *>(&sC[t][lane * 4])
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < kMultiUnroll; ++k) {
             const float2 d2 = __ffma2_rn(make_float2(s[k].x, s[k].y), make_float2(c4.x, c4.y),
                                          __fmul2_rn(make_float2(s[k].z, s[k].w), make_float2(c4.z, c4.w)));
-            part[k] = d2.x + d2.y;
+            part[k * NP + t] = d2.x + d2.y;
         }
-        // transpose-reduce: offsets 16, 8, 4 halve the rows held per lane,
-        // offsets 2, 1 finish; lane bits 4..2 name the row
+    }
 #pragma unroll
-        for (int lvl = 0; lvl < 3; ++lvl) {
-            const int half = 4 >> lvl, off = 16 >> lvl;
-            const bool upper = lane & off;
+    for (int lvl = 0; lvl < LEVELS; ++lvl) {
+        const int half = M >> (lvl + 1), off = 16 >> lvl;
+        const bool upper = lane & off;
 #pragma unroll
-            for (int i = 0; i < half; ++i) {
-                const float send = upper ? part[i] : part[i + half];
-                const float keep = upper ? part[i + half] : part[i];
-                part[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        for (int i = 0; i < half; ++i) {
+            const float send = upper ? part[i] : part[i + half];
+            const float keep = upper ? part[i + half] : part[i];
+            part[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+    // the lane bits not folded: a plain butterfly over the one value left
+#pragma unroll
+    for (int off = (1 << (5 - LEVELS)) >> 1; off > 0; off >>= 1)
+        part[0] += __shfl_xor_sync(0xffffffffu, part[0], off);
+    // Lane L now holds the values of index (L >> (5 - LEVELS)) * V + j,
+    // j < V = M >> LEVELS (its folded lane bits name the halves it kept);
+    // lanes that share those bits hold the same values, and the first writes.
+    constexpr int V = M >> LEVELS;
+    if ((lane & ((1 << (5 - LEVELS)) - 1)) == 0) {
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const int idx = (lane >> (5 - LEVELS)) * V + j;
+            const int k = idx / NP, t = idx - k * NP;
+            const int r = k * kMultiWarps + warp;
+            if (t < NT && r < P) {
+                float v = expf(sCs[t]) * part[j] + Dh * sX[t][r];
+                for (int q = 0; q <= t; ++q) v = fmaf(sL[t][q], sX[q][r], v);
+                store_out(y + (((size_t)b * nt + t) * H + h) * P + r, v);
             }
-        }
-        float acc = part[0];
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        const int k = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-        const int r = k * kMultiWarps + warp;
-        if ((lane & 3) == 0 && r < P) {
-            float v = expf(sCs[t]) * acc + Dh * sX[t][r];
-            for (int j = 0; j <= t; ++j) v = fmaf(sL[t][j], sX[j][r], v);
-            store_out(y + (((size_t)b * nt + t) * H + h) * P + r, v);
         }
     }
 }
@@ -350,8 +373,18 @@ template <int N, typename TIn, typename TOut>
 static cudaError_t launch_multi_t(const MultiUpdateArgs &a, cudaStream_t stream)
 {
     const unsigned grid = (unsigned)((size_t)a.batch * a.nheads);
-    if (N == 128 && a.head_dim <= 64 && a.ntok <= kVerifyMaxTok && !a.inter && !a.accept_len && a.y) {
-        state_verify_kernel<TIn, TOut><<<grid, kMultiWarps * 32, 0, stream>>>(a);
+    if (N == 128 && a.head_dim <= 64 && a.ntok >= 1 && a.ntok <= kVerifyMaxTok && !a.inter &&
+        !a.accept_len && a.y) {
+        switch (a.ntok) {
+        case 1: state_verify_kernel<TIn, TOut, 1><<<grid, kMultiWarps * 32, 0, stream>>>(a); break;
+        case 2: state_verify_kernel<TIn, TOut, 2><<<grid, kMultiWarps * 32, 0, stream>>>(a); break;
+        case 3: state_verify_kernel<TIn, TOut, 3><<<grid, kMultiWarps * 32, 0, stream>>>(a); break;
+        case 4: state_verify_kernel<TIn, TOut, 4><<<grid, kMultiWarps * 32, 0, stream>>>(a); break;
+        case 5: state_verify_kernel<TIn, TOut, 5><<<grid, kMultiWarps * 32, 0, stream>>>(a); break;
+        case 6: state_verify_kernel<TIn, TOut, 6><<<grid, kMultiWarps * 32, 0, stream>>>(a); break;
+        case 7: state_verify_kernel<TIn, TOut, 7><<<grid, kMultiWarps * 32, 0, stream>>>(a); break;
+        default: state_verify_kernel<TIn, TOut, 8><<<grid, kMultiWarps * 32, 0, stream>>>(a); break;
+        }
         return cudaGetLastError();
     }
     state_update_multi_kernel<N, TIn, TOut><<<grid, kMultiWarps * 32, 0, stream>>>(a);
