@@ -532,7 +532,12 @@ conv1d_update_kernel(ConvArgs a)
 }
 
 // Vectorised decode for dim % V == 0: V adjacent channels per thread, whose
-// state windows are (K-1) consecutive 16-byte vectors of the state row.
+// state windows are (K-1) consecutive 16-byte vectors of the state row.  A
+// thread serves kUpdateRows batch rows of its channels: the loads of all of
+// them go out first, and the weights and bias (the same for every row) are
+// loaded once for them.
+constexpr int kUpdateRows = 2;
+
 template <typename TIn, typename TOut, int K>
 __global__ void __launch_bounds__(kVecThreads)
 conv1d_update_vec_kernel(ConvArgs a)
@@ -541,30 +546,38 @@ conv1d_update_vec_kernel(ConvArgs a)
     constexpr int W = K > 1 ? K - 1 : 1;
     using Raw = typename ConvVec<TIn>::Raw;
     const int c0 = (blockIdx.y * kVecThreads + threadIdx.x) * V;
-    const int b = blockIdx.x;
     const int dim = a.dim;
     if (c0 >= dim) return;
-    long row = b;
-    if (a.slot_idx) {
-        const int slot = __ldg(a.slot_idx + b);
-        if (slot < 0) return;                   // padding row
-        if (slot >= a.max_slots) {
-            if (c0 == 0) report_status(a.status_dev, 6);
-            return;
+    const TIn *x = static_cast<const TIn *>(a.x);
+    // the rows' state rows (-1: nothing to do), commit counts, state windows
+    // and first tokens, all requested before any arithmetic
+    long rows[kUpdateRows];
+    int commits[kUpdateRows];
+    Raw raw[kUpdateRows][W], x0[kUpdateRows];
+#pragma unroll
+    for (int j = 0; j < kUpdateRows; ++j) {
+        const int b = blockIdx.x * kUpdateRows + j;
+        rows[j] = -1;
+        commits[j] = 0;
+        if (b >= a.nseq) continue;
+        long row = b;
+        if (a.slot_idx) {
+            const int slot = __ldg(a.slot_idx + b);
+            if (slot < 0) continue;                 // padding row
+            if (slot >= a.max_slots) {
+                if (c0 == 0) report_status(a.status_dev, 6);
+                continue;
+            }
+            row = slot;
         }
-        row = slot;
-    }
-    const int commit = conv_commit_count(a, b);
-    if (commit < 0) return;
-    // state of channels c0..c0+V-1: V*(K-1) values, channel-major
-    TIn *st = static_cast<TIn *>(a.state) + ((size_t)row * dim + c0) * (K - 1);
-    float win[W][V];   // win[j][v]: channel c0+v, window slot j (oldest first)
+        const int commit = conv_commit_count(a, b);
+        if (commit < 0) continue;
+        rows[j] = row;
+        commits[j] = commit;
+        const TIn *st = static_cast<const TIn *>(a.state) + ((size_t)row * dim + c0) * (K - 1);
 #pragma unroll
-    for (int i = 0; i < K - 1; ++i) {
-        float f[V];
-        unpack_row(*reinterpret_cast<const Raw *>(st + (size_t)i * V), f);
-#pragma unroll
-        for (int e = 0; e < V; ++e) win[(i * V + e) % W][(i * V + e) / W] = f[e];
+        for (int i = 0; i < K - 1; ++i) raw[j][i] = *reinterpret_cast<const Raw *>(st + (size_t)i * V);
+        if (a.ntok > 0) x0[j] = load_row(x + (size_t)b * a.ntok * dim + c0);
     }
     float w[V * K], bias[V];
 #pragma unroll
@@ -574,33 +587,49 @@ conv1d_update_vec_kernel(ConvArgs a)
     }
 #pragma unroll
     for (int v = 0; v < V; ++v) bias[v] = a.bias ? __ldg(a.bias + c0 + v) : 0.f;
-    for (int t = 0; t < a.ntok; ++t) {
-        const size_t xi = ((size_t)b * a.ntok + t) * dim + c0;
-        float cur[V], out[V];
-        unpack_row(load_row(static_cast<const TIn *>(a.x) + xi), cur);
 #pragma unroll
-        for (int v = 0; v < V; ++v) {
-            float acc = bias[v];
+    for (int j = 0; j < kUpdateRows; ++j) {
+        if (rows[j] < 0) continue;
+        const int b = blockIdx.x * kUpdateRows + j;
+        const int commit = commits[j];
+        // state of channels c0..c0+V-1: V*(K-1) values, channel-major
+        TIn *st = static_cast<TIn *>(a.state) + ((size_t)rows[j] * dim + c0) * (K - 1);
+        float win[W][V];   // win[i][v]: channel c0+v, window slot i (oldest first)
 #pragma unroll
-            for (int j = 0; j < K - 1; ++j) acc = fmaf(w[v * K + j], win[j][v], acc);
-            acc = fmaf(w[v * K + K - 1], cur[v], acc);
-            out[v] = conv_act(acc, a.activation);
+        for (int i = 0; i < K - 1; ++i) {
+            float f[V];
+            unpack_row(raw[j][i], f);
+#pragma unroll
+            for (int e = 0; e < V; ++e) win[(i * V + e) % W][(i * V + e) / W] = f[e];
         }
-        if (a.y) store_row<V>(static_cast<TOut *>(a.y) + xi, out);
+        for (int t = 0; t < a.ntok; ++t) {
+            const size_t xi = ((size_t)b * a.ntok + t) * dim + c0;
+            float cur[V], out[V];
+            unpack_row(t == 0 ? x0[j] : load_row(x + xi), cur);
 #pragma unroll
-        for (int j = 0; j < K - 2; ++j)
+            for (int v = 0; v < V; ++v) {
+                float acc = bias[v];
 #pragma unroll
-            for (int v = 0; v < V; ++v) win[j][v] = win[j + 1][v];
-        if (K > 1)
+                for (int i = 0; i < K - 1; ++i) acc = fmaf(w[v * K + i], win[i][v], acc);
+                acc = fmaf(w[v * K + K - 1], cur[v], acc);
+                out[v] = conv_act(acc, a.activation);
+            }
+            if (a.y) store_row<V>(static_cast<TOut *>(a.y) + xi, out);
 #pragma unroll
-            for (int v = 0; v < V; ++v) win[W - 1][v] = cur[v];
-        if (t + 1 == commit) {
+            for (int i = 0; i < K - 2; ++i)
 #pragma unroll
-            for (int i = 0; i < K - 1; ++i) {
-                float f[V];
+                for (int v = 0; v < V; ++v) win[i][v] = win[i + 1][v];
+            if (K > 1)
 #pragma unroll
-                for (int e = 0; e < V; ++e) f[e] = win[(i * V + e) % W][(i * V + e) / W];
-                store_row<V>(st + (size_t)i * V, f);
+                for (int v = 0; v < V; ++v) win[W - 1][v] = cur[v];
+            if (t + 1 == commit) {
+#pragma unroll
+                for (int i = 0; i < K - 1; ++i) {
+                    float f[V];
+#pragma unroll
+                    for (int e = 0; e < V; ++e) f[e] = win[(i * V + e) % W][(i * V + e) / W];
+                    store_row<V>(st + (size_t)i * V, f);
+                }
             }
         }
     }
@@ -651,7 +680,8 @@ static cudaError_t launch_conv_t(const ConvArgs &a, cudaStream_t stream)
     constexpr int V = ConvVec<TIn>::V;
     if (a.update) {
         if (a.dim % V == 0) {
-            const dim3 grid((unsigned)a.nseq, (unsigned)((a.dim / V + kVecThreads - 1) / kVecThreads));
+            const dim3 grid((unsigned)((a.nseq + kUpdateRows - 1) / kUpdateRows),
+                            (unsigned)((a.dim / V + kVecThreads - 1) / kVecThreads));
             switch (a.width) {
             case 1: conv1d_update_vec_kernel<TIn, TOut, 1><<<grid, kVecThreads, 0, stream>>>(a); break;
             case 2: conv1d_update_vec_kernel<TIn, TOut, 2><<<grid, kVecThreads, 0, stream>>>(a); break;
